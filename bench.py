@@ -1,0 +1,423 @@
+"""Benchmark of the retrieve-and-inject path on B200.
+
+Workload (default): Llama-3.1-8B shapes (32 layers, 8 KV heads, head_dim 128,
+theta 5e5 with llama3 scaling), a fact store of 10 000 facts with lengths
+uniform in 16..64 tokens (~52 GB of bf16 K+V), and one batch of 100 requests,
+each injecting k=50 distinct facts after a 64-token prefix into its own
+shuffled 256-block table of a 25 600-block paged cache (block size 16).
+
+One step = one whole batch through the path: segment composition (plan
+kernel) + gather, RoPE re-rotation and paged scatter of K and V for every
+layer and KV head (inject kernel).  Inputs are synthetic and seeded; the
+26 GB read and 26 GB written per step are far larger than the 126 MB L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank is an independent replica
+with its own store and batch (requests are independent; no collective on the
+data path), so the scaling is weak and the value is the sum over ranks of
+tokens divided by the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (the plain fp64 C definition of the
+path) on the host cores, on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+sys.path.insert(0, os.path.join(ROOT, "tests"))
+
+METRIC = "injected KV tokens/s and achieved HBM GB/s (vs ~8 TB/s); per-batch inject µs"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["kv_cache_injection_gather_b200/csrc/inject_kernels.cuh",
+                  "kv_cache_injection_gather_b200/csrc/inject_store.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(bytes_per_token_algo: float):
+    """DRAM bytes per injected token of the inject kernel from the committed
+    ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "inject_kernel_traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except Exception:
+        return None, None
+    if rec.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None, rec
+    return float(rec["dram_bytes_per_token"]), rec
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(wl, requests, device=None):
+    """Host arrays for the oracle on a subset of requests: the facts those
+    requests use (regenerated by the seeded generator) and a compact cache
+    holding only their blocks."""
+    import oracle
+    import synth
+    m, b = wl.model, wl.batch
+    L, H, D = m.num_layers, m.num_kv_heads, m.head_dim
+    used = np.unique(np.concatenate([b.fact_ids[b.req_offsets[r]:b.req_offsets[r + 1]]
+                                     for r in requests]))
+    remap = {int(f): i for i, f in enumerate(used)}
+    st = oracle.Store(L, H, D, int(wl.fact_lens[used].sum()), len(used))
+    gen = None
+    if device is not None:
+        import torch
+        gen = torch.empty(L * H * int(wl.fact_lens.max()) * D, dtype=torch.int16,
+                          device=f"cuda:{device}")
+    for f in used:
+        n = int(wl.fact_lens[f])
+        if gen is None:
+            k, v = synth.fact_kv(wl.seed, int(f), L, H, n, D)
+        else:  # the generator's device implementation (same definition, faster)
+            cnt = L * H * n * D
+            cs = 0
+            synth.fill_device(gen.data_ptr(), cnt, wl.seed, synth.fact_stream(int(f), False), 0, cs)
+            k = gen[:cnt].cpu().numpy().view(np.uint16).reshape(L, H, n, D)
+            synth.fill_device(gen.data_ptr(), cnt, wl.seed, synth.fact_stream(int(f), True), 0, cs)
+            v = gen[:cnt].cpu().numpy().view(np.uint16).reshape(L, H, n, D)
+        st.put(k, v)
+    ids, offs, bts = [], [0], []
+    for i, r in enumerate(requests):
+        seg = b.fact_ids[b.req_offsets[r]:b.req_offsets[r + 1]]
+        ids.extend(remap[int(f)] for f in seg)
+        offs.append(len(ids))
+        bts.append(np.arange(i * b.max_blocks, (i + 1) * b.max_blocks, dtype=np.int32))
+    nb = len(requests) * b.max_blocks
+    shape = (L, nb, b.block_size, H, D)
+    kc = np.zeros(shape, np.uint16)
+    vc = np.zeros(shape, np.uint16)
+    inv = oracle.rope_inv_freq(D, m.rope_theta, m.scaling())
+    args = (st, inv, np.array(offs, np.int32), np.array(ids, np.int32),
+            b.start_pos[list(requests)], np.stack(bts), kc, vc, b.block_size)
+    tokens = sum(int(wl.fact_lens[b.fact_ids[b.req_offsets[r]:b.req_offsets[r + 1]]].sum())
+                 for r in requests)
+    return args, tokens
+
+
+def time_oracle(args, threads: int) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    rc, _ = oracle.inject_batch(*args, num_threads=threads)
+    dt = time.perf_counter() - t0
+    if rc != oracle.OK:
+        raise RuntimeError(f"oracle status {rc}")
+    return dt
+
+
+def cpu_baseline(wl, device, budget_s=15.0):
+    """The oracle as it stands, on the host cores, on a bounded sample."""
+    import oracle
+    threads = oracle.max_threads()
+    args, tok = oracle_sample(wl, [0], device)
+    dt = time_oracle(args, threads)
+    n_req = int(max(1, min(wl.batch.num_requests, budget_s / max(dt, 1e-3))))
+    if n_req > 1:
+        del args
+        args, tok = oracle_sample(wl, list(range(n_req)), device)
+        dt = time_oracle(args, threads)
+    return {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {n_req} of {wl.batch.num_requests} requests ({tok} tokens, all "
+                      f"{wl.model.num_layers} layers x {wl.model.num_kv_heads} KV heads), "
+                      f"{dt:.2f} s"}
+
+
+# ------------------------------------------------------------------ main
+
+def workload_config(wl, extra=None):
+    m, b = wl.model, wl.batch
+    cfg = {"workload": "llama3.1-8b-shapes 10k-fact store, 100 requests x k=50, block 16, "
+                       "cache 25600 blocks",
+           "model_shapes": m.name, "layers": m.num_layers, "kv_heads": m.num_kv_heads,
+           "head_dim": m.head_dim, "rope": "theta 5e5, llama3 scaling (8, 1, 4, 8192)",
+           "requests": b.num_requests, "k": int(b.req_offsets[1] - b.req_offsets[0]),
+           "facts": len(wl.fact_lens), "fact_len": "uniform 16..64",
+           "tokens_per_batch": wl.tokens(), "block_size": b.block_size,
+           "num_blocks": b.num_blocks, "start_pos": 64,
+           "l2": "inputs larger than L2 (26 GB read + 26 GB written per step)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def run_reference(args, rank, world):
+    import synth
+    if rank != 0:
+        return 0
+    wl = synth.llama_batch(0)
+    sample_args, tok = oracle_sample(wl, [0], None if not _cuda() else 0)
+    import oracle
+    threads = oracle.max_threads()
+    for _ in range(args.warmup):
+        time_oracle(sample_args, threads)
+    times = [time_oracle(sample_args, threads) for _ in range(args.steps)]
+    total = sum(times)
+    value = tok * args.steps / total
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, {"reference_step": "request 0 of the batch"}),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"request 0 of the batch ({tok} tokens, all layers and "
+                                       f"heads) per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _cuda():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from gpu_common import batch_tensors, make_cache, make_store
+    from kv_cache_injection_gather_b200 import binding as B
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the inject path has no CPU fallback)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synth.llama_batch(seed=rank)
+    m, b = wl.model, wl.batch
+    store = make_store(wl, on_device_gen=True, device=local_rank)
+    kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False)
+    ro, ids, sp, bt = batch_tensors(b, local_rank)
+    n_tok = wl.tokens()
+    slots = torch.empty(n_tok, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        store.inject(ro, ids, sp, bt, desc, slots, stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        step()
+    rc, _ = store.last_error()
+    if rc != 0:
+        raise RuntimeError(f"inject failed during warm-up: {B.status_string(rc)}")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local_rank)
+    clocks = ClockSampler(gpu_id)
+    # ---- device-resident timed region
+    store.set_timing(True)
+    store.kernel_time()  # reset
+    barrier()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    kern_ms, kern_n = store.kernel_time()
+    store.set_timing(False)
+    rc, _ = store.last_error()
+    if rc != 0:
+        raise RuntimeError(f"inject failed: {B.status_string(rc)}")
+
+    # ---- end to end through the host entry point: index arrays from pinned
+    # host memory in, slot mapping and status back to pinned host memory
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
+    h_ro, h_ids, h_sp, h_bt = pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos), pin(b.block_tables)
+    h_slots = torch.empty(n_tok, dtype=torch.int64).pin_memory()
+    h2d = sum(t.numel() * 4 for t in (h_ro, h_ids, h_sp, h_bt))
+    d2h = n_tok * 8 + 16
+    for _ in range(max(1, args.warmup // 2)):
+        store.inject_host(h_ro, h_ids, h_sp, h_bt, desc, h_slots, stream.cuda_stream)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        rc = store.inject_host(h_ro, h_ids, h_sp, h_bt, desc, h_slots, stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(f"inject_host failed: {B.status_string(rc)}")
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    # ---- max over ranks
+    vals = torch.tensor([ms, e2e_ms, kern_ms / max(kern_n, 1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, kern_avg_ms = vals.tolist()
+    ms_step = ms / args.steps
+    tokens_all = n_tok * world
+    value = tokens_all / (ms_step / 1e3)
+    algo_bytes = n_tok * 2 * m.bytes_per_token   # read K+V + write K+V
+    peak, peak_kind = hbm_peak()
+    achieved = algo_bytes / (kern_avg_ms / 1e3) / 1e9
+    traffic_pt, rec = recorded_traffic(2 * m.bytes_per_token)
+    baseline = cpu_baseline(wl, local_rank) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if rank != 0:
+        store.close()
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(wl, {"parallelism": f"replicas x{world}"}),
+        "us_per_batch": ms_step * 1e3,
+        "gbs_per_gpu": algo_bytes / (ms_step / 1e3) / 1e9,
+        "kernel_us": kern_avg_ms * 1e3,
+        "clocks": clk,
+        "e2e": {"value": tokens_all / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": None if traffic_pt is None else traffic_pt * n_tok,
+                     "algorithmic_bytes": algo_bytes,
+                     "kernel": "inject_kernel (plan_kernel excluded)"},
+        "cpu_baseline": baseline,
+    }
+    print(json.dumps(line), flush=True)
+    store.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    try:
+        if args.impl == "reference":
+            rc = run_reference(args, rank, world)
+        else:
+            rc = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

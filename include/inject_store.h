@@ -1,0 +1,219 @@
+/*
+ * inject_store.h -- C-ABI of the B200 retrieve-and-inject library
+ * (libinjectstore.so).
+ *
+ * What it computes follows the online phase of InferScale ("InferScale:
+ * GPU-Native KV Injection for Personalized LLM Serving", summaries at
+ * gist.science/{ja,nl,it}/paper/2607.27090, technical summary, section
+ * "Methodology -- 2. Online phase: Chunked RoPE and KV injection"):
+ *
+ *   Pre-RoPE storage   keys are captured before RoPE and kept, with the raw
+ *                      values, in a fact store on the GPU;
+ *   Dynamic rotation   the retrieved facts are composed into one contiguous
+ *                      segment and each stored key gets the RoPE rotation of
+ *                      its new serving position (Theorem 6: exact);
+ *   Injection          the composed K/V are scatter-copied into the paged KV
+ *                      cache, so the model prefills only the query tokens.
+ *
+ * Conventions for every call:
+ *   - All functions return IS_OK (0) or a negative IS_ERR_* status and never
+ *     abort the process.  Device-side problems found while a batch runs are
+ *     recorded on the device and returned by is_last_error().
+ *   - Tensors are bf16 (IEEE binary32 upper halves) passed as void*; integer
+ *     arrays are int32 or int64 as declared.  "device" pointers must be
+ *     addresses on the store's GPU; "host or device" pointers may be either
+ *     (unified addressing decides).  No call takes ownership of a caller
+ *     array; every array must stay valid until the work on `stream` that
+ *     uses it has finished.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *   - One store must not be used by two batches at the same time: batches on
+ *     one store are ordered on one stream, or ordered by the caller.
+ *   - Thread safety: a store is not internally locked.
+ */
+#ifndef INJECT_STORE_H
+#define INJECT_STORE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define IS_OK 0
+#define IS_ERR_INVALID_ARG (-1)   /* bad pointer, size, geometry or CSR     */
+#define IS_ERR_BAD_FACT_ID (-2)   /* a fact id outside [0, num_facts)       */
+#define IS_ERR_POSITION (-3)      /* segment runs past the request's table  */
+#define IS_ERR_BAD_BLOCK (-4)     /* block-table entry outside the cache    */
+#define IS_ERR_CAPACITY (-5)      /* store, batch or slot-output too small  */
+#define IS_ERR_OOM (-6)           /* device or pinned allocation failed     */
+#define IS_ERR_CUDA (-7)          /* a CUDA runtime call failed             */
+#define IS_ERR_TIMEOUT (-8)       /* a bounded host wait ran out            */
+#define IS_ERR_NOT_SUPPORTED (-9) /* shape outside what the kernels handle  */
+
+/* ---- configuration ----------------------------------------------------- */
+#define IS_ROPE_ROTATE_HALF 0   /* pairs (i, i + D/2): Llama/Mistral/Qwen HF  */
+#define IS_ROPE_INTERLEAVED 1   /* pairs (2i, 2i + 1)                         */
+#define IS_SCALING_NONE 0
+#define IS_SCALING_LLAMA3 1     /* Llama-3.1 wavelength-band frequency rule   */
+#define IS_TIER_DEVICE 0        /* whole store in HBM                         */
+#define IS_TIER_HOST 1          /* store in pinned host memory + HBM hot set  */
+
+typedef struct {
+  int32_t num_layers;        /* L >= 1                                        */
+  int32_t num_kv_heads;      /* H >= 1                                        */
+  int32_t head_dim;          /* D in {32, 64, 128, 256}                       */
+  int32_t rope_style;        /* IS_ROPE_*                                     */
+  double rope_theta;         /* base theta > 0; inv_freq_i = theta^(-2i/D)    */
+  int32_t rope_scaling;      /* IS_SCALING_*                                  */
+  double scale_factor;       /* llama3: factor (8)                            */
+  double low_freq_factor;    /* llama3: low (1)                               */
+  double high_freq_factor;   /* llama3: high (4)                              */
+  int32_t original_max_position; /* llama3: original context (8192)          */
+  int64_t capacity_tokens;   /* tokens per (layer, head) plane of the store   */
+  int32_t max_facts;         /* fact-id capacity                              */
+  int32_t max_batch_requests;/* per-batch request limit (0: 4096)             */
+  int32_t max_batch_fact_ids;/* per-batch fact-id limit (0: 1 << 20)          */
+  int32_t max_batch_blocks;  /* per-batch touched cache blocks over all
+                                requests (0: max(65536, 256 * requests))     */
+  int32_t tier;              /* IS_TIER_*                                     */
+  int64_t hot_capacity_tokens; /* IS_TIER_HOST: tokens of the HBM hot set     */
+} is_store_config_t;
+
+/* Paged KV cache.  Element (layer l, block b, in-block token o, head h,
+ * dim d) of K is ((uint16_t*)k_cache)[l*layer_stride + b*block_stride +
+ * o*token_stride + h*head_stride + d]; V alike with the same strides.
+ * Strides are in elements and multiples of 8; caches 16-byte aligned.
+ * [L][num_blocks][B][H][D] (token-major) and [L][num_blocks][H][B][D]
+ * (head-major) are both expressible.  Slot s = b*B + o. */
+typedef struct {
+  void* k_cache;
+  void* v_cache;
+  int64_t layer_stride;
+  int64_t block_stride;
+  int64_t token_stride;
+  int64_t head_stride;
+  int32_t num_blocks;
+  int32_t block_size;        /* B in [1, 128]                                 */
+} is_cache_t;
+
+typedef struct is_store is_store_t;  /* opaque; owned by the library */
+
+/* ---- store lifetime ---------------------------------------------------- */
+
+/* Create a fact store on `device`.  Pre-RoPE storage (technical summary,
+ * Online phase, "Pre-RoPE storage"): K and V arenas, bf16, layout
+ * [L][H][capacity_tokens][D] (one token plane per layer and KV head), plus
+ * a per-fact offset/length table.  Allocates the arenas (cudaMalloc, or
+ * cudaHostAlloc for IS_TIER_HOST), the RoPE frequency table (fp64, computed
+ * on the device) and the per-batch work space.  *out receives the store.
+ * Errors: INVALID_ARG (null, out-of-range field), NOT_SUPPORTED (head_dim),
+ * OOM, CUDA.  Nothing is leaked on error. */
+int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out);
+
+/* Free everything the store owns.  Waits for the store's work to finish.
+ * A NULL store is ignored. */
+void is_store_destroy(is_store_t* store);
+
+/* Append one fact: k_pre and v are bf16 [L][H][len][D] (host or device),
+ * the key taken BEFORE RoPE and the raw value (technical summary, Online
+ * phase, "Pre-RoPE storage").  The fact gets the next token range of every
+ * plane and the next id (ids are dense, in put order).  Synchronous: the
+ * caller's buffers may be reused on return.  Errors: INVALID_ARG (null,
+ * len <= 0), CAPACITY (tokens or ids exhausted), CUDA. */
+int is_store_put_fact(is_store_t* store, const void* k_pre, const void* v, int32_t len,
+                      int32_t* fact_id_out);
+
+/* Number of facts, and a fact's token offset in every plane and length. */
+int is_store_num_facts(const is_store_t* store, int32_t* num_facts_out);
+int is_store_fact_info(const is_store_t* store, int32_t fact_id, int64_t* offset_out,
+                       int32_t* len_out);
+
+/* Copy a stored fact back out as bf16 [L][H][len][D] (host or device
+ * destination; synchronous).  Errors: INVALID_ARG, BAD_FACT_ID, CUDA. */
+int is_store_read_fact(is_store_t* store, int32_t fact_id, void* k_out, void* v_out);
+
+/* Device addresses of the K and V arenas and the plane stride in tokens
+ * (for callers that fill or inspect the store in place).  For
+ * IS_TIER_HOST these are the device-mapped addresses of the host arenas. */
+int is_store_arena(const is_store_t* store, void** k_arena_out, void** v_arena_out,
+                   int64_t* plane_tokens_out);
+
+/* ---- the hot path ------------------------------------------------------ */
+
+/* Inject one batch (technical summary, Online phase, "Dynamic rotation" and
+ * "Injection").  Request r owns fact_ids[req_fact_offsets[r] ..
+ * req_fact_offsets[r+1]) in retrieval order.  Token t of its j-th fact is
+ * placed at position start_pos[r] + (lengths of facts 0..j-1) + t, i.e. the
+ * facts form one contiguous segment.  For every such token, every layer and
+ * every KV head:
+ *     V cache row at slot  <- stored V row                (bit copy)
+ *     K cache row at slot  <- bf16_rne(R(pos) . stored pre-RoPE K row)
+ * with slot = block_tables[r][pos / B] * B + pos % B and R(pos) the RoPE
+ * rotation of the store's configuration (fp64 angles, fp32 rotation).
+ * No other cache element is written.
+ *
+ * Arguments (all arrays on the device):
+ *   req_fact_offsets  int32 [num_requests + 1], CSR, [0] = 0,
+ *                     [num_requests] = num_fact_ids
+ *   fact_ids          int32 [num_fact_ids]; duplicates allowed
+ *   start_pos         int32 [num_requests], first injected position
+ *   block_tables      int32 [num_requests][max_blocks_per_req]
+ *   cache             geometry and base pointers of the paged cache
+ *   slot_mapping_out  optional int64 [slot_mapping_capacity]: the slot of
+ *                     every injected token, requests in order, segment order
+ *                     within a request; -1 for tokens not written.  NULL
+ *                     skips it.
+ * Asynchronous on `stream`.  Returns host-side validation errors
+ * (INVALID_ARG, CAPACITY when num_requests or num_fact_ids exceed the
+ * store's batch limits, NOT_SUPPORTED, CUDA); device-side errors are found
+ * by is_last_error():
+ *   INVALID_ARG  CSR does not cover num_fact_ids (nothing written), a
+ *                malformed request range or negative start (request skipped)
+ *   BAD_FACT_ID  id outside the store (its request skipped)
+ *   POSITION     segment past max_blocks_per_req * B (request skipped)
+ *   BAD_BLOCK    table entry outside [0, num_blocks) (that block skipped)
+ *   CAPACITY     more tokens than slot_mapping_capacity (nothing written)
+ * Requests must not share slots (the winner is undefined). */
+int is_inject_batch(is_store_t* store, int32_t num_requests, const int32_t* req_fact_offsets,
+                    const int32_t* fact_ids, int32_t num_fact_ids, const int32_t* start_pos,
+                    const int32_t* block_tables, int32_t max_blocks_per_req,
+                    const is_cache_t* cache, int64_t* slot_mapping_out,
+                    int64_t slot_mapping_capacity, void* stream);
+
+/* The same batch with the four index arrays in HOST memory (pinned memory
+ * makes the copies asynchronous) and slot_mapping_out, if not NULL, in host
+ * memory.  Copies the arrays into store-owned device buffers, runs the
+ * batch, copies the slots back, waits for `stream` and returns the batch's
+ * status (host-side or device-side, as for is_inject_batch +
+ * is_last_error).  The caches stay on the device. */
+int is_inject_batch_host(is_store_t* store, int32_t num_requests,
+                         const int32_t* req_fact_offsets, const int32_t* fact_ids,
+                         int32_t num_fact_ids, const int32_t* start_pos,
+                         const int32_t* block_tables, int32_t max_blocks_per_req,
+                         const is_cache_t* cache, int64_t* slot_mapping_out,
+                         int64_t slot_mapping_capacity, void* stream);
+
+/* Wait for `stream`, then return and clear the first device-side error
+ * recorded since the previous call (IS_OK if none).  *detail_out, if not
+ * NULL, receives the offending index (request, CSR entry or block). */
+int is_last_error(is_store_t* store, void* stream, int64_t* detail_out);
+
+/* ---- measurement -------------------------------------------------------- */
+
+/* Enable (1) or disable (0) CUDA-event timing of the inject kernel itself
+ * (the plan kernel excluded).  While enabled each batch records two events
+ * on its stream around the inject kernel. */
+int is_store_set_timing(is_store_t* store, int enable);
+
+/* Sum of inject-kernel durations (ms) and number of timed launches since
+ * the previous call; waits for the recorded events.  Resets the sums. */
+int is_store_kernel_time(is_store_t* store, double* total_ms_out, int64_t* launches_out);
+
+/* Human-readable name of a status code (static string). */
+const char* is_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* INJECT_STORE_H */

@@ -1,0 +1,193 @@
+"""ctypes binding of libinjectstore.so (include/inject_store.h).
+
+Argument marshalling only: every step of the inject path runs in the CUDA
+library.  Pointers are plain integers (``tensor.data_ptr()``) and streams are
+``torch.cuda.Stream.cuda_stream`` integers; no torch type crosses the C-ABI.
+If the shared library is missing this module raises at import: there is no
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libinjectstore.so")
+
+IS_OK = 0
+IS_ERR_INVALID_ARG = -1
+IS_ERR_BAD_FACT_ID = -2
+IS_ERR_POSITION = -3
+IS_ERR_BAD_BLOCK = -4
+IS_ERR_CAPACITY = -5
+IS_ERR_OOM = -6
+IS_ERR_CUDA = -7
+IS_ERR_TIMEOUT = -8
+IS_ERR_NOT_SUPPORTED = -9
+
+IS_ROPE_ROTATE_HALF = 0
+IS_ROPE_INTERLEAVED = 1
+IS_SCALING_NONE = 0
+IS_SCALING_LLAMA3 = 1
+IS_TIER_DEVICE = 0
+IS_TIER_HOST = 1
+
+_I32, _I64, _F64, _P = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+
+
+class is_store_config_t(ctypes.Structure):
+    _fields_ = [
+        ("num_layers", _I32), ("num_kv_heads", _I32), ("head_dim", _I32), ("rope_style", _I32),
+        ("rope_theta", _F64), ("rope_scaling", _I32), ("scale_factor", _F64),
+        ("low_freq_factor", _F64), ("high_freq_factor", _F64), ("original_max_position", _I32),
+        ("capacity_tokens", _I64), ("max_facts", _I32), ("max_batch_requests", _I32),
+        ("max_batch_fact_ids", _I32), ("max_batch_blocks", _I32), ("tier", _I32),
+        ("hot_capacity_tokens", _I64),
+    ]
+
+
+class is_cache_t(ctypes.Structure):
+    _fields_ = [
+        ("k_cache", _P), ("v_cache", _P), ("layer_stride", _I64), ("block_stride", _I64),
+        ("token_stride", _I64), ("head_stride", _I64), ("num_blocks", _I32), ("block_size", _I32),
+    ]
+
+
+class InjectError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m kv_cache_injection_gather_b200.build` "
+        "(the inject path has no Python or CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_SIGNATURES = {
+    "is_store_create": (ctypes.c_int, [ctypes.POINTER(is_store_config_t), ctypes.c_int,
+                                       ctypes.POINTER(_P)]),
+    "is_store_destroy": (None, [_P]),
+    "is_store_put_fact": (ctypes.c_int, [_P, _P, _P, _I32, ctypes.POINTER(_I32)]),
+    "is_store_num_facts": (ctypes.c_int, [_P, ctypes.POINTER(_I32)]),
+    "is_store_fact_info": (ctypes.c_int, [_P, _I32, ctypes.POINTER(_I64), ctypes.POINTER(_I32)]),
+    "is_store_read_fact": (ctypes.c_int, [_P, _I32, _P, _P]),
+    "is_store_arena": (ctypes.c_int, [_P, ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                      ctypes.POINTER(_I64)]),
+    "is_inject_batch": (ctypes.c_int, [_P, _I32, _P, _P, _I32, _P, _P, _I32,
+                                       ctypes.POINTER(is_cache_t), _P, _I64, _P]),
+    "is_inject_batch_host": (ctypes.c_int, [_P, _I32, _P, _P, _I32, _P, _P, _I32,
+                                            ctypes.POINTER(is_cache_t), _P, _I64, _P]),
+    "is_last_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(_I64)]),
+    "is_store_set_timing": (ctypes.c_int, [_P, ctypes.c_int]),
+    "is_store_kernel_time": (ctypes.c_int, [_P, ctypes.POINTER(_F64), ctypes.POINTER(_I64)]),
+    "is_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+for _name, (_res, _args) in _SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.is_status_string(status).decode()
+
+
+def check(status: int, where: str = "call") -> None:
+    if status != IS_OK:
+        raise InjectError(status, where)
+
+
+# ---- the C-ABI, same names -------------------------------------------------
+
+def is_store_create(cfg: is_store_config_t, device: int = 0) -> int:
+    out = _P()
+    check(_lib.is_store_create(ctypes.byref(cfg), device, ctypes.byref(out)), "is_store_create")
+    return out.value
+
+
+def is_store_destroy(store: int) -> None:
+    _lib.is_store_destroy(store)
+
+
+def is_store_put_fact(store: int, k_pre_ptr: int, v_ptr: int, length: int) -> int:
+    fid = _I32()
+    check(_lib.is_store_put_fact(store, k_pre_ptr, v_ptr, length, ctypes.byref(fid)),
+          "is_store_put_fact")
+    return fid.value
+
+
+def is_store_num_facts(store: int) -> int:
+    n = _I32()
+    check(_lib.is_store_num_facts(store, ctypes.byref(n)), "is_store_num_facts")
+    return n.value
+
+
+def is_store_fact_info(store: int, fact_id: int) -> tuple[int, int]:
+    off, ln = _I64(), _I32()
+    check(_lib.is_store_fact_info(store, fact_id, ctypes.byref(off), ctypes.byref(ln)),
+          "is_store_fact_info")
+    return off.value, ln.value
+
+
+def is_store_read_fact(store: int, fact_id: int, k_out_ptr: int, v_out_ptr: int) -> None:
+    check(_lib.is_store_read_fact(store, fact_id, k_out_ptr, v_out_ptr), "is_store_read_fact")
+
+
+def is_store_arena(store: int) -> tuple[int, int, int]:
+    k, v, t = _P(), _P(), _I64()
+    check(_lib.is_store_arena(store, ctypes.byref(k), ctypes.byref(v), ctypes.byref(t)),
+          "is_store_arena")
+    return k.value, v.value, t.value
+
+
+def is_inject_batch(store: int, num_requests: int, req_fact_offsets: int, fact_ids: int,
+                    num_fact_ids: int, start_pos: int, block_tables: int,
+                    max_blocks_per_req: int, cache: is_cache_t, slot_mapping_out: int | None,
+                    slot_mapping_capacity: int, stream: int = 0) -> int:
+    """Asynchronous; returns the host-side status (raises on error)."""
+    rc = _lib.is_inject_batch(store, num_requests, req_fact_offsets, fact_ids, num_fact_ids,
+                              start_pos, block_tables, max_blocks_per_req, ctypes.byref(cache),
+                              slot_mapping_out, slot_mapping_capacity, stream)
+    check(rc, "is_inject_batch")
+    return rc
+
+
+def is_inject_batch_host(store: int, num_requests: int, req_fact_offsets: int, fact_ids: int,
+                         num_fact_ids: int, start_pos: int, block_tables: int,
+                         max_blocks_per_req: int, cache: is_cache_t,
+                         slot_mapping_out: int | None, slot_mapping_capacity: int,
+                         stream: int = 0) -> int:
+    """Host index arrays in, status out (waits for the stream).  Returns the
+    batch status without raising, so callers can inspect device errors."""
+    return _lib.is_inject_batch_host(store, num_requests, req_fact_offsets, fact_ids,
+                                     num_fact_ids, start_pos, block_tables, max_blocks_per_req,
+                                     ctypes.byref(cache), slot_mapping_out,
+                                     slot_mapping_capacity, stream)
+
+
+def is_last_error(store: int, stream: int = 0) -> tuple[int, int]:
+    detail = _I64()
+    rc = _lib.is_last_error(store, stream, ctypes.byref(detail))
+    return rc, detail.value
+
+
+def is_store_set_timing(store: int, enable: bool) -> None:
+    check(_lib.is_store_set_timing(store, int(bool(enable))), "is_store_set_timing")
+
+
+def is_store_kernel_time(store: int) -> tuple[float, int]:
+    ms, n = _F64(), _I64()
+    check(_lib.is_store_kernel_time(store, ctypes.byref(ms), ctypes.byref(n)),
+          "is_store_kernel_time")
+    return ms.value, n.value
+
+
+def is_status_string(status: int) -> str:
+    return status_string(status)

@@ -1,0 +1,535 @@
+// Device code of the retrieve-and-inject path for sm_100a.
+//
+// Two kernels per batch (technical summary of "InferScale: GPU-Native KV
+// Injection for Personalized LLM Serving", section "Methodology -- 2. Online
+// phase: Chunked RoPE and KV injection"):
+//
+//   plan_kernel    one CTA.  Composes every request's retrieved facts into one
+//                  contiguous segment ("Dynamic rotation": the facts are laid
+//                  out as one segment at new serving positions), validates the
+//                  batch, and writes one descriptor per touched cache block.
+//   inject_kernel  persistent grid.  Per work unit (one cache block of one
+//                  request x a range of layers) it gathers the stored pre-RoPE
+//                  K and raw V rows of the block's tokens, rotates K to the
+//                  tokens' positions (RoPE, fp64 angles, fp32 rotation, bf16
+//                  round-to-nearest-even), and writes K and V into the paged
+//                  cache ("Injection": scatter-copy into the paged KV cache).
+//
+// The path is a copy with a small rotation: bandwidth-bound on HBM.  Every
+// global access is a 16-byte vector; a block's tokens of one layer are one
+// contiguous run of the cache (token-major layout), written by consecutive
+// threads.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace isk {
+
+// Status codes, same values as inject_store.h.
+enum : int32_t {
+  kOk = 0,
+  kErrInvalidArg = -1,
+  kErrBadFactId = -2,
+  kErrPosition = -3,
+  kErrBadBlock = -4,
+  kErrCapacity = -5,
+};
+
+struct DevStatus {
+  int32_t code;
+  int32_t pad;
+  long long detail;
+};
+
+// Written by plan_kernel, read by inject_kernel.
+struct PlanHeader {
+  int32_t total_blocks;      // touched cache blocks over all valid requests
+  int32_t layers_per_unit;   // layers one work unit covers
+  int32_t units_per_block;   // ceil(L / layers_per_unit)
+  int32_t total_units;       // total_blocks * units_per_block (0: write nothing)
+  unsigned int next_unit;    // dynamic work counter, reset by plan_kernel
+  int32_t pad;
+  long long total_tokens;    // segment tokens over all requests
+};
+
+// One touched cache block of one request.
+struct BlockDesc {
+  int32_t r;     // request
+  int32_t b;     // logical block index in the request's table
+  int32_t j;     // CSR index of the first fact with a token in the block
+  int32_t pad;
+};
+
+__device__ __forceinline__ void record_error(DevStatus* st, int32_t code, long long detail) {
+  if (atomicCAS(&st->code, 0, code) == 0) st->detail = detail;
+}
+
+// ---------------------------------------------------------------- plan kernel
+
+struct PlanArgs {
+  int32_t R;
+  const int32_t* req_off;    // [R+1]
+  const int32_t* fact_ids;   // [num_ids]
+  int32_t num_ids;
+  const int32_t* start_pos;  // [R]
+  int32_t max_blocks;
+  int32_t B;
+  int32_t L;
+  const int32_t* fact_len;   // store: [num_facts]
+  int32_t num_facts;
+  int64_t* slot_out;         // optional
+  int64_t slot_cap;
+  int32_t grid_ctas;         // size of the inject grid (for unit sizing)
+  int32_t max_batch_blocks;  // capacity of desc
+  // work space
+  int32_t* seg;              // [num_ids]   segment offset of each CSR entry (-1: bad id)
+  int32_t* req_nblk;         // [R]         touched blocks (0 when invalid)
+  int32_t* req_blk0;         // [R+1]       exclusive prefix of req_nblk
+  long long* req_tok0;       // [R+1]       exclusive prefix of segment lengths
+  int32_t* req_len;          // [R]         segment length (valid facts)
+  int32_t* req_valid;        // [R]
+  BlockDesc* desc;           // [max_batch_blocks]
+  PlanHeader* hdr;
+  DevStatus* st;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int s_bad;
+  __shared__ int s_wsum_blk[NW];
+  __shared__ long long s_wsum_tok[NW];
+
+  if (tid == 0) {
+    const bool bad = a.R < 0 || a.req_off[0] != 0 || a.req_off[a.R] != a.num_ids;
+    s_bad = bad;
+    if (bad) {
+      record_error(a.st, kErrInvalidArg, -1);
+      a.hdr->total_blocks = 0;
+      a.hdr->total_units = 0;
+      a.hdr->units_per_block = 1;
+      a.hdr->layers_per_unit = a.L;
+      a.hdr->next_unit = 0;
+      a.hdr->total_tokens = 0;
+    }
+  }
+  __syncthreads();
+  if (s_bad) return;
+
+  // Phase 1, one warp per request: segment offsets of its facts (exclusive
+  // prefix of their lengths, in retrieval order), length, validity, blocks.
+  for (int r = warp; r < a.R; r += NW) {
+    const int32_t j0 = a.req_off[r], j1 = a.req_off[r + 1];
+    int32_t err = kOk;
+    long long S = 0;
+    if (j0 < 0 || j1 < j0 || j1 > a.num_ids) {
+      err = kErrInvalidArg;  // malformed range: no tokens
+    } else {
+      for (int32_t base = j0; base < j1; base += 32) {
+        const int32_t j = base + lane;
+        int32_t len = 0;
+        bool ok = true;
+        if (j < j1) {
+          const int32_t f = a.fact_ids[j];
+          ok = f >= 0 && f < a.num_facts;
+          len = ok ? a.fact_len[f] : 0;
+        }
+        int32_t x = len;  // inclusive warp scan
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int32_t y = __shfl_up_sync(0xffffffffu, x, d);
+          if (lane >= d) x += y;
+        }
+        if (j < j1) a.seg[j] = ok ? int32_t(S + x - len) : -1;
+        const unsigned badm = __ballot_sync(0xffffffffu, j < j1 && !ok);
+        if (badm && err == kOk) err = kErrBadFactId;
+        S += __shfl_sync(0xffffffffu, x, 31);
+      }
+    }
+    const int32_t start = a.start_pos[r];
+    if (err == kOk && start < 0) err = kErrInvalidArg;
+    if (err == kOk && (long long)start + S > (long long)a.max_blocks * a.B) err = kErrPosition;
+    if (lane == 0) {
+      int32_t nblk = 0;
+      if (err == kOk && S > 0) nblk = int32_t((start + S - 1) / a.B - start / a.B + 1);
+      a.req_nblk[r] = nblk;
+      a.req_len[r] = int32_t(S);
+      a.req_valid[r] = err == kOk;
+      if (err != kOk) record_error(a.st, err, r);
+    }
+  }
+  __syncthreads();
+
+  // Phase 2: exclusive prefixes over requests (blocks and tokens).  Thread t
+  // owns a contiguous run of requests.
+  const int per = (a.R + NT - 1) / NT;
+  const int r0 = min(a.R, tid * per), r1 = min(a.R, r0 + per);
+  int32_t my_blk = 0;
+  long long my_tok = 0;
+  for (int r = r0; r < r1; ++r) { my_blk += a.req_nblk[r]; my_tok += a.req_len[r]; }
+  int32_t xb = my_blk;
+  long long xt = my_tok;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t yb = __shfl_up_sync(0xffffffffu, xb, d);
+    const long long yt = __shfl_up_sync(0xffffffffu, xt, d);
+    if (lane >= d) { xb += yb; xt += yt; }
+  }
+  if (lane == 31) { s_wsum_blk[warp] = xb; s_wsum_tok[warp] = xt; }
+  __syncthreads();
+  int32_t wb = 0;
+  long long wt = 0;
+  for (int w = 0; w < warp; ++w) { wb += s_wsum_blk[w]; wt += s_wsum_tok[w]; }
+  int32_t eb = wb + xb - my_blk;
+  long long et = wt + xt - my_tok;
+  for (int r = r0; r < r1; ++r) {
+    a.req_blk0[r] = eb;
+    a.req_tok0[r] = et;
+    eb += a.req_nblk[r];
+    et += a.req_len[r];
+  }
+  if (tid == NT - 1) {
+    a.req_blk0[a.R] = eb;
+    a.req_tok0[a.R] = et;
+  }
+  __syncthreads();
+  const int32_t total_blocks = a.req_blk0[a.R];
+  const long long total_tokens = a.req_tok0[a.R];
+  const bool over_slots = a.slot_out != nullptr && total_tokens > a.slot_cap;
+  const bool over_blocks = total_blocks > a.max_batch_blocks;
+
+  if (tid == 0) {
+    // Work-unit size: enough units for ~32 per CTA, layers split evenly.
+    long long want = (long long)a.grid_ctas * 32;
+    int32_t upb = 1;
+    if (total_blocks > 0 && (long long)total_blocks < want)
+      upb = int32_t(min((long long)a.L, (want + total_blocks - 1) / total_blocks));
+    const int32_t lpu = (a.L + upb - 1) / upb;
+    upb = (a.L + lpu - 1) / lpu;
+    a.hdr->layers_per_unit = lpu;
+    a.hdr->units_per_block = upb;
+    a.hdr->total_blocks = total_blocks;
+    a.hdr->total_tokens = total_tokens;
+    a.hdr->next_unit = 0;
+    a.hdr->total_units = (over_slots || over_blocks) ? 0 : total_blocks * upb;
+    if (over_slots || over_blocks) record_error(a.st, kErrCapacity, total_tokens);
+  }
+  if (over_slots || over_blocks) return;
+
+  // Phase 3, one warp per request: block descriptors (lanes over facts), and
+  // -1 slots for the tokens of invalid requests.
+  for (int r = warp; r < a.R; r += NW) {
+    const int32_t j0 = a.req_off[r], j1 = a.req_off[r + 1];
+    const long long t0 = a.req_tok0[r];
+    if (!a.req_valid[r]) {
+      if (a.slot_out)
+        for (int32_t i = lane; i < a.req_len[r]; i += 32) a.slot_out[t0 + i] = -1;
+      continue;
+    }
+    const int32_t nblk = a.req_nblk[r];
+    if (nblk == 0) continue;
+    const int32_t start = a.start_pos[r];
+    const int32_t fb = start / a.B;            // first logical block
+    const int32_t g0 = a.req_blk0[r];
+    // Fact j covers segment indices [seg[j], seg[j] + len_j).  Block bi >= 1
+    // starts at segment index (fb + bi) * B - start; block 0 starts at 0.
+    for (int32_t base = j0; base < j1; base += 32) {
+      const int32_t j = base + lane;
+      if (j >= j1) continue;
+      const int32_t s = a.seg[j];
+      const int32_t len = a.fact_len[a.fact_ids[j]];
+      if (len == 0) continue;
+      const int32_t e = s + len;               // exclusive end
+      // blocks bi whose first segment index lies in [s, e)
+      int32_t bi_lo = (s + start + a.B - 1) / a.B - fb;
+      const int32_t bi_hi = (e + start + a.B - 1) / a.B - fb;  // exclusive
+      if (s == 0) bi_lo = 0;
+      for (int32_t bi = max(bi_lo, 0); bi < bi_hi && bi < nblk; ++bi) {
+        BlockDesc d;
+        d.r = r;
+        d.b = fb + bi;
+        d.j = j;
+        d.pad = 0;
+        a.desc[g0 + bi] = d;
+      }
+    }
+  }
+}
+
+// -------------------------------------------------------------- inject kernel
+
+struct InjectArgs {
+  const uint16_t* k_store;   // [L][H][T_cap][D]
+  const uint16_t* v_store;
+  int64_t plane;             // T_cap * D  (elements between (l,h) planes)
+  const int64_t* fact_off;   // store token offset of each fact
+  const int32_t* fact_len;
+  const double* inv_freq;    // [D/2]
+  int32_t L, H;
+  const int32_t* req_off;
+  const int32_t* fact_ids;
+  const int32_t* start_pos;
+  const int32_t* block_tables;
+  int32_t max_blocks;
+  uint16_t* k_cache;
+  uint16_t* v_cache;
+  int64_t ls, bs, ts, hs;    // cache strides (elements)
+  int32_t num_blocks, B;
+  int64_t* slot_out;
+  const int32_t* seg;
+  const long long* req_tok0;
+  const BlockDesc* desc;
+  PlanHeader* hdr;
+  DevStatus* st;
+};
+
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_stream(uint16_t* p, const uint4& v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Index (in float2 units) of the cos/sin entry of frequency i for in-block
+// token o, laid out so that the lanes of one row read consecutive 16-byte
+// words (no shared-memory bank conflicts):
+//   rotate-half: vector c' = i / 8 of a half row, element e = i % 8
+//                float4 index (o * 4 + e / 2) * (D / 16) + c', half e % 2
+//   interleaved: vector c = i / 4, pair m = i % 4
+//                float4 index (o * 2 + m / 2) * (D / 8) + c, half m % 2
+template <int D, int STYLE>
+__device__ __forceinline__ int cs_index(int o, int i) {
+  if (STYLE == 0) {
+    const int cp = i >> 3, e = i & 7;
+    return (((o * 4 + (e >> 1)) * (D / 16) + cp) << 1) + (e & 1);
+  } else {
+    const int c = i >> 2, m = i & 3;
+    return (((o * 2 + (m >> 1)) * (D / 8) + c) << 1) + (m & 1);
+  }
+}
+
+// Rotate one 16-byte vector (8 bf16) of a key row.
+//   own: this lane's vector; c: its index in the row (0 .. D/8-1)
+//   cs: cos/sin table of this token (float4 words as laid out above)
+template <int D, int STYLE>
+__device__ __forceinline__ uint4 rotate_vec(const uint4 own, int c, const float4* cs_tok) {
+  const uint32_t w[4] = {own.x, own.y, own.z, own.w};
+  float x[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) { x[2 * q] = bf_lo(w[q]); x[2 * q + 1] = bf_hi(w[q]); }
+  float y[8];
+  if (STYLE == 0) {
+    // Pair (i, i + D/2): the partner vector sits D/16 lanes away.
+    constexpr int VH = D / 16;
+    uint32_t pw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) pw[q] = __shfl_xor_sync(0xffffffffu, w[q], VH);
+    float p[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) { p[2 * q] = bf_lo(pw[q]); p[2 * q + 1] = bf_hi(pw[q]); }
+    const bool first = c < VH;
+    const int cp = first ? c : c - VH;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 t = cs_tok[q * VH + cp];  // {cos, sin} of elements 2q, 2q+1
+      const float s0 = first ? -t.y : t.y, s1 = first ? -t.w : t.w;
+      // first half:  x cos - partner sin;  second half: x cos + partner sin
+      y[2 * q] = fmaf(x[2 * q], t.x, p[2 * q] * s0);
+      y[2 * q + 1] = fmaf(x[2 * q + 1], t.z, p[2 * q + 1] * s1);
+    }
+  } else {
+    // Pairs (2m, 2m+1) inside the vector.
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float4 t = cs_tok[h * (D / 8) + c];  // pairs 2h and 2h+1 of this vector
+      const int a0 = 4 * h, a1 = 4 * h + 2;
+      y[a0] = fmaf(x[a0], t.x, -(x[a0 + 1] * t.y));
+      y[a0 + 1] = fmaf(x[a0 + 1], t.x, x[a0] * t.y);
+      y[a1] = fmaf(x[a1], t.z, -(x[a1 + 1] * t.w));
+      y[a1 + 1] = fmaf(x[a1 + 1], t.z, x[a1] * t.w);
+    }
+  }
+  uint4 out;
+  out.x = pack_bf16(y[0], y[1]);
+  out.y = pack_bf16(y[2], y[3]);
+  out.z = pack_bf16(y[4], y[5]);
+  out.w = pack_bf16(y[6], y[7]);
+  return out;
+}
+
+constexpr int kMaxBlockSize = 128;
+
+// x / d and x % d for a divisor fixed per launch: shifts when d is a power
+// of two (POW2), plain division otherwise.
+template <bool POW2>
+struct Divisor {
+  int d, sh;
+  __device__ __forceinline__ int div(int x) const { return POW2 ? (x >> sh) : x / d; }
+  __device__ __forceinline__ int mod(int x) const { return POW2 ? (x & (d - 1)) : x % d; }
+};
+
+__device__ __forceinline__ int ilog2(int x) { return 31 - __clz(x); }
+
+// Persistent gather-rotate-scatter kernel.  Work unit u covers global block
+// gb = u % total_blocks and layers [lg * lpu, min(L, (lg + 1) * lpu)),
+// lg = u / total_blocks, so CTAs running side by side read neighbouring
+// tokens of the same layers.  Units are taken from an atomic counter; the
+// next unit is fetched while the current one is copied.
+//
+// Inside a unit the vectors are numbered v = ((l - l0) * B + o) * H * D/8 +
+// h * D/8 + c (layer, in-block slot, head, 16-byte vector of the row), so
+// consecutive threads write consecutive 16-byte words of the token-major
+// cache and read whole 256-byte head rows of the store.  POW2: H and B are
+// powers of two (all index splits are shifts).
+template <int D, int STYLE, int NT, int VPT, bool POW2>
+__global__ void __launch_bounds__(NT, 2) inject_kernel(InjectArgs a) {
+  constexpr int VPR = D / 8;  // 16-byte vectors per head row
+  constexpr int LOG_VPR = (VPR == 4) ? 2 : (VPR == 8) ? 3 : (VPR == 16) ? 4 : 5;
+  extern __shared__ float4 s_cs4[];            // [B * D/4] cos/sin of the block
+  __shared__ long long s_src[kMaxBlockSize];  // store token of each slot (-1: none)
+  __shared__ int s_unit;
+
+  const int tid = threadIdx.x;
+  const int total_units = a.hdr->total_units;
+  const int total_blocks = a.hdr->total_blocks;
+  const int lpu = a.hdr->layers_per_unit;
+  const int B = a.B;
+  const int H = a.H;
+  const int row_vecs = H * VPR;         // vectors per token (all heads)
+  const int vecs_layer = B * row_vecs;  // vectors per block and layer
+  const Divisor<POW2> by_layer{vecs_layer, POW2 ? ilog2(vecs_layer) : 0};
+  const Divisor<POW2> by_row{row_vecs, POW2 ? ilog2(row_vecs) : 0};
+
+  int next = 0;
+  if (tid == 0) next = int(atomicAdd(&a.hdr->next_unit, 1u));
+  for (;;) {
+    __syncthreads();  // the previous unit's tables are no longer read
+    if (tid == 0) {
+      s_unit = next;
+      if (next < total_units) next = int(atomicAdd(&a.hdr->next_unit, 1u));
+    }
+    __syncthreads();
+    const int u = s_unit;
+    if (u >= total_units) break;
+    const int gb = u % total_blocks;
+    const int lg = u / total_blocks;
+    const BlockDesc d = a.desc[gb];
+    const int r = d.r;
+    const int start = a.start_pos[r];
+    const int j1 = a.req_off[r + 1];
+    const long long tok0 = a.req_tok0[r];
+    const int len_r = int(a.req_tok0[r + 1] - tok0);
+    const int blk_pos = d.b * B;                       // position of in-block slot 0
+    const int o_lo = max(start - blk_pos, 0);
+    const int o_hi = min(start + len_r - blk_pos, B);  // exclusive
+    const int phys = a.block_tables[(long long)r * a.max_blocks + d.b];
+    const bool phys_ok = phys >= 0 && phys < a.num_blocks;
+    const int l0 = lg * lpu, l1 = min(a.L, l0 + lpu);
+
+    // Store token of each in-block slot: walk forward from the block's
+    // first fact (facts cover consecutive segment ranges).
+    if (tid < B) {
+      const int o = tid;
+      long long src = -1;
+      if (o >= o_lo && o < o_hi) {
+        const int i = blk_pos + o - start;  // segment index
+        int j = d.j;
+        while (j + 1 < j1 && a.seg[j + 1] <= i) ++j;
+        src = a.fact_off[a.fact_ids[j]] + (i - a.seg[j]);
+        if (lg == 0 && a.slot_out) a.slot_out[tok0 + i] = phys_ok ? (long long)phys * B + o : -1;
+      }
+      s_src[o] = src;
+    }
+    if (!phys_ok) {
+      if (tid == 0 && lg == 0) record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + d.b);
+      continue;  // uniform; the loop top holds the barrier
+    }
+    // cos/sin of every (slot, frequency): fp64 angle and sincos, kept fp32.
+    for (int e = tid; e < B * (D / 2); e += NT) {
+      const int o = e / (D / 2), i = e % (D / 2);
+      double sn, cn;
+      sincos(double(blk_pos + o) * a.inv_freq[i], &sn, &cn);
+      reinterpret_cast<float2*>(s_cs4)[cs_index<D, STYLE>(o, i)] = make_float2(float(cn), float(sn));
+    }
+    __syncthreads();
+
+    const int total = (l1 - l0) * vecs_layer;
+    const uint16_t* kst = a.k_store;
+    const uint16_t* vst = a.v_store;
+    for (int base = 0; base < total; base += NT * VPT) {
+      uint4 kv[VPT], vv[VPT];
+#pragma unroll
+      for (int q = 0; q < VPT; ++q) {
+        const int v = base + q * NT + tid;
+        const int l = l0 + by_layer.div(v);
+        const int rem = by_layer.mod(v);
+        const int o = by_row.div(rem), hv = by_row.mod(rem);
+        const long long src = v < total ? s_src[o] : -1;
+        kv[q] = make_uint4(0, 0, 0, 0);
+        vv[q] = kv[q];
+        if (src >= 0) {
+          const long long so = (long long)(l * H + (hv >> LOG_VPR)) * a.plane + src * D +
+                               (hv & (VPR - 1)) * 8;
+          kv[q] = ld_stream(kst + so);
+          vv[q] = ld_stream(vst + so);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < VPT; ++q) {
+        const int v = base + q * NT + tid;
+        const int l = l0 + by_layer.div(v);
+        const int rem = by_layer.mod(v);
+        const int o = v < total ? by_row.div(rem) : 0, hv = by_row.mod(rem);
+        const int c = hv & (VPR - 1);
+        const uint4 kr = rotate_vec<D, STYLE>(kv[q], c, s_cs4 + o * (D / 4));
+        if (v < total && s_src[o] >= 0) {
+          const long long dst = (long long)l * a.ls + (long long)phys * a.bs + (long long)o * a.ts +
+                                (long long)(hv >> LOG_VPR) * a.hs + c * 8;
+          st_stream(a.k_cache + dst, kr);
+          st_stream(a.v_cache + dst, vv[q]);
+        }
+      }
+    }
+  }
+}
+
+// RoPE frequencies, fp64: inv_freq_i = theta^(-2i/D), optionally with the
+// Llama-3.1 wavelength-band rule (wavelength 2 pi / f below orig/high: kept;
+// above orig/low: divided by factor; between: blended with weight
+// (orig / wavelength - low) / (high - low) on the unscaled frequency).
+__global__ void inv_freq_kernel(double* out, int D, double theta, int scaling, double factor,
+                                double low, double high, double orig) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= D / 2) return;
+  double f = pow(theta, -2.0 * double(i) / double(D));
+  if (scaling == 1) {
+    const double wl = 2.0 * 3.14159265358979323846 / f;
+    if (wl > orig / low) {
+      f = f / factor;
+    } else if (wl >= orig / high) {
+      const double w = (orig / wl - low) / (high - low);
+      f = (1.0 - w) * (f / factor) + w * f;
+    }
+  }
+  out[i] = f;
+}
+
+}  // namespace isk

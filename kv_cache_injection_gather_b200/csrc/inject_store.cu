@@ -1,0 +1,512 @@
+// Host side of libinjectstore.so: the fact store, the C-ABI declared in
+// include/inject_store.h, and the launches of the plan and inject kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "inject_store.h"
+#include "inject_kernels.cuh"
+
+namespace {
+
+constexpr int kPlanThreads = 1024;
+constexpr int kInjectThreads = 256;
+constexpr int kVecsPerThread = 8;
+constexpr int kDefaultMaxRequests = 4096;
+constexpr int kDefaultMaxFactIds = 1 << 20;
+constexpr int kMaxTimedLaunches = 4096;
+
+struct TimedLaunch {
+  cudaEvent_t start, stop;
+};
+
+}  // namespace
+
+struct is_store {
+  is_store_config_t cfg{};
+  int device = 0;
+  int sm_count = 148;
+  // arenas [L][H][T_cap][D] bf16
+  uint16_t* k = nullptr;
+  uint16_t* v = nullptr;
+  bool host_arena = false;
+  // fact table
+  int64_t* d_off = nullptr;
+  int32_t* d_len = nullptr;
+  std::vector<int64_t> h_off;
+  std::vector<int32_t> h_len;
+  int64_t used_tokens = 0;
+  int32_t num_facts = 0;
+  double* d_inv_freq = nullptr;
+  // per-batch work space
+  int32_t max_req = 0, max_ids = 0, max_blocks = 0;
+  int32_t* ws_seg = nullptr;
+  int32_t* ws_nblk = nullptr;
+  int32_t* ws_blk0 = nullptr;
+  long long* ws_tok0 = nullptr;
+  int32_t* ws_len = nullptr;
+  int32_t* ws_valid = nullptr;
+  isk::BlockDesc* ws_desc = nullptr;
+  isk::PlanHeader* ws_hdr = nullptr;
+  isk::DevStatus* d_status = nullptr;
+  // staging for is_inject_batch_host
+  int32_t* stage = nullptr;
+  size_t stage_elems = 0;
+  int64_t* stage_slots = nullptr;
+  int64_t stage_slot_elems = 0;
+  // timing
+  bool timing = false;
+  std::vector<TimedLaunch> events;
+  size_t events_used = 0;
+  // kernel configuration
+  int inject_grid = 0;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+template <typename T>
+cudaError_t dalloc(T** p, size_t count) {
+  return cudaMalloc(reinterpret_cast<void**>(p), std::max<size_t>(count, 1) * sizeof(T));
+}
+
+void free_store(is_store* s) {
+  if (!s) return;
+  cudaFree(s->d_off);
+  cudaFree(s->d_len);
+  cudaFree(s->d_inv_freq);
+  cudaFree(s->ws_seg);
+  cudaFree(s->ws_nblk);
+  cudaFree(s->ws_blk0);
+  cudaFree(s->ws_tok0);
+  cudaFree(s->ws_len);
+  cudaFree(s->ws_valid);
+  cudaFree(s->ws_desc);
+  cudaFree(s->ws_hdr);
+  cudaFree(s->d_status);
+  cudaFree(s->stage);
+  cudaFree(s->stage_slots);
+  if (s->host_arena) {
+    cudaFreeHost(s->k);
+    cudaFreeHost(s->v);
+  } else {
+    cudaFree(s->k);
+    cudaFree(s->v);
+  }
+  for (auto& e : s->events) {
+    cudaEventDestroy(e.start);
+    cudaEventDestroy(e.stop);
+  }
+  delete s;
+}
+
+bool head_dim_supported(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
+
+template <int D, int STYLE, bool POW2>
+void* inject_fn() {
+  return reinterpret_cast<void*>(&isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, POW2>);
+}
+
+template <bool POW2>
+void* pick_inject_t(int D, int style) {
+  switch (D) {
+    case 32: return style ? inject_fn<32, 1, POW2>() : inject_fn<32, 0, POW2>();
+    case 64: return style ? inject_fn<64, 1, POW2>() : inject_fn<64, 0, POW2>();
+    case 128: return style ? inject_fn<128, 1, POW2>() : inject_fn<128, 0, POW2>();
+    case 256: return style ? inject_fn<256, 1, POW2>() : inject_fn<256, 0, POW2>();
+    default: return nullptr;
+  }
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// The inject kernel for a head dim, RoPE style and (H, B): the shift variant
+// when both are powers of two.
+void* pick_inject(int D, int style, int H, int B) {
+  return (is_pow2(H) && is_pow2(B)) ? pick_inject_t<true>(D, style) : pick_inject_t<false>(D, style);
+}
+
+size_t cs_smem_bytes(int D, int B) { return size_t(B) * size_t(D / 2) * sizeof(float2); }
+
+int grow_stage(is_store* s, size_t elems, int64_t slot_elems) {
+  if (elems > s->stage_elems) {
+    cudaFree(s->stage);
+    s->stage = nullptr;
+    s->stage_elems = 0;
+    if (dalloc(&s->stage, elems) != cudaSuccess) return IS_ERR_OOM;
+    s->stage_elems = elems;
+  }
+  if (slot_elems > s->stage_slot_elems) {
+    cudaFree(s->stage_slots);
+    s->stage_slots = nullptr;
+    s->stage_slot_elems = 0;
+    if (dalloc(&s->stage_slots, size_t(slot_elems)) != cudaSuccess) return IS_ERR_OOM;
+    s->stage_slot_elems = slot_elems;
+  }
+  return IS_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* is_status_string(int status) {
+  switch (status) {
+    case IS_OK: return "ok";
+    case IS_ERR_INVALID_ARG: return "invalid argument";
+    case IS_ERR_BAD_FACT_ID: return "fact id outside the store";
+    case IS_ERR_POSITION: return "segment runs past the request's block table";
+    case IS_ERR_BAD_BLOCK: return "block-table entry outside the cache";
+    case IS_ERR_CAPACITY: return "capacity exceeded";
+    case IS_ERR_OOM: return "allocation failed";
+    case IS_ERR_CUDA: return "CUDA runtime error";
+    case IS_ERR_TIMEOUT: return "timed out";
+    case IS_ERR_NOT_SUPPORTED: return "not supported";
+    default: return "unknown status";
+  }
+}
+
+int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) {
+  if (!cfg || !out) return IS_ERR_INVALID_ARG;
+  *out = nullptr;
+  const is_store_config_t& c = *cfg;
+  if (c.num_layers < 1 || c.num_kv_heads < 1 || c.head_dim < 2 || c.head_dim % 2) return IS_ERR_INVALID_ARG;
+  if (!(c.rope_theta > 0.0) || (c.rope_style != IS_ROPE_ROTATE_HALF && c.rope_style != IS_ROPE_INTERLEAVED))
+    return IS_ERR_INVALID_ARG;
+  if (c.rope_scaling != IS_SCALING_NONE && c.rope_scaling != IS_SCALING_LLAMA3) return IS_ERR_INVALID_ARG;
+  if (c.rope_scaling == IS_SCALING_LLAMA3 &&
+      (!(c.scale_factor > 0.0) || !(c.low_freq_factor > 0.0) || !(c.high_freq_factor > c.low_freq_factor) ||
+       c.original_max_position <= 0))
+    return IS_ERR_INVALID_ARG;
+  if (c.capacity_tokens < 1 || c.max_facts < 1 || c.max_batch_requests < 0 || c.max_batch_fact_ids < 0 ||
+      c.max_batch_blocks < 0)
+    return IS_ERR_INVALID_ARG;
+  if (c.tier != IS_TIER_DEVICE && c.tier != IS_TIER_HOST) return IS_ERR_INVALID_ARG;
+  if (!head_dim_supported(c.head_dim)) return IS_ERR_NOT_SUPPORTED;
+  if (c.tier == IS_TIER_HOST) return IS_ERR_NOT_SUPPORTED;  // host tier: separate entry points
+  if (c.capacity_tokens > (int64_t(1) << 31) - 1) return IS_ERR_NOT_SUPPORTED;
+
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return IS_ERR_CUDA;
+  DeviceGuard guard(device);
+
+  is_store* s = new (std::nothrow) is_store();
+  if (!s) return IS_ERR_OOM;
+  s->cfg = c;
+  s->device = device;
+  cudaDeviceGetAttribute(&s->sm_count, cudaDevAttrMultiProcessorCount, device);
+  s->max_req = c.max_batch_requests ? c.max_batch_requests : kDefaultMaxRequests;
+  s->max_ids = c.max_batch_fact_ids ? c.max_batch_fact_ids : kDefaultMaxFactIds;
+  s->max_blocks = c.max_batch_blocks ? c.max_batch_blocks
+                                     : int32_t(std::max<int64_t>(65536, int64_t(256) * s->max_req));
+
+  const size_t plane_elems = size_t(c.capacity_tokens) * size_t(c.head_dim);
+  const size_t arena_elems = size_t(c.num_layers) * size_t(c.num_kv_heads) * plane_elems;
+  bool ok = dalloc(&s->k, arena_elems) == cudaSuccess && dalloc(&s->v, arena_elems) == cudaSuccess &&
+            dalloc(&s->d_off, size_t(c.max_facts)) == cudaSuccess &&
+            dalloc(&s->d_len, size_t(c.max_facts)) == cudaSuccess &&
+            dalloc(&s->d_inv_freq, size_t(c.head_dim / 2)) == cudaSuccess &&
+            dalloc(&s->ws_seg, size_t(s->max_ids)) == cudaSuccess &&
+            dalloc(&s->ws_nblk, size_t(s->max_req)) == cudaSuccess &&
+            dalloc(&s->ws_blk0, size_t(s->max_req) + 1) == cudaSuccess &&
+            dalloc(&s->ws_tok0, size_t(s->max_req) + 1) == cudaSuccess &&
+            dalloc(&s->ws_len, size_t(s->max_req)) == cudaSuccess &&
+            dalloc(&s->ws_valid, size_t(s->max_req)) == cudaSuccess &&
+            dalloc(&s->ws_desc, size_t(s->max_blocks)) == cudaSuccess &&
+            dalloc(&s->ws_hdr, 1) == cudaSuccess && dalloc(&s->d_status, 1) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_store(s);
+    return IS_ERR_OOM;
+  }
+  s->h_off.assign(size_t(c.max_facts), 0);
+  s->h_len.assign(size_t(c.max_facts), 0);
+  cudaMemset(s->d_len, 0, sizeof(int32_t) * size_t(c.max_facts));
+  cudaMemset(s->d_off, 0, sizeof(int64_t) * size_t(c.max_facts));
+  cudaMemset(s->d_status, 0, sizeof(isk::DevStatus));
+  cudaMemset(s->ws_hdr, 0, sizeof(isk::PlanHeader));
+  const int nf = c.head_dim / 2;
+  isk::inv_freq_kernel<<<(nf + 127) / 128, 128>>>(
+      s->d_inv_freq, c.head_dim, c.rope_theta, c.rope_scaling, c.scale_factor, c.low_freq_factor,
+      c.high_freq_factor, double(c.original_max_position));
+
+  // Persistent inject grid: resident CTAs per SM x SMs, for the largest
+  // cos/sin table (B = 128) so one grid size serves every block size.
+  const size_t smem_max = cs_smem_bytes(c.head_dim, isk::kMaxBlockSize);
+  for (int variant = 0; variant < 2; ++variant) {
+    void* f = variant ? pick_inject_t<true>(c.head_dim, c.rope_style)
+                      : pick_inject_t<false>(c.head_dim, c.rope_style);
+    cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
+  }
+  void* fn = pick_inject_t<true>(c.head_dim, c.rope_style);
+  int per_sm = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kInjectThreads, cs_smem_bytes(c.head_dim, 16));
+  s->inject_grid = std::max(1, per_sm) * s->sm_count;
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaGetLastError() != cudaSuccess) {
+    free_store(s);
+    return IS_ERR_CUDA;
+  }
+  *out = s;
+  return IS_OK;
+}
+
+void is_store_destroy(is_store_t* s) {
+  if (!s) return;
+  DeviceGuard guard(s->device);
+  cudaDeviceSynchronize();
+  free_store(s);
+}
+
+int is_store_put_fact(is_store_t* s, const void* k_pre, const void* v, int32_t len,
+                      int32_t* fact_id_out) {
+  if (!s || !k_pre || !v || len <= 0) return IS_ERR_INVALID_ARG;
+  if (s->num_facts >= s->cfg.max_facts || s->used_tokens + len > s->cfg.capacity_tokens)
+    return IS_ERR_CAPACITY;
+  DeviceGuard guard(s->device);
+  const is_store_config_t& c = s->cfg;
+  const size_t row = size_t(c.head_dim) * sizeof(uint16_t);
+  const size_t width = size_t(len) * row;                    // one fact run of one plane
+  const size_t dpitch = size_t(c.capacity_tokens) * row;     // distance between planes
+  const size_t height = size_t(c.num_layers) * size_t(c.num_kv_heads);
+  const size_t off_bytes = size_t(s->used_tokens) * row;
+  char* kd = reinterpret_cast<char*>(s->k) + off_bytes;
+  char* vd = reinterpret_cast<char*>(s->v) + off_bytes;
+  const int32_t id = s->num_facts;
+  const int64_t off = s->used_tokens;
+  if (cudaMemcpy2D(kd, dpitch, k_pre, width, width, height, cudaMemcpyDefault) != cudaSuccess ||
+      cudaMemcpy2D(vd, dpitch, v, width, width, height, cudaMemcpyDefault) != cudaSuccess ||
+      cudaMemcpy(s->d_off + id, &off, sizeof(off), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(s->d_len + id, &len, sizeof(len), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaGetLastError();
+    return IS_ERR_CUDA;
+  }
+  s->h_off[size_t(id)] = off;
+  s->h_len[size_t(id)] = len;
+  s->num_facts = id + 1;
+  s->used_tokens = off + len;
+  if (fact_id_out) *fact_id_out = id;
+  return IS_OK;
+}
+
+int is_store_num_facts(const is_store_t* s, int32_t* out) {
+  if (!s || !out) return IS_ERR_INVALID_ARG;
+  *out = s->num_facts;
+  return IS_OK;
+}
+
+int is_store_fact_info(const is_store_t* s, int32_t id, int64_t* off, int32_t* len) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  if (id < 0 || id >= s->num_facts) return IS_ERR_BAD_FACT_ID;
+  if (off) *off = s->h_off[size_t(id)];
+  if (len) *len = s->h_len[size_t(id)];
+  return IS_OK;
+}
+
+int is_store_read_fact(is_store_t* s, int32_t id, void* k_out, void* v_out) {
+  if (!s || (!k_out && !v_out)) return IS_ERR_INVALID_ARG;
+  if (id < 0 || id >= s->num_facts) return IS_ERR_BAD_FACT_ID;
+  DeviceGuard guard(s->device);
+  const is_store_config_t& c = s->cfg;
+  const size_t row = size_t(c.head_dim) * sizeof(uint16_t);
+  const size_t width = size_t(s->h_len[size_t(id)]) * row;
+  const size_t spitch = size_t(c.capacity_tokens) * row;
+  const size_t height = size_t(c.num_layers) * size_t(c.num_kv_heads);
+  const size_t off_bytes = size_t(s->h_off[size_t(id)]) * row;
+  if (k_out && cudaMemcpy2D(k_out, width, reinterpret_cast<char*>(s->k) + off_bytes, spitch, width,
+                            height, cudaMemcpyDefault) != cudaSuccess)
+    return IS_ERR_CUDA;
+  if (v_out && cudaMemcpy2D(v_out, width, reinterpret_cast<char*>(s->v) + off_bytes, spitch, width,
+                            height, cudaMemcpyDefault) != cudaSuccess)
+    return IS_ERR_CUDA;
+  return IS_OK;
+}
+
+int is_store_arena(const is_store_t* s, void** k, void** v, int64_t* plane_tokens) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  if (k) *k = s->k;
+  if (v) *v = s->v;
+  if (plane_tokens) *plane_tokens = s->cfg.capacity_tokens;
+  return IS_OK;
+}
+
+int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int32_t* fact_ids,
+                    int32_t num_ids, const int32_t* start_pos, const int32_t* block_tables,
+                    int32_t max_blocks_per_req, const is_cache_t* cache, int64_t* slot_out,
+                    int64_t slot_cap, void* stream) {
+  if (!s || !cache || R < 0 || num_ids < 0 || max_blocks_per_req < 1) return IS_ERR_INVALID_ARG;
+  if (R > 0 && (!req_off || !start_pos || !block_tables)) return IS_ERR_INVALID_ARG;
+  if (num_ids > 0 && !fact_ids) return IS_ERR_INVALID_ARG;
+  if (R == 0 && !req_off) return IS_ERR_INVALID_ARG;
+  if (R > s->max_req || num_ids > s->max_ids) return IS_ERR_CAPACITY;
+  const is_cache_t& c = *cache;
+  if (!c.k_cache || !c.v_cache || c.num_blocks < 1 || c.block_size < 1 ||
+      c.block_size > isk::kMaxBlockSize)
+    return IS_ERR_INVALID_ARG;
+  if (!aligned16(c.k_cache) || !aligned16(c.v_cache) || c.layer_stride % 8 || c.block_stride % 8 ||
+      c.token_stride % 8 || c.head_stride % 8 || c.layer_stride < 0 || c.block_stride < 0 ||
+      c.token_stride < 0 || c.head_stride < 0)
+    return IS_ERR_INVALID_ARG;
+  if (slot_out && slot_cap < 0) return IS_ERR_INVALID_ARG;
+  if (int64_t(max_blocks_per_req) * c.block_size > (int64_t(1) << 31) - 1) return IS_ERR_NOT_SUPPORTED;
+  DeviceGuard guard(s->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const is_store_config_t& cf = s->cfg;
+
+  isk::PlanArgs pa;
+  pa.R = R;
+  pa.req_off = req_off;
+  pa.fact_ids = fact_ids;
+  pa.num_ids = num_ids;
+  pa.start_pos = start_pos;
+  pa.max_blocks = max_blocks_per_req;
+  pa.B = c.block_size;
+  pa.L = cf.num_layers;
+  pa.fact_len = s->d_len;
+  pa.num_facts = s->num_facts;
+  pa.slot_out = slot_out;
+  pa.slot_cap = slot_cap;
+  pa.grid_ctas = s->inject_grid;
+  pa.max_batch_blocks = s->max_blocks;
+  pa.seg = s->ws_seg;
+  pa.req_nblk = s->ws_nblk;
+  pa.req_blk0 = s->ws_blk0;
+  pa.req_tok0 = s->ws_tok0;
+  pa.req_len = s->ws_len;
+  pa.req_valid = s->ws_valid;
+  pa.desc = s->ws_desc;
+  pa.hdr = s->ws_hdr;
+  pa.st = s->d_status;
+  isk::plan_kernel<kPlanThreads><<<1, kPlanThreads, 0, st>>>(pa);
+
+  isk::InjectArgs ia;
+  ia.k_store = s->k;
+  ia.v_store = s->v;
+  ia.plane = int64_t(cf.capacity_tokens) * cf.head_dim;
+  ia.fact_off = s->d_off;
+  ia.fact_len = s->d_len;
+  ia.inv_freq = s->d_inv_freq;
+  ia.L = cf.num_layers;
+  ia.H = cf.num_kv_heads;
+  ia.req_off = req_off;
+  ia.fact_ids = fact_ids;
+  ia.start_pos = start_pos;
+  ia.block_tables = block_tables;
+  ia.max_blocks = max_blocks_per_req;
+  ia.k_cache = static_cast<uint16_t*>(c.k_cache);
+  ia.v_cache = static_cast<uint16_t*>(c.v_cache);
+  ia.ls = c.layer_stride;
+  ia.bs = c.block_stride;
+  ia.ts = c.token_stride;
+  ia.hs = c.head_stride;
+  ia.num_blocks = c.num_blocks;
+  ia.B = c.block_size;
+  ia.slot_out = slot_out;
+  ia.seg = s->ws_seg;
+  ia.req_tok0 = s->ws_tok0;
+  ia.desc = s->ws_desc;
+  ia.hdr = s->ws_hdr;
+  ia.st = s->d_status;
+  void* fn = pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size);
+  void* args[] = {&ia};
+  TimedLaunch* ev = nullptr;
+  if (s->timing && s->events_used < size_t(kMaxTimedLaunches)) {
+    if (s->events_used == s->events.size()) {
+      TimedLaunch e{};
+      if (cudaEventCreate(&e.start) == cudaSuccess && cudaEventCreate(&e.stop) == cudaSuccess)
+        s->events.push_back(e);
+    }
+    if (s->events_used < s->events.size()) ev = &s->events[s->events_used++];
+  }
+  if (ev) cudaEventRecord(ev->start, st);
+  cudaError_t e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), args,
+                                   cs_smem_bytes(cf.head_dim, c.block_size), st);
+  if (ev) cudaEventRecord(ev->stop, st);
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
+  return IS_OK;
+}
+
+int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const int32_t* fact_ids,
+                         int32_t num_ids, const int32_t* start_pos, const int32_t* block_tables,
+                         int32_t max_blocks_per_req, const is_cache_t* cache, int64_t* slot_out,
+                         int64_t slot_cap, void* stream) {
+  if (!s || !cache || R < 0 || num_ids < 0 || max_blocks_per_req < 1 || !req_off) return IS_ERR_INVALID_ARG;
+  if ((R > 0 && (!start_pos || !block_tables)) || (num_ids > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
+  if (R > s->max_req || num_ids > s->max_ids) return IS_ERR_CAPACITY;
+  if (slot_out && slot_cap < 0) return IS_ERR_INVALID_ARG;
+  DeviceGuard guard(s->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n_off = size_t(R) + 1, n_ids = size_t(num_ids), n_sp = size_t(R);
+  const size_t n_bt = size_t(R) * size_t(max_blocks_per_req);
+  const int64_t n_slots = slot_out ? slot_cap : 0;
+  int rc = grow_stage(s, n_off + n_ids + n_sp + n_bt + 4, n_slots);
+  if (rc != IS_OK) return rc;
+  int32_t* d_off = s->stage;
+  int32_t* d_ids = d_off + n_off;
+  int32_t* d_sp = d_ids + n_ids;
+  int32_t* d_bt = d_sp + n_sp;
+  if (cudaMemcpyAsync(d_off, req_off, n_off * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      (n_ids && cudaMemcpyAsync(d_ids, fact_ids, n_ids * 4, cudaMemcpyHostToDevice, st) != cudaSuccess) ||
+      (n_sp && cudaMemcpyAsync(d_sp, start_pos, n_sp * 4, cudaMemcpyHostToDevice, st) != cudaSuccess) ||
+      (n_bt && cudaMemcpyAsync(d_bt, block_tables, n_bt * 4, cudaMemcpyHostToDevice, st) != cudaSuccess))
+    return IS_ERR_CUDA;
+  rc = is_inject_batch(s, R, d_off, d_ids, num_ids, d_sp, d_bt, max_blocks_per_req, cache,
+                       slot_out ? s->stage_slots : nullptr, slot_cap, stream);
+  if (rc != IS_OK) return rc;
+  if (slot_out && slot_cap > 0 &&
+      cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess)
+    return IS_ERR_CUDA;
+  return is_last_error(s, stream, nullptr);
+}
+
+int is_last_error(is_store_t* s, void* stream, int64_t* detail) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  DeviceGuard guard(s->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  isk::DevStatus h{};
+  if (cudaStreamSynchronize(st) != cudaSuccess) return IS_ERR_CUDA;
+  if (cudaMemcpy(&h, s->d_status, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return IS_ERR_CUDA;
+  if (h.code != 0 && cudaMemset(s->d_status, 0, sizeof(h)) != cudaSuccess) return IS_ERR_CUDA;
+  if (detail) *detail = h.detail;
+  return h.code;
+}
+
+int is_store_set_timing(is_store_t* s, int enable) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  s->timing = enable != 0;
+  return IS_OK;
+}
+
+int is_store_kernel_time(is_store_t* s, double* total_ms, int64_t* launches) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  DeviceGuard guard(s->device);
+  double sum = 0.0;
+  for (size_t i = 0; i < s->events_used; ++i) {
+    if (cudaEventSynchronize(s->events[i].stop) != cudaSuccess) return IS_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, s->events[i].start, s->events[i].stop) != cudaSuccess) return IS_ERR_CUDA;
+    sum += ms;
+  }
+  if (total_ms) *total_ms = sum;
+  if (launches) *launches = int64_t(s->events_used);
+  s->events_used = 0;
+  return IS_OK;
+}
+
+}  // extern "C"

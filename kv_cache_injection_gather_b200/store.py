@@ -1,0 +1,178 @@
+"""Torch-facing convenience over the C-ABI (marshalling only).
+
+``FactStore`` owns one ``is_store_t``; tensors are passed to the library as
+raw device pointers with their strides checked here.  Every byte of the
+inject path is produced by the CUDA kernels in libinjectstore.so.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import binding as B
+
+
+@dataclass
+class RopeConfig:
+    theta: float
+    style: int = B.IS_ROPE_ROTATE_HALF
+    llama3: dict | None = None   # factor, low_freq_factor, high_freq_factor, original_max_position
+
+
+def _i32(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.int32 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 tensor")
+    return t
+
+
+class _DeviceArray:
+    """__cuda_array_interface__ wrapper so torch can view library memory."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = dict(shape=tuple(shape), typestr=typestr,
+                                             data=(ptr, False), version=3, strides=None)
+
+
+def cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor, head_major: bool = False) -> B.is_cache_t:
+    """Describe bf16 caches shaped [L][num_blocks][B][H][D] (token-major) or
+    [L][num_blocks][H][B][D] (head-major) to the library."""
+    for t in (k_cache, v_cache):
+        if t.dtype != torch.bfloat16 or t.dim() != 5 or not t.is_cuda or t.stride(-1) != 1:
+            raise ValueError("caches must be CUDA bf16 [L][num_blocks][.][.][D] with unit last stride")
+    if k_cache.shape != v_cache.shape or k_cache.stride() != v_cache.stride():
+        raise ValueError("K and V caches must share shape and strides")
+    L, nb, a, b, D = k_cache.shape
+    ls, bs, sa, sb, _ = k_cache.stride()
+    if head_major:
+        H, blk, hs, ts = a, b, sa, sb
+    else:
+        blk, H, ts, hs = a, b, sa, sb
+    return B.is_cache_t(k_cache.data_ptr(), v_cache.data_ptr(), ls, bs, ts, hs, nb, blk)
+
+
+class FactStore:
+    """A GPU-resident fact store of pre-RoPE keys and raw values."""
+
+    def __init__(self, num_layers: int, num_kv_heads: int, head_dim: int, rope: RopeConfig,
+                 capacity_tokens: int, max_facts: int, device: int = 0,
+                 max_batch_requests: int = 0, max_batch_fact_ids: int = 0,
+                 max_batch_blocks: int = 0):
+        cfg = B.is_store_config_t()
+        cfg.num_layers, cfg.num_kv_heads, cfg.head_dim = num_layers, num_kv_heads, head_dim
+        cfg.rope_style, cfg.rope_theta = rope.style, rope.theta
+        if rope.llama3:
+            cfg.rope_scaling = B.IS_SCALING_LLAMA3
+            cfg.scale_factor = rope.llama3["factor"]
+            cfg.low_freq_factor = rope.llama3["low_freq_factor"]
+            cfg.high_freq_factor = rope.llama3["high_freq_factor"]
+            cfg.original_max_position = int(rope.llama3["original_max_position"])
+        cfg.capacity_tokens, cfg.max_facts = capacity_tokens, max_facts
+        cfg.max_batch_requests, cfg.max_batch_fact_ids = max_batch_requests, max_batch_fact_ids
+        cfg.max_batch_blocks = max_batch_blocks
+        cfg.tier = B.IS_TIER_DEVICE
+        self.L, self.H, self.D = num_layers, num_kv_heads, head_dim
+        self.device = device
+        self.capacity_tokens = capacity_tokens
+        self.handle = B.is_store_create(cfg, device)
+
+    # ---- lifetime
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            B.is_store_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # ---- facts
+    def put_fact(self, k_pre: torch.Tensor, v: torch.Tensor) -> int:
+        """k_pre, v: bf16 [L][H][len][D] on the host or this device."""
+        if k_pre.shape != v.shape or k_pre.dim() != 4 or k_pre.shape[0] != self.L \
+                or k_pre.shape[1] != self.H or k_pre.shape[3] != self.D:
+            raise ValueError("fact must be [L][H][len][D]")
+        if k_pre.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+            raise ValueError("fact tensors must be bf16")
+        k_pre, v = k_pre.contiguous(), v.contiguous()
+        return B.is_store_put_fact(self.handle, k_pre.data_ptr(), v.data_ptr(), k_pre.shape[2])
+
+    @property
+    def num_facts(self) -> int:
+        return B.is_store_num_facts(self.handle)
+
+    def fact_info(self, fact_id: int) -> tuple[int, int]:
+        return B.is_store_fact_info(self.handle, fact_id)
+
+    def read_fact(self, fact_id: int) -> tuple[torch.Tensor, torch.Tensor]:
+        _, n = self.fact_info(fact_id)
+        dev = torch.device("cuda", self.device)
+        k = torch.empty((self.L, self.H, n, self.D), dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        B.is_store_read_fact(self.handle, fact_id, k.data_ptr(), v.data_ptr())
+        return k, v
+
+    def arena(self) -> tuple[torch.Tensor, torch.Tensor]:
+        """Views of the K and V arenas as bf16 [L][H][capacity_tokens][D]."""
+        kp, vp, t = B.is_store_arena(self.handle)
+        shape = (self.L, self.H, t, self.D)
+        dev = torch.device("cuda", self.device)
+        k = torch.as_tensor(_DeviceArray(kp, shape, "<i2"), device=dev).view(torch.bfloat16)
+        v = torch.as_tensor(_DeviceArray(vp, shape, "<i2"), device=dev).view(torch.bfloat16)
+        return k, v
+
+    # ---- the hot path
+    def inject(self, req_offsets: torch.Tensor, fact_ids: torch.Tensor, start_pos: torch.Tensor,
+               block_tables: torch.Tensor, cache: B.is_cache_t,
+               slot_mapping: torch.Tensor | None = None, stream: int | None = None) -> None:
+        """Asynchronous inject of one batch; all index tensors on the device."""
+        _i32(req_offsets, "req_offsets"), _i32(fact_ids, "fact_ids")
+        _i32(start_pos, "start_pos"), _i32(block_tables, "block_tables")
+        R = start_pos.numel()
+        if block_tables.dim() != 2 or block_tables.shape[0] != R:
+            raise ValueError("block_tables must be [R][max_blocks]")
+        if slot_mapping is not None and (slot_mapping.dtype != torch.int64 or not slot_mapping.is_contiguous()):
+            raise ValueError("slot_mapping must be contiguous int64")
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device).cuda_stream
+        B.is_inject_batch(self.handle, R, req_offsets.data_ptr(), fact_ids.data_ptr(),
+                          fact_ids.numel(), start_pos.data_ptr(), block_tables.data_ptr(),
+                          block_tables.shape[1], cache,
+                          None if slot_mapping is None else slot_mapping.data_ptr(),
+                          0 if slot_mapping is None else slot_mapping.numel(), stream)
+
+    def inject_host(self, req_offsets: torch.Tensor, fact_ids: torch.Tensor,
+                    start_pos: torch.Tensor, block_tables: torch.Tensor, cache: B.is_cache_t,
+                    slot_mapping: torch.Tensor | None = None, stream: int | None = None) -> int:
+        """Index tensors in host memory (pinned for asynchronous copies);
+        waits and returns the batch status."""
+        for t in (req_offsets, fact_ids, start_pos, block_tables):
+            if t.is_cuda:
+                raise ValueError("inject_host takes host tensors")
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device).cuda_stream
+        return B.is_inject_batch_host(
+            self.handle, start_pos.numel(), req_offsets.data_ptr(), fact_ids.data_ptr(),
+            fact_ids.numel(), start_pos.data_ptr(), block_tables.data_ptr(),
+            block_tables.shape[1], cache,
+            None if slot_mapping is None else slot_mapping.data_ptr(),
+            0 if slot_mapping is None else slot_mapping.numel(), stream)
+
+    def last_error(self, stream: int | None = None) -> tuple[int, int]:
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device).cuda_stream
+        return B.is_last_error(self.handle, stream)
+
+    def set_timing(self, enable: bool) -> None:
+        B.is_store_set_timing(self.handle, enable)
+
+    def kernel_time(self) -> tuple[float, int]:
+        return B.is_store_kernel_time(self.handle)

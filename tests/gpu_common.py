@@ -1,0 +1,87 @@
+"""Helpers shared by the GPU tests, the smoke check and the benchmark:
+building a FactStore and a paged cache from a seeded synthetic workload.
+
+Input generation only (synth), plus marshalling into the library; no part
+of the inject arithmetic lives here.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+from kv_cache_injection_gather_b200 import FactStore, RopeConfig, cache_desc
+
+CACHE_FILL_SEED = 7
+
+
+def rope_of(model: synth.Model, style: int = 0) -> RopeConfig:
+    return RopeConfig(theta=model.rope_theta, style=style, llama3=model.scaling())
+
+
+def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = None,
+               device: int = 0, extra_tokens: int = 0, **limits) -> FactStore:
+    """Put every fact of the workload, in id order (ids equal indices).
+
+    Small stores are generated on the host (numpy) and copied; large ones are
+    generated on the device by the same counter-based definition."""
+    m = wl.model
+    total = int(wl.fact_lens.sum()) + extra_tokens
+    store = FactStore(m.num_layers, m.num_kv_heads, m.head_dim, rope_of(m, style), total,
+                      len(wl.fact_lens), device=device, **limits)
+    if on_device_gen is None:
+        on_device_gen = total * m.bytes_per_token > (64 << 20)
+    dev = torch.device("cuda", device)
+    if on_device_gen:
+        maxlen = int(wl.fact_lens.max())
+        kbuf = torch.empty(m.num_layers * m.num_kv_heads * maxlen * m.head_dim,
+                           dtype=torch.bfloat16, device=dev)
+        vbuf = torch.empty_like(kbuf)
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        for f, n in enumerate(wl.fact_lens):
+            n = int(n)
+            cnt = m.num_layers * m.num_kv_heads * n * m.head_dim
+            synth.fill_device(kbuf.data_ptr(), cnt, wl.seed, synth.fact_stream(f, False), 0, stream)
+            synth.fill_device(vbuf.data_ptr(), cnt, wl.seed, synth.fact_stream(f, True), 0, stream)
+            shape = (m.num_layers, m.num_kv_heads, n, m.head_dim)
+            fid = store.put_fact(kbuf[:cnt].view(shape), vbuf[:cnt].view(shape))
+            assert fid == f
+        torch.cuda.synchronize(dev)
+    else:
+        for f, n in enumerate(wl.fact_lens):
+            k, v = synth.fact_kv(wl.seed, f, m.num_layers, m.num_kv_heads, int(n), m.head_dim)
+            kt = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16)
+            vt = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16)
+            assert store.put_fact(kt, vt) == f
+    return store
+
+
+def cache_shape(wl: synth.Workload, head_major: bool = False):
+    m, b = wl.model, wl.batch
+    if head_major:
+        return (m.num_layers, b.num_blocks, m.num_kv_heads, b.block_size, m.head_dim)
+    return (m.num_layers, b.num_blocks, b.block_size, m.num_kv_heads, m.head_dim)
+
+
+def make_cache(wl: synth.Workload, device: int = 0, fill: bool = True, head_major: bool = False):
+    """K and V caches (bf16, device); filled with seeded values so untouched
+    slots can be checked, or left uninitialised."""
+    shape = cache_shape(wl, head_major)
+    dev = torch.device("cuda", device)
+    k = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    v = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    if fill:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        synth.fill_device(k.data_ptr(), k.numel(), CACHE_FILL_SEED, synth.TAG_CACHE | 0, 0, stream)
+        synth.fill_device(v.data_ptr(), v.numel(), CACHE_FILL_SEED, synth.TAG_CACHE | 1, 0, stream)
+    return k, v, cache_desc(k, v, head_major)
+
+
+def batch_tensors(batch: synth.Batch, device: int = 0):
+    dev = torch.device("cuda", device)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)  # noqa: E731
+    return (t(batch.req_offsets), t(batch.fact_ids), t(batch.start_pos), t(batch.block_tables))
+
+
+def to_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().view(torch.int16).cpu().numpy().view(np.uint16)

@@ -1,0 +1,299 @@
+"""GPU path (through the C-ABI) against the CPU oracle on the same seeded
+inputs.
+
+Bar: V, slot mapping and every untouched cache element bit-exact; rotated K
+within |err| <= 2^-8 |ref| + 1e-3 elementwise, ref = the oracle's fp64
+rotation before rounding (the stated tolerance; one bf16 rounding alone
+stays inside it, a rounding flip next to a midpoint too).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_common import (CACHE_FILL_SEED, batch_tensors, make_cache, make_store, to_bits)
+from kv_cache_injection_gather_b200 import binding as B
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 2.0 ** -8, 1e-3
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+# ------------------------------------------------------------------ oracle side
+
+def oracle_run(wl: synth.Workload, style=0, head_major=False, slot_capacity=None):
+    m, b = wl.model, wl.batch
+    st = oracle.Store(m.num_layers, m.num_kv_heads, m.head_dim, max(int(wl.fact_lens.sum()), 1),
+                      len(wl.fact_lens))
+    for f, n in enumerate(wl.fact_lens):
+        st.put(*synth.fact_kv(wl.seed, f, m.num_layers, m.num_kv_heads, int(n), m.head_dim))
+    shape = ((m.num_layers, b.num_blocks, m.num_kv_heads, b.block_size, m.head_dim) if head_major
+             else (m.num_layers, b.num_blocks, b.block_size, m.num_kv_heads, m.head_dim))
+    kc = synth.bf16_block(CACHE_FILL_SEED, synth.TAG_CACHE | 0, shape)
+    vc = synth.bf16_block(CACHE_FILL_SEED, synth.TAG_CACHE | 1, shape)
+    kref = np.full(shape, np.nan)
+    strides = oracle.cache_strides(b.num_blocks, b.block_size, m.num_kv_heads, m.head_dim,
+                                   head_major)
+    f = oracle.rope_inv_freq(m.head_dim, m.rope_theta, m.scaling())
+    rc, slots = oracle.inject_batch(st, f, b.req_offsets, b.fact_ids, b.start_pos, b.block_tables,
+                                    kc, vc, b.block_size, strides=strides, style=style, k_ref=kref,
+                                    slot_capacity=slot_capacity)
+    return rc, slots, kc, vc, kref
+
+
+def gpu_run(wl: synth.Workload, style=0, head_major=False, slot_capacity=None, store=None):
+    _need_gpu()
+    own = store is None
+    if own:
+        store = make_store(wl, style)
+    k, v, desc = make_cache(wl, head_major=head_major)
+    ro, ids, sp, bt = batch_tensors(wl.batch)
+    n_tok = int(wl.fact_lens[wl.batch.fact_ids[(wl.batch.fact_ids >= 0) &
+                                               (wl.batch.fact_ids < len(wl.fact_lens))]].sum())
+    cap = n_tok if slot_capacity is None else slot_capacity
+    slots = torch.full((max(cap, 1),), -7, dtype=torch.int64, device="cuda")
+    store.inject(ro, ids, sp, bt, desc, slots[:cap] if cap else slots[:0])
+    rc, _ = store.last_error()
+    out = rc, slots[:cap].cpu().numpy(), to_bits(k), to_bits(v)
+    if own:
+        store.close()
+    return out
+
+
+def assert_parity(o, g):
+    orc, oslots, okc, ovc, kref = o
+    grc, gslots, gkc, gvc = g
+    assert grc == orc
+    assert np.array_equal(gslots[: len(oslots)], oslots)
+    assert np.array_equal(gvc, ovc), "V or untouched V slots differ"
+    written = ~np.isnan(kref)
+    assert np.array_equal(gkc[~written], okc[~written]), "untouched K slots changed"
+    got = oracle.bf16_to_f64(gkc[written])
+    ref = kref[written]
+    err = np.abs(got - ref)
+    bad = err > REL * np.abs(ref) + ABS
+    assert not bad.any(), f"{bad.sum()} K elements out of tolerance, max err {err.max()}"
+    exact = np.mean(gkc[written] == okc[written]) if written.any() else 1.0
+    assert exact > 0.999, f"only {exact:.5f} of K bit-identical to the oracle's rounding"
+    return exact
+
+
+# ------------------------------------------------------------------ tests
+
+def test_device_generator_matches_host():
+    _need_gpu()
+    n = 1 << 20
+    t = torch.empty(n, dtype=torch.int16, device="cuda")
+    synth.fill_device(t.data_ptr(), n, 123, synth.fact_stream(77, True), 5000,
+                      torch.cuda.current_stream().cuda_stream)
+    host = synth.bf16_bits(123, synth.fact_stream(77, True), np.arange(5000, 5000 + n))
+    assert np.array_equal(t.cpu().numpy().view(np.uint16), host)
+
+
+@pytest.mark.parametrize("style", [0, 1])
+@pytest.mark.parametrize("start", [32, 37, 0])
+def test_tiny_parity(start, style):
+    wl = synth.tiny(0, start_pos=start)
+    assert_parity(oracle_run(wl, style), gpu_run(wl, style))
+
+
+def _ragged(model, seed, B=16, R=7, max_k=9, lens=(1, 40), num_facts=40, starts=None,
+            spare_blocks=3):
+    rng = np.random.default_rng(seed)
+    fl = rng.integers(lens[0], lens[1] + 1, num_facts).astype(np.int32)
+    ids = [rng.choice(num_facts, int(rng.integers(0, max_k + 1)), replace=True) for _ in range(R)]
+    if R > 1:
+        ids[1] = np.zeros(0, np.int64)  # an empty request
+    sp = (rng.integers(0, 70, R) if starts is None else np.asarray(starts)).astype(np.int32)
+    need = max(-(-(int(sp[r]) + int(fl[ids[r]].sum())) // B) for r in range(R)) + spare_blocks
+    batch = synth.make_batch(rng, ids, sp, B, R * need, need)
+    return synth.Workload("ragged", model, fl, batch, seed)
+
+
+SHAPES = [
+    # name, L, H, D, theta, llama3, B, style, head_major
+    ("llama-like", 3, 8, 128, 5e5, True, 16, 0, False),
+    ("qwen-like", 2, 4, 128, 1e6, False, 16, 0, False),
+    ("interleaved", 2, 4, 128, 1e4, False, 16, 1, False),
+    ("head-major", 2, 8, 128, 5e5, True, 16, 0, True),
+    ("h3-generic", 2, 3, 128, 1e4, False, 16, 0, False),
+    ("d64-b8", 2, 2, 64, 1e4, False, 8, 0, False),
+    ("d256-b32", 1, 2, 256, 1e4, False, 32, 1, False),
+    ("d32-b1", 2, 1, 32, 1e4, False, 1, 0, False),
+    ("b128", 1, 2, 64, 1e4, False, 128, 0, False),
+    ("b12-generic", 2, 2, 64, 1e4, False, 12, 0, True),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
+def test_ragged_batches_parity(shape):
+    name, L, H, D, theta, ll3, B_, style, hm = shape
+    model = synth.Model(name, L, H, D, theta, llama3=ll3)
+    wl = _ragged(model, seed=sum(name.encode()), B=B_)
+    assert_parity(oracle_run(wl, style, hm), gpu_run(wl, style, hm))
+
+
+def test_long_segments_many_blocks():
+    """Facts longer than several blocks; positions up to ~5k (fp32 angle range
+    the kernel must handle with fp64 angles)."""
+    model = synth.Model("long", 2, 2, 128, 5e5, llama3=True)
+    wl = _ragged(model, seed=3, R=3, max_k=6, lens=(100, 400), num_facts=12,
+                 starts=[0, 3000, 4097])
+    assert_parity(oracle_run(wl), gpu_run(wl))
+
+
+def test_empty_batch_and_empty_requests():
+    model = synth.Model("e", 1, 2, 64, 1e4)
+    rng = np.random.default_rng(0)
+    fl = rng.integers(1, 20, 10).astype(np.int32)
+    b0 = synth.make_batch(rng, [], np.zeros(0), 16, 4, 1)
+    wl0 = synth.Workload("empty", model, fl, b0)
+    assert_parity(oracle_run(wl0), gpu_run(wl0))
+    b1 = synth.make_batch(rng, [np.zeros(0, int)] * 3, [5, 0, 16], 16, 6, 2)
+    wl1 = synth.Workload("empty-requests", model, fl, b1)
+    assert_parity(oracle_run(wl1), gpu_run(wl1))
+
+
+def _error_wl(kind):
+    wl = synth.tiny(0)
+    b = wl.batch
+    ids = np.concatenate([b.fact_ids[:2], b.fact_ids[2:4]]).astype(np.int32)
+    ro = np.array([0, 2, 4], np.int32)
+    sp = np.array([0, 40], np.int32)
+    bt = np.stack([np.arange(0, 20), np.arange(20, 40)]).astype(np.int32)
+    if kind == "bad_fact":
+        ids[2] = 9999
+    elif kind == "position":
+        sp[1] = 20 * 16 - 3
+    elif kind == "bad_block":
+        bt[1, 3] = 64
+    elif kind == "negative_block":
+        bt[0, 0] = -5
+    elif kind == "negative_start":
+        sp[0] = -1
+    elif kind == "csr":
+        ro = np.array([0, 2, 3], np.int32)
+    elif kind == "csr_range":
+        # request 0 ends past the id list, request 1 ends before it starts
+        ro = np.array([0, 5, 4], np.int32)
+    batch = synth.Batch(ro, ids, sp, bt, 16, 64)
+    return synth.Workload("err-" + kind, wl.model, wl.fact_lens, batch, wl.seed)
+
+
+@pytest.mark.parametrize("kind", ["bad_fact", "position", "bad_block", "negative_block",
+                                  "negative_start", "csr", "csr_range"])
+def test_device_errors_match_oracle(kind):
+    wl = _error_wl(kind)
+    o = oracle_run(wl)
+    assert o[0] != oracle.OK
+    assert_parity(o, gpu_run(wl))
+
+
+def test_slot_capacity_error_writes_nothing():
+    wl = synth.tiny(0)
+    o = oracle_run(wl, slot_capacity=3)
+    g = gpu_run(wl, slot_capacity=3)
+    assert o[0] == g[0] == oracle.ERR_CAPACITY
+    assert np.array_equal(g[2], o[2]) and np.array_equal(g[3], o[3])
+
+
+def test_host_entry_point_matches_device_entry_point():
+    _need_gpu()
+    wl = _ragged(synth.Model("h", 2, 4, 128, 1e6), seed=11)
+    store = make_store(wl)
+    b = wl.batch
+    n_tok = int(wl.fact_lens[b.fact_ids].sum())
+    k1, v1, d1 = make_cache(wl)
+    k2, v2, d2 = make_cache(wl)
+    ro, ids, sp, bt = batch_tensors(b)
+    s1 = torch.empty(n_tok, dtype=torch.int64, device="cuda")
+    store.inject(ro, ids, sp, bt, d1, s1)
+    assert store.last_error()[0] == 0
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
+    s2 = torch.empty(n_tok, dtype=torch.int64).pin_memory()
+    rc = store.inject_host(pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos),
+                           pin(b.block_tables), d2, s2)
+    assert rc == 0
+    assert torch.equal(k1, k2) and torch.equal(v1, v2)
+    assert torch.equal(s1.cpu(), s2)
+    store.close()
+
+
+def test_store_put_read_and_arena():
+    _need_gpu()
+    wl = synth.tiny(0)
+    m = wl.model
+    store = make_store(wl)
+    ka, va = store.arena()
+    for f in (0, 5, 63):
+        off, n = store.fact_info(f)
+        k, v = synth.fact_kv(wl.seed, f, m.num_layers, m.num_kv_heads, n, m.head_dim)
+        kr, vr = store.read_fact(f)
+        assert np.array_equal(to_bits(kr), k) and np.array_equal(to_bits(vr), v)
+        assert np.array_equal(to_bits(ka[:, :, off:off + n]), k)
+        assert np.array_equal(to_bits(va[:, :, off:off + n]), v)
+    assert store.num_facts == 64
+    with pytest.raises(B.InjectError):
+        store.fact_info(64)
+    store.close()
+
+
+def test_repeatable_and_stream_ordered():
+    """Two batches in a row on a side stream give identical bytes; the timing
+    hook counts one launch per batch."""
+    _need_gpu()
+    wl = _ragged(synth.Model("r", 2, 8, 128, 5e5, llama3=True), seed=5)
+    store = make_store(wl)
+    s = torch.cuda.Stream()
+    k, v, d = make_cache(wl)
+    k2, v2, d2 = make_cache(wl)
+    ro, ids, sp, bt = batch_tensors(wl.batch)
+    torch.cuda.synchronize()
+    store.set_timing(True)
+    with torch.cuda.stream(s):
+        store.inject(ro, ids, sp, bt, d)
+        store.inject(ro, ids, sp, bt, d2)
+    assert store.last_error(s.cuda_stream)[0] == 0
+    ms, n = store.kernel_time()
+    assert n == 2 and ms > 0
+    assert torch.equal(k, k2) and torch.equal(v, v2)
+    store.close()
+
+
+def test_llama_single_request_full_store():
+    """Llama-3.1-8B shapes, 10k facts of 16-64 tokens (about 52 GB of store),
+    one request of k=5 after a 64-token prefix; whole cache compared."""
+    _need_gpu()
+    wl = synth.llama_single(0)
+    store = make_store(wl, on_device_gen=True)
+    g = gpu_run(wl, store=store)
+    store.close()
+    # the oracle needs only the five injected facts: renumber them 0..4
+    ids = wl.batch.fact_ids
+    sub = synth.Workload(wl.name, wl.model, wl.fact_lens[ids],
+                         synth.Batch(wl.batch.req_offsets, np.arange(len(ids), dtype=np.int32),
+                                     wl.batch.start_pos, wl.batch.block_tables,
+                                     wl.batch.block_size, wl.batch.num_blocks), wl.seed)
+    # regenerate the injected facts under their original ids
+    m = wl.model
+    st = oracle.Store(m.num_layers, m.num_kv_heads, m.head_dim, int(sub.fact_lens.sum()), len(ids))
+    for f in ids:
+        st.put(*synth.fact_kv(wl.seed, int(f), m.num_layers, m.num_kv_heads,
+                              int(wl.fact_lens[f]), m.head_dim))
+    b = sub.batch
+    shape = (m.num_layers, b.num_blocks, b.block_size, m.num_kv_heads, m.head_dim)
+    kc = synth.bf16_block(CACHE_FILL_SEED, synth.TAG_CACHE | 0, shape)
+    vc = synth.bf16_block(CACHE_FILL_SEED, synth.TAG_CACHE | 1, shape)
+    kref = np.full(shape, np.nan)
+    f = oracle.rope_inv_freq(m.head_dim, m.rope_theta, m.scaling())
+    rc, slots = oracle.inject_batch(st, f, b.req_offsets, b.fact_ids, b.start_pos, b.block_tables,
+                                    kc, vc, b.block_size, k_ref=kref)
+    assert_parity((rc, slots, kc, vc, kref), g)
