@@ -211,27 +211,45 @@ def cpu_baseline(wl, device, budget_s=15.0):
 
 # ------------------------------------------------------------------ main
 
-def workload_config(wl, extra=None):
+WORKLOADS = {
+    # name: (description, builder)
+    "llama-batch": ("llama3.1-8b-shapes 10k-fact store, 100 requests x k=50, block 16, "
+                    "cache 25600 blocks", lambda seed: _synth().llama_batch(seed)),
+    "llama-batch-small": ("llama3.1-8b-shapes 500-fact store, 10 requests x k=20, block 16, "
+                          "cache 640 blocks (profiling case, ~4 GB on the device)",
+                          lambda seed: _synth().llama_batch(seed, num_facts=500, R=10, k=20,
+                                                            slots_per_request=1024)),
+    "llama-single": ("llama3.1-8b-shapes 10k-fact store, 1 request x k=5, block 16, 64 blocks",
+                     lambda seed: _synth().llama_single(seed)),
+}
+
+
+def _synth():
+    import synth
+    return synth
+
+
+def workload_config(wl, name="llama-batch", extra=None):
     m, b = wl.model, wl.batch
-    cfg = {"workload": "llama3.1-8b-shapes 10k-fact store, 100 requests x k=50, block 16, "
-                       "cache 25600 blocks",
+    cfg = {"workload": WORKLOADS[name][0],
            "model_shapes": m.name, "layers": m.num_layers, "kv_heads": m.num_kv_heads,
            "head_dim": m.head_dim, "rope": "theta 5e5, llama3 scaling (8, 1, 4, 8192)",
            "requests": b.num_requests, "k": int(b.req_offsets[1] - b.req_offsets[0]),
            "facts": len(wl.fact_lens), "fact_len": "uniform 16..64",
+           "store_gb": round(float(wl.fact_lens.sum()) * m.bytes_per_token / 1e9, 2),
            "tokens_per_batch": wl.tokens(), "block_size": b.block_size,
            "num_blocks": b.num_blocks, "start_pos": 64,
-           "l2": "inputs larger than L2 (26 GB read + 26 GB written per step)"}
+           "l2": f"inputs larger than L2 ({wl.tokens() * m.bytes_per_token / 1e9:.1f} GB read + "
+                 f"the same written per step, L2 126 MB)"}
     if extra:
         cfg.update(extra)
     return cfg
 
 
 def run_reference(args, rank, world):
-    import synth
     if rank != 0:
         return 0
-    wl = synth.llama_batch(0)
+    wl = WORKLOADS[args.workload][1](0)
     sample_args, tok = oracle_sample(wl, [0], None if not _cuda() else 0)
     import oracle
     threads = oracle.max_threads()
@@ -244,7 +262,8 @@ def run_reference(args, rank, world):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(wl, {"reference_step": "request 0 of the batch"}),
+            "config": workload_config(wl, args.workload,
+                                      {"reference_step": "request 0 of the batch"}),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                              "kind": "oracle",
                              "sample": f"request 0 of the batch ({tok} tokens, all layers and "
@@ -267,7 +286,6 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    import synth
     from gpu_common import batch_tensors, make_cache, make_store
     from kv_cache_injection_gather_b200 import binding as B
 
@@ -275,7 +293,7 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("bench.py needs a CUDA device (the inject path has no CPU fallback)")
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = synth.llama_batch(seed=rank)
+    wl = WORKLOADS[args.workload][1](rank)
     m, b = wl.model, wl.batch
     store = make_store(wl, on_device_gen=True, device=local_rank)
     kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False)
@@ -364,7 +382,8 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": workload_config(wl, {"parallelism": f"replicas x{world}"}),
+        "data": "synthetic",
+        "config": workload_config(wl, args.workload, {"parallelism": f"replicas x{world}"}),
         "us_per_batch": ms_step * 1e3,
         "gbs_per_gpu": algo_bytes / (ms_step / 1e3) / 1e9,
         "kernel_us": kern_avg_ms * 1e3,
@@ -392,6 +411,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama-batch",
+                    help="llama-batch is the benchmark; the others are smaller cases for "
+                         "profiling and latency")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
