@@ -213,6 +213,67 @@ int is_store_kernel_time(is_store_t* store, double* total_ms_out, int64_t* launc
 /* Human-readable name of a status code (static string). */
 const char* is_status_string(int status);
 
+/* ---- allocation-free variant ------------------------------------------- */
+
+/* Limits of is_inject_batch_noalloc (its fixed work space). */
+#define IS_NOALLOC_MAX_REQUESTS 1024
+#define IS_NOALLOC_MAX_FACT_IDS 65536
+#define IS_NOALLOC_MAX_BLOCKS 65536   /* touched cache blocks per batch */
+#define IS_NOALLOC_MAX_HEAD_DIM 256
+
+/* The inject batch of is_inject_batch for callers that cannot allocate
+ * device memory.  The paper has no counterpart: this is a deployment
+ * variant of the same plan and inject kernels, not a step of the method.
+ *
+ * Who needs it: code that runs where cudaMalloc is off limits -- inside a
+ * serving engine whose memory pool already owns the whole GPU (a call to
+ * cudaMalloc would fail or fragment the pool), in a region the engine is
+ * recording into a CUDA graph, or in a plugin whose host may not create
+ * allocations behind its back.  Such a caller cannot create an is_store_t
+ * (creation allocates), so it passes the store's contents itself.
+ *
+ * The per-batch work space (segment offsets, per-request sums, block
+ * descriptors, plan header, status word, RoPE frequencies) lives in one
+ * fixed array of about 1.3 MB in the library's device globals, which every
+ * GPU that loads the library keeps until the process exits.  The call
+ * itself calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments:
+ *   cfg           num_layers, num_kv_heads, head_dim (<= 256) and the RoPE
+ *                 fields as for is_store_create; the capacity, batch-limit
+ *                 and tier fields are ignored
+ *   k_store, v_store  device bf16 arenas [L][H][plane_tokens][D]
+ *   fact_offsets  device int64 [num_facts]: first token of each fact in
+ *                 every plane
+ *   fact_lens     device int32 [num_facts]
+ *   the batch arguments, cache and slot mapping as for is_inject_batch
+ *   status_out    optional device buffer of 16 bytes that receives the
+ *                 batch's device status: int32 code (an IS_* value), int32
+ *                 padding, int64 detail (as is_last_error's detail)
+ *   stream        as for is_inject_batch; the work is asynchronous
+ * The device is the current device; every pointer must be on it.
+ *
+ * Limits: num_requests <= IS_NOALLOC_MAX_REQUESTS and num_fact_ids <=
+ * IS_NOALLOC_MAX_FACT_IDS, else IS_ERR_CAPACITY is returned and nothing is
+ * launched; a batch that touches more than IS_NOALLOC_MAX_BLOCKS cache
+ * blocks writes nothing and reports IS_ERR_CAPACITY in status_out.
+ *
+ * The first call on a device looks up the work space's device address
+ * (cudaGetSymbolAddress) and the kernels' launch settings; make that first
+ * call before any stream capture.  All calls share the one work space and
+ * each starts by clearing its status word: calls whose work overlaps on the
+ * GPU (two streams, two host threads) race and must be ordered by the
+ * caller, for instance by issuing them on one stream. */
+int is_inject_batch_noalloc(const is_store_config_t* cfg, const void* k_store,
+                            const void* v_store, int64_t plane_tokens,
+                            const int64_t* fact_offsets, const int32_t* fact_lens,
+                            int32_t num_facts, int32_t num_requests,
+                            const int32_t* req_fact_offsets, const int32_t* fact_ids,
+                            int32_t num_fact_ids, const int32_t* start_pos,
+                            const int32_t* block_tables, int32_t max_blocks_per_req,
+                            const is_cache_t* cache, int64_t* slot_mapping_out,
+                            int64_t slot_mapping_capacity, void* status_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

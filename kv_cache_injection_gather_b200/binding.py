@@ -32,6 +32,11 @@ IS_SCALING_LLAMA3 = 1
 IS_TIER_DEVICE = 0
 IS_TIER_HOST = 1
 
+IS_NOALLOC_MAX_REQUESTS = 1024
+IS_NOALLOC_MAX_FACT_IDS = 65536
+IS_NOALLOC_MAX_BLOCKS = 65536
+IS_NOALLOC_MAX_HEAD_DIM = 256
+
 _I32, _I64, _F64, _P = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
 
 
@@ -84,6 +89,9 @@ _SIGNATURES = {
     "is_store_set_timing": (ctypes.c_int, [_P, ctypes.c_int]),
     "is_store_kernel_time": (ctypes.c_int, [_P, ctypes.POINTER(_F64), ctypes.POINTER(_I64)]),
     "is_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "is_inject_batch_noalloc": (ctypes.c_int, [ctypes.POINTER(is_store_config_t), _P, _P, _I64,
+                                               _P, _P, _I32, _I32, _P, _P, _I32, _P, _P, _I32,
+                                               ctypes.POINTER(is_cache_t), _P, _I64, _P, _P]),
 }
 for _name, (_res, _args) in _SIGNATURES.items():
     _fn = getattr(_lib, _name)
@@ -191,3 +199,22 @@ def is_store_kernel_time(store: int) -> tuple[float, int]:
 
 def is_status_string(status: int) -> str:
     return status_string(status)
+
+
+def is_inject_batch_noalloc(cfg: is_store_config_t, k_store: int, v_store: int,
+                            plane_tokens: int, fact_offsets: int, fact_lens: int, num_facts: int,
+                            num_requests: int, req_fact_offsets: int, fact_ids: int,
+                            num_fact_ids: int, start_pos: int, block_tables: int,
+                            max_blocks_per_req: int, cache: is_cache_t,
+                            slot_mapping_out: int | None, slot_mapping_capacity: int,
+                            status_out: int | None, stream: int = 0) -> int:
+    """The batch for callers that cannot allocate device memory: the store's
+    arenas and fact table are passed in, the work space is the library's
+    fixed device array.  Asynchronous; returns the host-side status
+    without raising.  The device status lands in status_out (16 bytes)."""
+    return _lib.is_inject_batch_noalloc(ctypes.byref(cfg), k_store, v_store, plane_tokens,
+                                        fact_offsets, fact_lens, num_facts, num_requests,
+                                        req_fact_offsets, fact_ids, num_fact_ids, start_pos,
+                                        block_tables, max_blocks_per_req, ctypes.byref(cache),
+                                        slot_mapping_out, slot_mapping_capacity, status_out,
+                                        stream)

@@ -510,3 +510,213 @@ int is_store_kernel_time(is_store_t* s, double* total_ms, int64_t* launches) {
 }
 
 }  // extern "C"
+
+// ===================================================================
+// Allocation-free entry point (is_inject_batch_noalloc).
+//
+// For callers that must not allocate device memory (an engine whose pool
+// owns the GPU, a region being captured into a CUDA graph, a plugin host
+// that forbids hidden allocations).  The per-batch work space is one fixed
+// device array in this module; the same plan and inject kernels as
+// is_inject_batch run on it.
+// ===================================================================
+
+#include <mutex>
+
+namespace {
+
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Work-space layout, byte offsets into g_noalloc_scratch.
+constexpr size_t kNaStatus = 0;
+constexpr size_t kNaHeader = align256(kNaStatus + sizeof(isk::DevStatus));
+constexpr size_t kNaInvFreq = align256(kNaHeader + sizeof(isk::PlanHeader));
+constexpr size_t kNaSeg = align256(kNaInvFreq + sizeof(double) * (IS_NOALLOC_MAX_HEAD_DIM / 2));
+constexpr size_t kNaNblk = align256(kNaSeg + sizeof(int32_t) * IS_NOALLOC_MAX_FACT_IDS);
+constexpr size_t kNaBlk0 = align256(kNaNblk + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
+constexpr size_t kNaTok0 = align256(kNaBlk0 + sizeof(int32_t) * (IS_NOALLOC_MAX_REQUESTS + 1));
+constexpr size_t kNaLen = align256(kNaTok0 + sizeof(long long) * (IS_NOALLOC_MAX_REQUESTS + 1));
+constexpr size_t kNaValid = align256(kNaLen + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
+constexpr size_t kNaDesc = align256(kNaValid + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
+constexpr size_t kNaBytes = align256(kNaDesc + sizeof(isk::BlockDesc) * IS_NOALLOC_MAX_BLOCKS);
+
+constexpr int kNaMaxDevices = 64;
+
+// Per-device launch settings, filled by the first call on the device.
+struct NoAllocDevice {
+  bool ready = false;
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
+  int grid[4][2] = {};               // inject grid per head-dim slot and RoPE style
+};
+
+NoAllocDevice g_na_devices[kNaMaxDevices];
+std::mutex g_na_mutex;
+
+int head_dim_slot(int d) { return d == 32 ? 0 : d == 64 ? 1 : d == 128 ? 2 : 3; }
+
+}  // namespace
+
+// The work space: one array per GPU that loads this library, kept until exit.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
+
+namespace {
+
+// Once per device, with that device current: the work space's device
+// address (host code cannot use the symbol itself as an address) and the
+// kernels' shared-memory limits and resident-CTA grid sizes.
+int noalloc_setup(int dev, NoAllocDevice** out) {
+  std::lock_guard<std::mutex> lock(g_na_mutex);
+  NoAllocDevice& d = g_na_devices[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return IS_ERR_CUDA;
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return IS_ERR_CUDA;
+    const int dims[4] = {32, 64, 128, 256};
+    for (int di = 0; di < 4; ++di)
+      for (int style = 0; style < 2; ++style) {
+        const int D = dims[di];
+        const size_t smem_max = cs_smem_bytes(D, isk::kMaxBlockSize);
+        void* f_pow2 = pick_inject_t<true>(D, style);
+        void* f_gen = pick_inject_t<false>(D, style);
+        if (cudaFuncSetAttribute(f_pow2, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max)) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(f_gen, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max)) !=
+                cudaSuccess)
+          return IS_ERR_CUDA;
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f_pow2, kInjectThreads,
+                                                          cs_smem_bytes(D, 16)) != cudaSuccess)
+          return IS_ERR_CUDA;
+        d.grid[di][style] = std::max(1, per_sm) * sms;
+      }
+    d.scratch = static_cast<unsigned char*>(p);
+    d.ready = true;
+  }
+  *out = &d;
+  return IS_OK;
+}
+
+}  // namespace
+
+extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void* k_store,
+                                       const void* v_store, int64_t plane_tokens,
+                                       const int64_t* fact_offsets, const int32_t* fact_lens,
+                                       int32_t num_facts, int32_t R, const int32_t* req_off,
+                                       const int32_t* fact_ids, int32_t num_ids,
+                                       const int32_t* start_pos, const int32_t* block_tables,
+                                       int32_t max_blocks_per_req, const is_cache_t* cache,
+                                       int64_t* slot_out, int64_t slot_cap, void* status_out,
+                                       void* stream) {
+  if (!cfg || !cache || !k_store || !v_store || plane_tokens < 1 || num_facts < 0 || R < 0 ||
+      num_ids < 0 || max_blocks_per_req < 1 || !req_off)
+    return IS_ERR_INVALID_ARG;
+  if (num_facts > 0 && (!fact_offsets || !fact_lens)) return IS_ERR_INVALID_ARG;
+  if ((R > 0 && (!start_pos || !block_tables)) || (num_ids > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
+  const is_store_config_t& c = *cfg;
+  if (c.num_layers < 1 || c.num_kv_heads < 1 || !(c.rope_theta > 0.0) ||
+      (c.rope_style != IS_ROPE_ROTATE_HALF && c.rope_style != IS_ROPE_INTERLEAVED) ||
+      (c.rope_scaling != IS_SCALING_NONE && c.rope_scaling != IS_SCALING_LLAMA3))
+    return IS_ERR_INVALID_ARG;
+  if (c.rope_scaling == IS_SCALING_LLAMA3 &&
+      (!(c.scale_factor > 0.0) || !(c.low_freq_factor > 0.0) || !(c.high_freq_factor > c.low_freq_factor) ||
+       c.original_max_position <= 0))
+    return IS_ERR_INVALID_ARG;
+  if (!head_dim_supported(c.head_dim) || c.head_dim > IS_NOALLOC_MAX_HEAD_DIM) return IS_ERR_NOT_SUPPORTED;
+  if (R > IS_NOALLOC_MAX_REQUESTS || num_ids > IS_NOALLOC_MAX_FACT_IDS) return IS_ERR_CAPACITY;
+  const is_cache_t& k = *cache;
+  if (!k.k_cache || !k.v_cache || k.num_blocks < 1 || k.block_size < 1 || k.block_size > isk::kMaxBlockSize)
+    return IS_ERR_INVALID_ARG;
+  if (!aligned16(k.k_cache) || !aligned16(k.v_cache) || !aligned16(k_store) || !aligned16(v_store) ||
+      k.layer_stride % 8 || k.block_stride % 8 || k.token_stride % 8 || k.head_stride % 8 ||
+      k.layer_stride < 0 || k.block_stride < 0 || k.token_stride < 0 || k.head_stride < 0)
+    return IS_ERR_INVALID_ARG;
+  if (slot_out && slot_cap < 0) return IS_ERR_INVALID_ARG;
+  if (int64_t(max_blocks_per_req) * k.block_size > (int64_t(1) << 31) - 1) return IS_ERR_NOT_SUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNaMaxDevices) return IS_ERR_CUDA;
+  NoAllocDevice* nd = nullptr;
+  int rc = noalloc_setup(dev, &nd);
+  if (rc != IS_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = nd->scratch;
+  auto* status = reinterpret_cast<isk::DevStatus*>(ws + kNaStatus);
+  auto* hdr = reinterpret_cast<isk::PlanHeader*>(ws + kNaHeader);
+  auto* inv_freq = reinterpret_cast<double*>(ws + kNaInvFreq);
+
+  // The status word is the only field read before it is written: clear it.
+  if (cudaMemsetAsync(status, 0, sizeof(isk::DevStatus), st) != cudaSuccess) return IS_ERR_CUDA;
+  const int nf = c.head_dim / 2;
+  isk::inv_freq_kernel<<<(nf + 127) / 128, 128, 0, st>>>(
+      inv_freq, c.head_dim, c.rope_theta, c.rope_scaling, c.scale_factor, c.low_freq_factor,
+      c.high_freq_factor, double(c.original_max_position));
+
+  const int grid = nd->grid[head_dim_slot(c.head_dim)][c.rope_style];
+  isk::PlanArgs pa;
+  pa.R = R;
+  pa.req_off = req_off;
+  pa.fact_ids = fact_ids;
+  pa.num_ids = num_ids;
+  pa.start_pos = start_pos;
+  pa.max_blocks = max_blocks_per_req;
+  pa.B = k.block_size;
+  pa.L = c.num_layers;
+  pa.fact_len = fact_lens;
+  pa.num_facts = num_facts;
+  pa.slot_out = slot_out;
+  pa.slot_cap = slot_cap;
+  pa.grid_ctas = grid;
+  pa.max_batch_blocks = IS_NOALLOC_MAX_BLOCKS;
+  pa.seg = reinterpret_cast<int32_t*>(ws + kNaSeg);
+  pa.req_nblk = reinterpret_cast<int32_t*>(ws + kNaNblk);
+  pa.req_blk0 = reinterpret_cast<int32_t*>(ws + kNaBlk0);
+  pa.req_tok0 = reinterpret_cast<long long*>(ws + kNaTok0);
+  pa.req_len = reinterpret_cast<int32_t*>(ws + kNaLen);
+  pa.req_valid = reinterpret_cast<int32_t*>(ws + kNaValid);
+  pa.desc = reinterpret_cast<isk::BlockDesc*>(ws + kNaDesc);
+  pa.hdr = hdr;
+  pa.st = status;
+  isk::plan_kernel<kPlanThreads><<<1, kPlanThreads, 0, st>>>(pa);
+
+  isk::InjectArgs ia;
+  ia.k_store = static_cast<const uint16_t*>(k_store);
+  ia.v_store = static_cast<const uint16_t*>(v_store);
+  ia.plane = plane_tokens * c.head_dim;
+  ia.fact_off = fact_offsets;
+  ia.fact_len = fact_lens;
+  ia.inv_freq = inv_freq;
+  ia.L = c.num_layers;
+  ia.H = c.num_kv_heads;
+  ia.req_off = req_off;
+  ia.fact_ids = fact_ids;
+  ia.start_pos = start_pos;
+  ia.block_tables = block_tables;
+  ia.max_blocks = max_blocks_per_req;
+  ia.k_cache = static_cast<uint16_t*>(k.k_cache);
+  ia.v_cache = static_cast<uint16_t*>(k.v_cache);
+  ia.ls = k.layer_stride;
+  ia.bs = k.block_stride;
+  ia.ts = k.token_stride;
+  ia.hs = k.head_stride;
+  ia.num_blocks = k.num_blocks;
+  ia.B = k.block_size;
+  ia.slot_out = slot_out;
+  ia.seg = pa.seg;
+  ia.req_tok0 = pa.req_tok0;
+  ia.desc = pa.desc;
+  ia.hdr = hdr;
+  ia.st = status;
+  void* fn = pick_inject(c.head_dim, c.rope_style, c.num_kv_heads, k.block_size);
+  void* args[] = {&ia};
+  if (cudaLaunchKernel(fn, dim3(unsigned(grid)), dim3(kInjectThreads), args,
+                       cs_smem_bytes(c.head_dim, k.block_size), st) != cudaSuccess)
+    return IS_ERR_CUDA;
+  if (status_out && cudaMemcpyAsync(status_out, status, sizeof(isk::DevStatus),
+                                    cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return IS_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? IS_OK : IS_ERR_CUDA;
+}
