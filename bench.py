@@ -282,6 +282,18 @@ def _cuda():
         return False
 
 
+def max_over_ranks(values, world):
+    """Element-wise max of per-rank numbers (timings) over all ranks."""
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.is_initialized() and \
+        dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -363,10 +375,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
 
     # ---- max over ranks
-    vals = torch.tensor([ms, e2e_ms, kern_ms / max(kern_n, 1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, kern_avg_ms = vals.tolist()
+    ms, e2e_ms, kern_avg_ms = max_over_ranks([ms, e2e_ms, kern_ms / max(kern_n, 1)], world)
     ms_step = ms / args.steps
     tokens_all = n_tok * world
     value = tokens_all / (ms_step / 1e3)

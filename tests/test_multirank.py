@@ -1,0 +1,123 @@
+"""The multi-GPU partitions on CPU: world_size-2 gloo ranks, the CPU oracle
+standing in for each rank's GPU.  Head shards and request shards each
+reproduce the single-rank result with no data exchange; the benchmark's
+max-over-ranks timing reduction works across processes."""
+from __future__ import annotations
+
+import os
+import socket
+import tempfile
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _tiny_multi(seed=0):
+    import synth
+    rng = np.random.default_rng(seed)
+    model = synth.Model("m", 2, 4, 64, 1e4)
+    lens = rng.integers(5, 30, 20).astype(np.int32)
+    ids = [rng.choice(20, int(rng.integers(1, 6)), replace=False) for _ in range(5)]
+    batch = synth.make_batch(rng, ids, rng.integers(0, 40, 5), 16, 5 * 12, 12)
+    return synth.Workload("m", model, lens, batch, seed)
+
+
+def _oracle_inject(wl, heads=None, batch=None):
+    import oracle
+    import synth
+    m = wl.model
+    b = batch or (wl.batch.req_offsets, wl.batch.fact_ids, wl.batch.start_pos, wl.batch.block_tables)
+    h0, h1 = heads or (0, m.num_kv_heads)
+    H = h1 - h0
+    st = oracle.Store(m.num_layers, H, m.head_dim, int(wl.fact_lens.sum()), len(wl.fact_lens))
+    for f, n in enumerate(wl.fact_lens):
+        k, v = synth.fact_kv(wl.seed, f, m.num_layers, m.num_kv_heads, int(n), m.head_dim)
+        st.put(k[:, h0:h1], v[:, h0:h1])
+    shape = (m.num_layers, wl.batch.num_blocks, wl.batch.block_size, H, m.head_dim)
+    kc, vc = np.zeros(shape, np.uint16), np.zeros(shape, np.uint16)
+    rc, slots = oracle.inject_batch(st, oracle.rope_inv_freq(m.head_dim, m.rope_theta), *b, kc, vc,
+                                    wl.batch.block_size)
+    assert rc == 0
+    return kc, vc, slots
+
+
+def _worker(rank, world, port, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        from kv_cache_injection_gather_b200 import shard
+        wl = _tiny_multi()
+        m = wl.model
+        # head shards: each rank computes its heads of every layer and slot
+        h0, h1 = shard.head_shard(m.num_kv_heads, world, rank)
+        kc, vc, _ = _oracle_inject(wl, heads=(h0, h1))
+        parts = [None] * world
+        dist.all_gather_object(parts, (h0, h1, kc, vc))
+        # request shards: each rank injects its own requests into the cache
+        b = wl.batch
+        sub = shard.request_shard(b.req_offsets, b.fact_ids, b.start_pos, b.block_tables, world, rank)
+        kr, vr, sr = _oracle_inject(wl, batch=sub[:4])
+        rparts = [None] * world
+        dist.all_gather_object(rparts, (kr, vr, sr))
+        # max over ranks of the step time, as the benchmark reports it
+        got = bench.max_over_ranks([10.0 + rank, 3.0 * (1 - rank)], world)
+        if rank == 0:
+            np.save(os.path.join(out_dir, "heads.npy"), np.array(parts, dtype=object), allow_pickle=True)
+            np.save(os.path.join(out_dir, "reqs.npy"), np.array(rparts, dtype=object), allow_pickle=True)
+            np.save(os.path.join(out_dir, "max.npy"), np.array(got))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_partitions_reproduce_single_rank_with_gloo():
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_worker, args=(world, _free_port(), d), nprocs=world, join=True,
+                           start_method="spawn")
+        heads = np.load(os.path.join(d, "heads.npy"), allow_pickle=True)
+        reqs = np.load(os.path.join(d, "reqs.npy"), allow_pickle=True)
+        mx = np.load(os.path.join(d, "max.npy"))
+    wl = _tiny_multi()
+    kf, vf, sf = _oracle_inject(wl)
+    # head shards concatenate to the full cache
+    k_cat = np.concatenate([p[2] for p in heads], axis=3)
+    v_cat = np.concatenate([p[3] for p in heads], axis=3)
+    assert np.array_equal(k_cat, kf) and np.array_equal(v_cat, vf)
+    # request shards write disjoint slots whose union is the full result
+    assert np.array_equal(np.concatenate([p[2] for p in reqs]), sf)
+    k_u, v_u = np.zeros_like(kf), np.zeros_like(vf)
+    for kr, vr, sr in reqs:
+        flat_k, flat_v = kr.reshape(kr.shape[0], -1, *kr.shape[3:]), vr.reshape(vr.shape[0], -1, *vr.shape[3:])
+        k_u.reshape(flat_k.shape)[:, sr] = flat_k[:, sr]
+        v_u.reshape(flat_v.shape)[:, sr] = flat_v[:, sr]
+    assert np.array_equal(k_u, kf) and np.array_equal(v_u, vf)
+    assert list(mx) == [11.0, 3.0]
+
+
+def test_contiguous_ranges_cover_everything():
+    from kv_cache_injection_gather_b200 import shard
+    for n in (0, 1, 5, 8, 101):
+        for w in (1, 2, 3, 8):
+            spans = [shard.contiguous_range(n, w, r) for r in range(w)]
+            assert spans[0][0] == 0 and spans[-1][1] == n
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+    with pytest.raises(ValueError):
+        shard.head_shard(8, 3, 0)
