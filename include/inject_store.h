@@ -133,6 +133,23 @@ int is_store_fact_info(const is_store_t* store, int32_t fact_id, int64_t* offset
  * destination; synchronous).  Errors: INVALID_ARG, BAD_FACT_ID, CUDA. */
 int is_store_read_fact(is_store_t* store, int32_t fact_id, void* k_out, void* v_out);
 
+/* Host tier (IS_TIER_HOST) only: choose the facts whose K/V are also kept in
+ * the HBM hot arenas (capacity hot_capacity_tokens per plane), the rest
+ * being read from pinned host memory over the host link while a batch runs
+ * (technical summary, Results, "Scalability": the KV store can be moved to
+ * host DRAM when GPU memory is too small).  fact_ids (host array, n
+ * entries; repeats ignored) replaces the previous hot set; the facts are
+ * copied in list order.  Waits for the device to go idle first, so no batch
+ * reads a half-updated set.  Errors: NOT_SUPPORTED (device tier),
+ * BAD_FACT_ID, CAPACITY (more tokens than the hot arenas hold; the old set
+ * is kept), INVALID_ARG, CUDA. */
+int is_store_set_hot(is_store_t* store, const int32_t* fact_ids, int32_t n);
+
+/* Tier of the store, hot-arena capacity and use (tokens per plane), and the
+ * number of hot facts (0 for a device-tier store). */
+int is_store_tier_info(const is_store_t* store, int32_t* tier_out, int64_t* hot_capacity_out,
+                       int64_t* hot_used_out, int32_t* hot_facts_out);
+
 /* Device addresses of the K and V arenas and the plane stride in tokens
  * (for callers that fill or inspect the store in place).  For
  * IS_TIER_HOST these are the device-mapped addresses of the host arenas. */

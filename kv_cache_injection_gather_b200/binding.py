@@ -89,6 +89,9 @@ _SIGNATURES = {
     "is_store_set_timing": (ctypes.c_int, [_P, ctypes.c_int]),
     "is_store_kernel_time": (ctypes.c_int, [_P, ctypes.POINTER(_F64), ctypes.POINTER(_I64)]),
     "is_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "is_store_set_hot": (ctypes.c_int, [_P, _P, _I32]),
+    "is_store_tier_info": (ctypes.c_int, [_P, ctypes.POINTER(_I32), ctypes.POINTER(_I64),
+                                          ctypes.POINTER(_I64), ctypes.POINTER(_I32)]),
     "is_inject_batch_noalloc": (ctypes.c_int, [ctypes.POINTER(is_store_config_t), _P, _P, _I64,
                                                _P, _P, _I32, _I32, _P, _P, _I32, _P, _P, _I32,
                                                ctypes.POINTER(is_cache_t), _P, _I64, _P, _P]),
@@ -199,6 +202,17 @@ def is_store_kernel_time(store: int) -> tuple[float, int]:
 
 def is_status_string(status: int) -> str:
     return status_string(status)
+
+
+def is_store_set_hot(store: int, fact_ids_host_ptr: int, n: int) -> None:
+    check(_lib.is_store_set_hot(store, fact_ids_host_ptr, n), "is_store_set_hot")
+
+
+def is_store_tier_info(store: int) -> tuple[int, int, int, int]:
+    t, cap, used, nf = _I32(), _I64(), _I64(), _I32()
+    check(_lib.is_store_tier_info(store, ctypes.byref(t), ctypes.byref(cap), ctypes.byref(used),
+                                  ctypes.byref(nf)), "is_store_tier_info")
+    return t.value, cap.value, used.value, nf.value
 
 
 def is_inject_batch_noalloc(cfg: is_store_config_t, k_store: int, v_store: int,

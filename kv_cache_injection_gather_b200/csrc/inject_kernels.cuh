@@ -284,6 +284,12 @@ struct InjectArgs {
   const BlockDesc* desc;
   PlanHeader* hdr;
   DevStatus* st;
+  // host tier only: the arenas above are device-mapped pinned host memory,
+  // and facts with hot_off[f] >= 0 are also held in these HBM arenas
+  const uint16_t* k_hot;     // [L][H][hot_cap][D]
+  const uint16_t* v_hot;
+  int64_t hot_plane;         // hot_cap * D
+  const int64_t* hot_off;    // [num_facts], -1 when the fact is not in HBM
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
@@ -398,13 +404,19 @@ __device__ __forceinline__ int ilog2(int x) { return 31 - __clz(x); }
 // h * D/8 + c (layer, in-block slot, head, 16-byte vector of the row), so
 // consecutive threads write consecutive 16-byte words of the token-major
 // cache and read whole 256-byte head rows of the store.  POW2: H and B are
-// powers of two (all index splits are shifts).
-template <int D, int STYLE, int NT, int VPT, bool POW2>
+// powers of two (all index splits are shifts).  HOST_TIER: the store lives
+// in pinned host memory read over the host link, except the facts that also
+// sit in the HBM hot arenas; the source of every slot is chosen per fact.
+template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER>
 __global__ void __launch_bounds__(NT, 2) inject_kernel(InjectArgs a) {
   constexpr int VPR = D / 8;  // 16-byte vectors per head row
   constexpr int LOG_VPR = (VPR == 4) ? 2 : (VPR == 8) ? 3 : (VPR == 16) ? 4 : 5;
   extern __shared__ float4 s_cs4[];            // [B * D/4] cos/sin of the block
   __shared__ long long s_src[kMaxBlockSize];  // store token of each slot (-1: none)
+  // host tier: per-slot K/V row bases (token offset applied) and plane stride
+  __shared__ const uint16_t* s_kb[HOST_TIER ? kMaxBlockSize : 1];
+  __shared__ const uint16_t* s_vb[HOST_TIER ? kMaxBlockSize : 1];
+  __shared__ long long s_pl[HOST_TIER ? kMaxBlockSize : 1];
   __shared__ int s_unit;
 
   const int tid = threadIdx.x;
@@ -453,7 +465,21 @@ __global__ void __launch_bounds__(NT, 2) inject_kernel(InjectArgs a) {
         const int i = blk_pos + o - start;  // segment index
         int j = d.j;
         while (j + 1 < j1 && a.seg[j + 1] <= i) ++j;
-        src = a.fact_off[a.fact_ids[j]] + (i - a.seg[j]);
+        const int f = a.fact_ids[j];
+        const int t = i - a.seg[j];
+        src = a.fact_off[f] + t;
+        if (HOST_TIER) {
+          const long long ho = a.hot_off[f];
+          if (ho >= 0) {
+            s_kb[o] = a.k_hot + (ho + t) * D;
+            s_vb[o] = a.v_hot + (ho + t) * D;
+            s_pl[o] = a.hot_plane;
+          } else {
+            s_kb[o] = a.k_store + src * D;
+            s_vb[o] = a.v_store + src * D;
+            s_pl[o] = a.plane;
+          }
+        }
         if (lg == 0 && a.slot_out) a.slot_out[tok0 + i] = phys_ok ? (long long)phys * B + o : -1;
       }
       s_src[o] = src;
@@ -486,10 +512,16 @@ __global__ void __launch_bounds__(NT, 2) inject_kernel(InjectArgs a) {
         kv[q] = make_uint4(0, 0, 0, 0);
         vv[q] = kv[q];
         if (src >= 0) {
-          const long long so = (long long)(l * H + (hv >> LOG_VPR)) * a.plane + src * D +
-                               (hv & (VPR - 1)) * 8;
-          kv[q] = ld_stream(kst + so);
-          vv[q] = ld_stream(vst + so);
+          if (HOST_TIER) {
+            const long long so = (long long)(l * H + (hv >> LOG_VPR)) * s_pl[o] + (hv & (VPR - 1)) * 8;
+            kv[q] = ld_stream(s_kb[o] + so);
+            vv[q] = ld_stream(s_vb[o] + so);
+          } else {
+            const long long so = (long long)(l * H + (hv >> LOG_VPR)) * a.plane + src * D +
+                                 (hv & (VPR - 1)) * 8;
+            kv[q] = ld_stream(kst + so);
+            vv[q] = ld_stream(vst + so);
+          }
         }
       }
 #pragma unroll

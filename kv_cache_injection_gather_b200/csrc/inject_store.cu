@@ -34,6 +34,16 @@ struct is_store {
   uint16_t* k = nullptr;
   uint16_t* v = nullptr;
   bool host_arena = false;
+  // host tier: device-mapped views of the pinned arenas and the HBM hot set
+  uint16_t* k_view = nullptr;
+  uint16_t* v_view = nullptr;
+  uint16_t* k_hot = nullptr;
+  uint16_t* v_hot = nullptr;
+  int64_t hot_cap = 0;
+  int64_t hot_used = 0;
+  int32_t hot_facts = 0;
+  int64_t* d_hot = nullptr;
+  std::vector<int64_t> h_hot;
   // fact table
   int64_t* d_off = nullptr;
   int32_t* d_len = nullptr;
@@ -100,6 +110,9 @@ void free_store(is_store* s) {
   cudaFree(s->d_status);
   cudaFree(s->stage);
   cudaFree(s->stage_slots);
+  cudaFree(s->k_hot);
+  cudaFree(s->v_hot);
+  cudaFree(s->d_hot);
   if (s->host_arena) {
     cudaFreeHost(s->k);
     cudaFreeHost(s->v);
@@ -116,18 +129,19 @@ void free_store(is_store* s) {
 
 bool head_dim_supported(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
 
-template <int D, int STYLE, bool POW2>
+template <int D, int STYLE, bool POW2, bool HOST_TIER>
 void* inject_fn() {
-  return reinterpret_cast<void*>(&isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, POW2>);
+  return reinterpret_cast<void*>(
+      &isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, POW2, HOST_TIER>);
 }
 
-template <bool POW2>
+template <bool POW2, bool HOST_TIER = false>
 void* pick_inject_t(int D, int style) {
   switch (D) {
-    case 32: return style ? inject_fn<32, 1, POW2>() : inject_fn<32, 0, POW2>();
-    case 64: return style ? inject_fn<64, 1, POW2>() : inject_fn<64, 0, POW2>();
-    case 128: return style ? inject_fn<128, 1, POW2>() : inject_fn<128, 0, POW2>();
-    case 256: return style ? inject_fn<256, 1, POW2>() : inject_fn<256, 0, POW2>();
+    case 32: return style ? inject_fn<32, 1, POW2, HOST_TIER>() : inject_fn<32, 0, POW2, HOST_TIER>();
+    case 64: return style ? inject_fn<64, 1, POW2, HOST_TIER>() : inject_fn<64, 0, POW2, HOST_TIER>();
+    case 128: return style ? inject_fn<128, 1, POW2, HOST_TIER>() : inject_fn<128, 0, POW2, HOST_TIER>();
+    case 256: return style ? inject_fn<256, 1, POW2, HOST_TIER>() : inject_fn<256, 0, POW2, HOST_TIER>();
     default: return nullptr;
   }
 }
@@ -135,9 +149,12 @@ void* pick_inject_t(int D, int style) {
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 // The inject kernel for a head dim, RoPE style and (H, B): the shift variant
-// when both are powers of two.
-void* pick_inject(int D, int style, int H, int B) {
-  return (is_pow2(H) && is_pow2(B)) ? pick_inject_t<true>(D, style) : pick_inject_t<false>(D, style);
+// when both are powers of two; the host-tier variant for stores in pinned
+// host memory.
+void* pick_inject(int D, int style, int H, int B, bool host_tier = false) {
+  const bool p2 = is_pow2(H) && is_pow2(B);
+  if (host_tier) return p2 ? pick_inject_t<true, true>(D, style) : pick_inject_t<false, true>(D, style);
+  return p2 ? pick_inject_t<true>(D, style) : pick_inject_t<false>(D, style);
 }
 
 size_t cs_smem_bytes(int D, int B) { return size_t(B) * size_t(D / 2) * sizeof(float2); }
@@ -199,7 +216,7 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
     return IS_ERR_INVALID_ARG;
   if (c.tier != IS_TIER_DEVICE && c.tier != IS_TIER_HOST) return IS_ERR_INVALID_ARG;
   if (!head_dim_supported(c.head_dim)) return IS_ERR_NOT_SUPPORTED;
-  if (c.tier == IS_TIER_HOST) return IS_ERR_NOT_SUPPORTED;  // host tier: separate entry points
+  if (c.tier == IS_TIER_HOST && c.hot_capacity_tokens < 0) return IS_ERR_INVALID_ARG;
   if (c.capacity_tokens > (int64_t(1) << 31) - 1) return IS_ERR_NOT_SUPPORTED;
 
   int ndev = 0;
@@ -218,8 +235,30 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
 
   const size_t plane_elems = size_t(c.capacity_tokens) * size_t(c.head_dim);
   const size_t arena_elems = size_t(c.num_layers) * size_t(c.num_kv_heads) * plane_elems;
-  bool ok = dalloc(&s->k, arena_elems) == cudaSuccess && dalloc(&s->v, arena_elems) == cudaSuccess &&
-            dalloc(&s->d_off, size_t(c.max_facts)) == cudaSuccess &&
+  bool ok = true;
+  if (c.tier == IS_TIER_HOST) {
+    // Pinned, device-mapped host arenas; reads cross the host link.
+    s->host_arena = true;
+    const size_t bytes = arena_elems * sizeof(uint16_t);
+    ok = cudaHostAlloc(reinterpret_cast<void**>(&s->k), bytes, cudaHostAllocMapped | cudaHostAllocPortable) ==
+             cudaSuccess &&
+         cudaHostAlloc(reinterpret_cast<void**>(&s->v), bytes, cudaHostAllocMapped | cudaHostAllocPortable) ==
+             cudaSuccess &&
+         cudaHostGetDevicePointer(reinterpret_cast<void**>(&s->k_view), s->k, 0) == cudaSuccess &&
+         cudaHostGetDevicePointer(reinterpret_cast<void**>(&s->v_view), s->v, 0) == cudaSuccess;
+    s->hot_cap = c.hot_capacity_tokens;
+    const size_t hot_elems = size_t(c.num_layers) * size_t(c.num_kv_heads) * size_t(s->hot_cap) * size_t(c.head_dim);
+    ok = ok && (s->hot_cap == 0 ||
+                (dalloc(&s->k_hot, hot_elems) == cudaSuccess && dalloc(&s->v_hot, hot_elems) == cudaSuccess));
+    ok = ok && dalloc(&s->d_hot, size_t(c.max_facts)) == cudaSuccess &&
+         cudaMemset(s->d_hot, 0xFF, sizeof(int64_t) * size_t(c.max_facts)) == cudaSuccess;
+    if (ok) s->h_hot.assign(size_t(c.max_facts), -1);
+  } else {
+    ok = dalloc(&s->k, arena_elems) == cudaSuccess && dalloc(&s->v, arena_elems) == cudaSuccess;
+    s->k_view = s->k;
+    s->v_view = s->v;
+  }
+  ok = ok && dalloc(&s->d_off, size_t(c.max_facts)) == cudaSuccess &&
             dalloc(&s->d_len, size_t(c.max_facts)) == cudaSuccess &&
             dalloc(&s->d_inv_freq, size_t(c.head_dim / 2)) == cudaSuccess &&
             dalloc(&s->ws_seg, size_t(s->max_ids)) == cudaSuccess &&
@@ -249,11 +288,10 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
   // Persistent inject grid: resident CTAs per SM x SMs, for the largest
   // cos/sin table (B = 128) so one grid size serves every block size.
   const size_t smem_max = cs_smem_bytes(c.head_dim, isk::kMaxBlockSize);
-  for (int variant = 0; variant < 2; ++variant) {
-    void* f = variant ? pick_inject_t<true>(c.head_dim, c.rope_style)
-                      : pick_inject_t<false>(c.head_dim, c.rope_style);
-    cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
-  }
+  void* variants[4] = {pick_inject_t<true>(c.head_dim, c.rope_style), pick_inject_t<false>(c.head_dim, c.rope_style),
+                       pick_inject_t<true, true>(c.head_dim, c.rope_style),
+                       pick_inject_t<false, true>(c.head_dim, c.rope_style)};
+  for (void* f : variants) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
   void* fn = pick_inject_t<true>(c.head_dim, c.rope_style);
   int per_sm = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kInjectThreads, cs_smem_bytes(c.head_dim, 16));
@@ -339,9 +377,59 @@ int is_store_read_fact(is_store_t* s, int32_t id, void* k_out, void* v_out) {
 
 int is_store_arena(const is_store_t* s, void** k, void** v, int64_t* plane_tokens) {
   if (!s) return IS_ERR_INVALID_ARG;
-  if (k) *k = s->k;
-  if (v) *v = s->v;
+  if (k) *k = s->k_view;
+  if (v) *v = s->v_view;
   if (plane_tokens) *plane_tokens = s->cfg.capacity_tokens;
+  return IS_OK;
+}
+
+int is_store_set_hot(is_store_t* s, const int32_t* fact_ids, int32_t n) {
+  if (!s || n < 0 || (n > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
+  if (!s->host_arena) return IS_ERR_NOT_SUPPORTED;
+  std::vector<int64_t> hot(size_t(s->cfg.max_facts), -1);
+  int64_t used = 0;
+  int32_t count = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t f = fact_ids[i];
+    if (f < 0 || f >= s->num_facts) return IS_ERR_BAD_FACT_ID;
+    if (hot[size_t(f)] >= 0) continue;  // listed twice
+    if (used + s->h_len[size_t(f)] > s->hot_cap) return IS_ERR_CAPACITY;
+    hot[size_t(f)] = used;
+    used += s->h_len[size_t(f)];
+    ++count;
+  }
+  DeviceGuard guard(s->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return IS_ERR_CUDA;  // no batch may read the old set
+  const is_store_config_t& c = s->cfg;
+  const size_t row = size_t(c.head_dim) * sizeof(uint16_t);
+  const size_t height = size_t(c.num_layers) * size_t(c.num_kv_heads);
+  for (int32_t f = 0; f < s->num_facts; ++f) {
+    if (hot[size_t(f)] < 0) continue;
+    const size_t width = size_t(s->h_len[size_t(f)]) * row;
+    const size_t src_off = size_t(s->h_off[size_t(f)]) * row, dst_off = size_t(hot[size_t(f)]) * row;
+    if (cudaMemcpy2D(reinterpret_cast<char*>(s->k_hot) + dst_off, size_t(s->hot_cap) * row,
+                     reinterpret_cast<const char*>(s->k) + src_off, size_t(c.capacity_tokens) * row, width,
+                     height, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy2D(reinterpret_cast<char*>(s->v_hot) + dst_off, size_t(s->hot_cap) * row,
+                     reinterpret_cast<const char*>(s->v) + src_off, size_t(c.capacity_tokens) * row, width,
+                     height, cudaMemcpyHostToDevice) != cudaSuccess)
+      return IS_ERR_CUDA;
+  }
+  if (cudaMemcpy(s->d_hot, hot.data(), sizeof(int64_t) * hot.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+    return IS_ERR_CUDA;
+  s->h_hot.swap(hot);
+  s->hot_used = used;
+  s->hot_facts = count;
+  return IS_OK;
+}
+
+int is_store_tier_info(const is_store_t* s, int32_t* tier, int64_t* hot_capacity, int64_t* hot_used,
+                       int32_t* hot_facts) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  if (tier) *tier = s->host_arena ? IS_TIER_HOST : IS_TIER_DEVICE;
+  if (hot_capacity) *hot_capacity = s->hot_cap;
+  if (hot_used) *hot_used = s->hot_used;
+  if (hot_facts) *hot_facts = s->hot_facts;
   return IS_OK;
 }
 
@@ -395,8 +483,12 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   isk::plan_kernel<kPlanThreads><<<1, kPlanThreads, 0, st>>>(pa);
 
   isk::InjectArgs ia;
-  ia.k_store = s->k;
-  ia.v_store = s->v;
+  ia.k_store = s->k_view;
+  ia.v_store = s->v_view;
+  ia.k_hot = s->k_hot;
+  ia.v_hot = s->v_hot;
+  ia.hot_plane = s->hot_cap * cf.head_dim;
+  ia.hot_off = s->d_hot;
   ia.plane = int64_t(cf.capacity_tokens) * cf.head_dim;
   ia.fact_off = s->d_off;
   ia.fact_len = s->d_len;
@@ -422,7 +514,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.desc = s->ws_desc;
   ia.hdr = s->ws_hdr;
   ia.st = s->d_status;
-  void* fn = pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size);
+  void* fn = pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena);
   void* args[] = {&ia};
   TimedLaunch* ev = nullptr;
   if (s->timing && s->events_used < size_t(kMaxTimedLaunches)) {

@@ -57,7 +57,7 @@ class FactStore:
     def __init__(self, num_layers: int, num_kv_heads: int, head_dim: int, rope: RopeConfig,
                  capacity_tokens: int, max_facts: int, device: int = 0,
                  max_batch_requests: int = 0, max_batch_fact_ids: int = 0,
-                 max_batch_blocks: int = 0):
+                 max_batch_blocks: int = 0, host_tier: bool = False, hot_capacity_tokens: int = 0):
         cfg = B.is_store_config_t()
         cfg.num_layers, cfg.num_kv_heads, cfg.head_dim = num_layers, num_kv_heads, head_dim
         cfg.rope_style, cfg.rope_theta = rope.style, rope.theta
@@ -70,7 +70,8 @@ class FactStore:
         cfg.capacity_tokens, cfg.max_facts = capacity_tokens, max_facts
         cfg.max_batch_requests, cfg.max_batch_fact_ids = max_batch_requests, max_batch_fact_ids
         cfg.max_batch_blocks = max_batch_blocks
-        cfg.tier = B.IS_TIER_DEVICE
+        cfg.tier = B.IS_TIER_HOST if host_tier else B.IS_TIER_DEVICE
+        cfg.hot_capacity_tokens = hot_capacity_tokens
         self.L, self.H, self.D = num_layers, num_kv_heads, head_dim
         self.device = device
         self.capacity_tokens = capacity_tokens
@@ -128,6 +129,16 @@ class FactStore:
         k = torch.as_tensor(_DeviceArray(kp, shape, "<i2"), device=dev).view(torch.bfloat16)
         v = torch.as_tensor(_DeviceArray(vp, shape, "<i2"), device=dev).view(torch.bfloat16)
         return k, v
+
+    def set_hot(self, fact_ids) -> None:
+        """Host tier: keep these facts (host int sequence) in the HBM hot arenas."""
+        import numpy as np
+        ids = np.ascontiguousarray(np.asarray(fact_ids, dtype=np.int32))
+        B.is_store_set_hot(self.handle, ids.ctypes.data, ids.size)
+
+    def tier_info(self) -> dict:
+        t, cap, used, nf = B.is_store_tier_info(self.handle)
+        return dict(tier=t, hot_capacity=cap, hot_used=used, hot_facts=nf)
 
     # ---- the hot path
     def inject(self, req_offsets: torch.Tensor, fact_ids: torch.Tensor, start_pos: torch.Tensor,

@@ -1,0 +1,81 @@
+"""Host-tier store (pinned host memory + HBM hot set), against the CPU oracle.
+
+The tier changes where rows are read from, never what is written: every
+parity bar of the device tier applies unchanged (the oracle knows no tiers).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_common import make_store
+from kv_cache_injection_gather_b200 import binding as B
+from test_gpu_parity import _ragged, assert_parity, gpu_run, oracle_run
+
+pytestmark = pytest.mark.gpu
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+@pytest.mark.parametrize("hot_part", ["none", "some", "all"])
+def test_host_tier_parity(hot_part):
+    _need_gpu()
+    model = synth.Model("qwen-like", 2, 4, 128, 1e6)
+    wl = _ragged(model, seed=21, R=6, max_k=8, lens=(1, 40), num_facts=30)
+    total = int(wl.fact_lens.sum())
+    store = make_store(wl, host_tier=True, hot_capacity_tokens=total)
+    if hot_part == "some":
+        store.set_hot(np.arange(0, 30, 3))
+    elif hot_part == "all":
+        store.set_hot(np.arange(30))
+    info = store.tier_info()
+    assert info["tier"] == B.IS_TIER_HOST
+    assert info["hot_facts"] == {"none": 0, "some": 10, "all": 30}[hot_part]
+    assert_parity(oracle_run(wl), gpu_run(wl, store=store))
+    store.close()
+
+
+def test_host_tier_llama_shapes_with_llama3_scaling():
+    _need_gpu()
+    model = synth.Model("llama-like", 3, 8, 128, 5e5, llama3=True)
+    wl = _ragged(model, seed=22, R=4, max_k=6, lens=(16, 64), num_facts=25)
+    store = make_store(wl, host_tier=True, hot_capacity_tokens=200)
+    lens = wl.fact_lens
+    hot, used = [], 0
+    for f in np.argsort(-lens):          # fill the hot set as far as it goes
+        if used + lens[f] <= 200:
+            hot.append(int(f))
+            used += int(lens[f])
+    store.set_hot(hot)
+    assert store.tier_info()["hot_used"] == used
+    assert_parity(oracle_run(wl), gpu_run(wl, store=store))
+    store.close()
+
+
+def test_set_hot_errors_keep_previous_set():
+    _need_gpu()
+    wl = synth.tiny(0)
+    store = make_store(wl, host_tier=True, hot_capacity_tokens=40)
+    store.set_hot([0])
+    before = store.tier_info()
+    with pytest.raises(B.InjectError) as e:
+        store.set_hot(list(range(64)))            # far more than 40 tokens
+    assert e.value.status == B.IS_ERR_CAPACITY
+    with pytest.raises(B.InjectError) as e:
+        store.set_hot([64])
+    assert e.value.status == B.IS_ERR_BAD_FACT_ID
+    assert store.tier_info() == before
+    assert_parity(oracle_run(wl), gpu_run(wl, store=store))
+    store.close()
+    dev = make_store(wl)
+    with pytest.raises(B.InjectError) as e:
+        dev.set_hot([0])
+    assert e.value.status == B.IS_ERR_NOT_SUPPORTED
+    assert dev.tier_info()["tier"] == B.IS_TIER_DEVICE
+    dev.close()
