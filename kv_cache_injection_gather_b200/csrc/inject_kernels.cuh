@@ -292,18 +292,39 @@ struct InjectArgs {
   const int64_t* hot_off;    // [num_facts], -1 when the fact is not in HBM
 };
 
+// Streaming 16-byte accesses: every store row is read once per batch and
+// every cache row written once, so neither is kept in L1; stores are marked
+// evict-first.  (IS_LOAD_HINT / IS_STORE_HINT select other forms when tuning.)
+#ifndef IS_LOAD_HINT
+#define IS_LOAD_HINT 0
+#endif
+#ifndef IS_STORE_HINT
+#define IS_STORE_HINT 0
+#endif
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
   uint4 v;
+#if IS_LOAD_HINT == 2
+  asm volatile("ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+#else
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
+#endif
   return v;
 }
 
 __device__ __forceinline__ void st_stream(uint16_t* p, const uint4& v) {
+#if IS_STORE_HINT == 1
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+#else
   asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w)
                : "memory");
+#endif
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -407,8 +428,8 @@ __device__ __forceinline__ int ilog2(int x) { return 31 - __clz(x); }
 // powers of two (all index splits are shifts).  HOST_TIER: the store lives
 // in pinned host memory read over the host link, except the facts that also
 // sit in the HBM hot arenas; the source of every slot is chosen per fact.
-template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER>
-__global__ void __launch_bounds__(NT, 2) inject_kernel(InjectArgs a) {
+template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER>
+__global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   constexpr int VPR = D / 8;  // 16-byte vectors per head row
   constexpr int LOG_VPR = (VPR == 4) ? 2 : (VPR == 8) ? 3 : (VPR == 16) ? 4 : 5;
   extern __shared__ float4 s_cs4[];            // [B * D/4] cos/sin of the block

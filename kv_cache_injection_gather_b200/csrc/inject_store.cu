@@ -14,8 +14,20 @@
 namespace {
 
 constexpr int kPlanThreads = 1024;
-constexpr int kInjectThreads = 256;
-constexpr int kVecsPerThread = 8;
+// Inject-kernel launch shape (compile-time knobs; the defaults are the
+// measured best on B200 for the Llama-3.1-8B-shaped batch).
+#ifndef IS_INJECT_THREADS
+#define IS_INJECT_THREADS 256
+#endif
+#ifndef IS_INJECT_VECS
+#define IS_INJECT_VECS 8
+#endif
+#ifndef IS_INJECT_MIN_BLOCKS
+#define IS_INJECT_MIN_BLOCKS 2
+#endif
+constexpr int kInjectThreads = IS_INJECT_THREADS;
+constexpr int kVecsPerThread = IS_INJECT_VECS;
+constexpr int kInjectMinBlocks = IS_INJECT_MIN_BLOCKS;
 constexpr int kDefaultMaxRequests = 4096;
 constexpr int kDefaultMaxFactIds = 1 << 20;
 constexpr int kMaxTimedLaunches = 4096;
@@ -132,7 +144,7 @@ bool head_dim_supported(int d) { return d == 32 || d == 64 || d == 128 || d == 2
 template <int D, int STYLE, bool POW2, bool HOST_TIER>
 void* inject_fn() {
   return reinterpret_cast<void*>(
-      &isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, POW2, HOST_TIER>);
+      &isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER>);
 }
 
 template <bool POW2, bool HOST_TIER = false>
