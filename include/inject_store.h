@@ -171,8 +171,8 @@ int is_store_arena(const is_store_t* store, void** k_arena_out, void** v_arena_o
  * No other cache element is written.
  *
  * Arguments (all arrays on the device):
- *   req_fact_offsets  int32 [num_requests + 1], CSR, [0] = 0,
- *                     [num_requests] = num_fact_ids
+ *   req_fact_offsets  int32 [num_requests + 1], CSR, non-decreasing,
+ *                     [0] = 0, [num_requests] = num_fact_ids
  *   fact_ids          int32 [num_fact_ids]; duplicates allowed
  *   start_pos         int32 [num_requests], first injected position
  *   block_tables      int32 [num_requests][max_blocks_per_req]
@@ -185,8 +185,9 @@ int is_store_arena(const is_store_t* store, void** k_arena_out, void** v_arena_o
  * (INVALID_ARG, CAPACITY when num_requests or num_fact_ids exceed the
  * store's batch limits, NOT_SUPPORTED, CUDA); device-side errors are found
  * by is_last_error():
- *   INVALID_ARG  CSR does not cover num_fact_ids (nothing written), a
- *                malformed request range or negative start (request skipped)
+ *   INVALID_ARG  CSR not starting at 0, not ending at num_fact_ids or with
+ *                a decreasing offset (nothing written); a negative start
+ *                (that request skipped)
  *   BAD_FACT_ID  id outside the store (its request skipped)
  *   POSITION     segment past max_blocks_per_req * B (request skipped)
  *   BAD_BLOCK    table entry outside [0, num_blocks) (that block skipped)

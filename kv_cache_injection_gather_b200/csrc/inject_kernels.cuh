@@ -25,6 +25,10 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#ifndef IS_UNITS_PER_CTA
+#define IS_UNITS_PER_CTA 256
+#endif
+
 namespace isk {
 
 // Status codes, same values as inject_store.h.
@@ -103,21 +107,45 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   __shared__ int s_wsum_blk[NW];
   __shared__ long long s_wsum_tok[NW];
 
-  if (tid == 0) {
-    const bool bad = a.R < 0 || a.req_off[0] != 0 || a.req_off[a.R] != a.num_ids;
-    s_bad = bad;
-    if (bad) {
-      record_error(a.st, kErrInvalidArg, -1);
-      a.hdr->total_blocks = 0;
-      a.hdr->total_units = 0;
-      a.hdr->units_per_block = 1;
-      a.hdr->layers_per_unit = a.L;
-      a.hdr->next_unit = 0;
-      a.hdr->total_tokens = 0;
+  // The inject grid may be scheduled now; it waits for this grid's results
+  // (griddepcontrol.wait) before reading any of them.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // The CSR must start at 0, end at num_ids and never decrease; otherwise
+  // the whole batch is rejected and nothing is written.
+  if (tid == 0) s_bad = a.R < 0 || a.req_off[0] != 0 || a.req_off[a.R] != a.num_ids;
+  __syncthreads();
+  for (int r = tid; r < a.R; r += NT)
+    if (a.req_off[r + 1] < a.req_off[r]) s_bad = 1;
+  __syncthreads();
+  if (tid == 0 && s_bad) {
+    record_error(a.st, kErrInvalidArg, -1);
+    a.hdr->total_blocks = 0;
+    a.hdr->total_units = 0;
+    a.hdr->units_per_block = 1;
+    a.hdr->layers_per_unit = a.L;
+    a.hdr->next_unit = 0;
+    a.hdr->total_tokens = 0;
+  }
+  if (s_bad) return;
+
+  // Phase 0, all threads: the length of every listed fact (-1 for an id
+  // outside the store), fetched in parallel into seg[], which phase 1 then
+  // overwrites with segment offsets.
+  for (int32_t base = 0; base < a.num_ids; base += NT * 4) {
+    int32_t f[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int32_t j = base + q * NT + tid;
+      f[q] = j < a.num_ids ? a.fact_ids[j] : -1;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int32_t j = base + q * NT + tid;
+      if (j < a.num_ids) a.seg[j] = (f[q] >= 0 && f[q] < a.num_facts) ? a.fact_len[f[q]] : -1;
     }
   }
   __syncthreads();
-  if (s_bad) return;
 
   // Phase 1, one warp per request: segment offsets of its facts (exclusive
   // prefix of their lengths, in retrieval order), length, validity, blocks.
@@ -130,13 +158,9 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     } else {
       for (int32_t base = j0; base < j1; base += 32) {
         const int32_t j = base + lane;
-        int32_t len = 0;
-        bool ok = true;
-        if (j < j1) {
-          const int32_t f = a.fact_ids[j];
-          ok = f >= 0 && f < a.num_facts;
-          len = ok ? a.fact_len[f] : 0;
-        }
+        const int32_t lj = j < j1 ? a.seg[j] : 0;
+        const bool ok = lj >= 0;
+        const int32_t len = ok ? lj : 0;
         int32_t x = len;  // inclusive warp scan
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -202,11 +226,20 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   const bool over_blocks = total_blocks > a.max_batch_blocks;
 
   if (tid == 0) {
-    // Work-unit size: enough units for ~32 per CTA, layers split evenly.
-    long long want = (long long)a.grid_ctas * 32;
+    // Work-unit size (layers per unit).  A batch whose one-layer units fit in
+    // about one wave of the grid uses one layer per unit: everything is in
+    // flight at once (latency).  Larger batches aim at ~IS_UNITS_PER_CTA
+    // units per CTA, so the dynamic schedule's tail (at most one unit) stays
+    // short, with at least two layers per unit so a unit's set-up (slot walk,
+    // cos/sin table) is shared by more than one layer's copy.
+    const long long grid = a.grid_ctas;
     int32_t upb = 1;
-    if (total_blocks > 0 && (long long)total_blocks < want)
-      upb = int32_t(min((long long)a.L, (want + total_blocks - 1) / total_blocks));
+    if (total_blocks > 0 && (long long)total_blocks * a.L <= 2 * grid) {
+      upb = a.L;
+    } else if (total_blocks > 0) {
+      const long long want = (grid * IS_UNITS_PER_CTA + total_blocks - 1) / total_blocks;
+      upb = int32_t(max(1LL, min(want, (long long)max(1, a.L / 2))));
+    }
     const int32_t lpu = (a.L + upb - 1) / upb;
     upb = (a.L + lpu - 1) / lpu;
     a.hdr->layers_per_unit = lpu;
@@ -236,11 +269,12 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     const int32_t g0 = a.req_blk0[r];
     // Fact j covers segment indices [seg[j], seg[j] + len_j).  Block bi >= 1
     // starts at segment index (fb + bi) * B - start; block 0 starts at 0.
+    const int32_t S = a.req_len[r];
     for (int32_t base = j0; base < j1; base += 32) {
       const int32_t j = base + lane;
       if (j >= j1) continue;
       const int32_t s = a.seg[j];
-      const int32_t len = a.fact_len[a.fact_ids[j]];
+      const int32_t len = (j + 1 < j1 ? a.seg[j + 1] : S) - s;  // valid request: all seg >= 0
       if (len == 0) continue;
       const int32_t e = s + len;               // exclusive end
       // blocks bi whose first segment index lies in [s, e)
@@ -441,6 +475,9 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   __shared__ int s_unit;
 
   const int tid = threadIdx.x;
+  // When launched as a programmatic dependent of the plan kernel, wait here
+  // for its results; without such a launch this returns at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int total_units = a.hdr->total_units;
   const int total_blocks = a.hdr->total_blocks;
   const int lpu = a.hdr->layers_per_unit;

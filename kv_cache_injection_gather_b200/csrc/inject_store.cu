@@ -78,6 +78,9 @@ struct is_store {
   // staging for is_inject_batch_host
   int32_t* stage = nullptr;
   size_t stage_elems = 0;
+  int32_t* host_stage = nullptr;   // pinned mirror of `stage`
+  size_t host_stage_elems = 0;
+  isk::DevStatus* host_status = nullptr;  // pinned
   int64_t* stage_slots = nullptr;
   int64_t stage_slot_elems = 0;
   // timing
@@ -122,6 +125,8 @@ void free_store(is_store* s) {
   cudaFree(s->d_status);
   cudaFree(s->stage);
   cudaFree(s->stage_slots);
+  cudaFreeHost(s->host_stage);
+  cudaFreeHost(s->host_status);
   cudaFree(s->k_hot);
   cudaFree(s->v_hot);
   cudaFree(s->d_hot);
@@ -174,11 +179,19 @@ size_t cs_smem_bytes(int D, int B) { return size_t(B) * size_t(D / 2) * sizeof(f
 int grow_stage(is_store* s, size_t elems, int64_t slot_elems) {
   if (elems > s->stage_elems) {
     cudaFree(s->stage);
+    cudaFreeHost(s->host_stage);
     s->stage = nullptr;
+    s->host_stage = nullptr;
     s->stage_elems = 0;
     if (dalloc(&s->stage, elems) != cudaSuccess) return IS_ERR_OOM;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&s->host_stage), elems * sizeof(int32_t),
+                      cudaHostAllocDefault) != cudaSuccess)
+      return IS_ERR_OOM;
     s->stage_elems = elems;
   }
+  if (!s->host_status && cudaHostAlloc(reinterpret_cast<void**>(&s->host_status), sizeof(isk::DevStatus),
+                                       cudaHostAllocDefault) != cudaSuccess)
+    return IS_ERR_OOM;
   if (slot_elems > s->stage_slot_elems) {
     cudaFree(s->stage_slots);
     s->stage_slots = nullptr;
@@ -537,10 +550,28 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
     }
     if (s->events_used < s->events.size()) ev = &s->events[s->events_used++];
   }
-  if (ev) cudaEventRecord(ev->start, st);
-  cudaError_t e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), args,
-                                   cs_smem_bytes(cf.head_dim, c.block_size), st);
-  if (ev) cudaEventRecord(ev->stop, st);
+  cudaError_t e;
+  if (ev) {
+    // Timed: events bracket the inject kernel alone (no early launch).
+    cudaEventRecord(ev->start, st);
+    e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), args,
+                         cs_smem_bytes(cf.head_dim, c.block_size), st);
+    cudaEventRecord(ev->stop, st);
+  } else {
+    // Programmatic dependent launch: the inject grid becomes resident while
+    // the plan kernel runs and starts work when the plan's results are ready.
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(unsigned(s->inject_grid));
+    lc.blockDim = dim3(kInjectThreads);
+    lc.dynamicSmemBytes = cs_smem_bytes(cf.head_dim, c.block_size);
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelExC(&lc, fn, args);
+  }
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
   return IS_OK;
 }
@@ -560,14 +591,17 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
   const int64_t n_slots = slot_out ? slot_cap : 0;
   int rc = grow_stage(s, n_off + n_ids + n_sp + n_bt + 4, n_slots);
   if (rc != IS_OK) return rc;
+  // Pack the four index arrays into one pinned buffer: one host-to-device copy.
+  int32_t* h = s->host_stage;
+  std::memcpy(h, req_off, n_off * 4);
+  if (n_ids) std::memcpy(h + n_off, fact_ids, n_ids * 4);
+  if (n_sp) std::memcpy(h + n_off + n_ids, start_pos, n_sp * 4);
+  if (n_bt) std::memcpy(h + n_off + n_ids + n_sp, block_tables, n_bt * 4);
   int32_t* d_off = s->stage;
   int32_t* d_ids = d_off + n_off;
   int32_t* d_sp = d_ids + n_ids;
   int32_t* d_bt = d_sp + n_sp;
-  if (cudaMemcpyAsync(d_off, req_off, n_off * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      (n_ids && cudaMemcpyAsync(d_ids, fact_ids, n_ids * 4, cudaMemcpyHostToDevice, st) != cudaSuccess) ||
-      (n_sp && cudaMemcpyAsync(d_sp, start_pos, n_sp * 4, cudaMemcpyHostToDevice, st) != cudaSuccess) ||
-      (n_bt && cudaMemcpyAsync(d_bt, block_tables, n_bt * 4, cudaMemcpyHostToDevice, st) != cudaSuccess))
+  if (cudaMemcpyAsync(d_off, h, (n_off + n_ids + n_sp + n_bt) * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return IS_ERR_CUDA;
   rc = is_inject_batch(s, R, d_off, d_ids, num_ids, d_sp, d_bt, max_blocks_per_req, cache,
                        slot_out ? s->stage_slots : nullptr, slot_cap, stream);
@@ -576,7 +610,14 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
       cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost, st) !=
           cudaSuccess)
     return IS_ERR_CUDA;
-  return is_last_error(s, stream, nullptr);
+  // Status back in the same stream, then one wait.
+  if (cudaMemcpyAsync(s->host_status, s->d_status, sizeof(isk::DevStatus), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return IS_ERR_CUDA;
+  const int code = s->host_status->code;
+  if (code != 0 && cudaMemset(s->d_status, 0, sizeof(isk::DevStatus)) != cudaSuccess) return IS_ERR_CUDA;
+  return code;
 }
 
 int is_last_error(is_store_t* s, void* stream, int64_t* detail) {

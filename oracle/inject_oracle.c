@@ -228,8 +228,10 @@ static int request_segment(const orc_store_t* s, const int32_t* req_off, const i
  * block table) keeps its token indices but none of its tokens is written.
  * Writes, per token, the request, the store token index, the position and
  * the slot (-1 when not written); arrays may be NULL, at most cap entries.
- * Returns the number of tokens, or ORC_ERR_INVALID_ARG when the CSR bounds
- * of the whole batch are wrong (then nothing is composed). */
+ * Returns the number of tokens, or ORC_ERR_INVALID_ARG when the CSR of the
+ * whole batch is wrong -- first offset not 0, last offset not the number of
+ * ids, or an offset smaller than the one before -- (then nothing is
+ * composed). */
 int64_t orc_segment(const orc_store_t* s, int32_t R, const int32_t* req_off, const int32_t* ids,
                     int32_t num_ids, const int32_t* start, const int32_t* bt, int32_t max_blocks,
                     int32_t B, int32_t num_blocks, int64_t cap, int32_t* tok_req,
@@ -239,6 +241,12 @@ int64_t orc_segment(const orc_store_t* s, int32_t R, const int32_t* req_off, con
     if (status) *status = ORC_ERR_INVALID_ARG;
     return ORC_ERR_INVALID_ARG;
   }
+  /* A CSR's offsets never decrease; one that does is not a batch. */
+  for (int32_t r = 0; r < R; ++r)
+    if (req_off[r + 1] < req_off[r]) {
+      if (status) *status = ORC_ERR_INVALID_ARG;
+      return ORC_ERR_INVALID_ARG;
+    }
   int64_t n = 0;
   for (int32_t r = 0; r < R; ++r) {
     int64_t S;

@@ -382,6 +382,9 @@ def test_inject_errors_and_isolation():
     k4 = kc4.copy()
     rc, _ = oracle.inject_batch(st, f, [0, 1], ids[:2], [0], bt[:1], kc4, vc4, 16)
     assert rc == oracle.ERR_INVALID_ARG and np.array_equal(kc4, k4)
+    # offsets that decrease (overlapping ranges): the whole batch is rejected
+    rc, _ = oracle.inject_batch(st, f, [0, 3, 2, 4], ids[:4], [0, 40, 80], bt, kc4, vc4, 16)
+    assert rc == oracle.ERR_INVALID_ARG and np.array_equal(kc4, k4)
     # slot output too small: nothing written
     rc, _ = oracle.inject_batch(st, f, [0, 2], ids[:2], [0], bt[:1], kc4, vc4, 16,
                                 slot_capacity=3)
