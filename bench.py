@@ -223,7 +223,7 @@ WORKLOADS = {
                      lambda seed: _synth().llama_single(seed)),
     "offload": ("qwen2.5-7b-shapes store of 16..48-token facts in pinned host memory, HBM hot "
                 "set = top 20% by Zipf rank, 100 requests x k=50 drawn Zipf(1.1), block 16",
-                lambda seed, n=100_000: _synth().offload(seed, num_facts=n)),
+                lambda seed, n=100_000: _synth().offload(seed, num_facts=n, extra_batches=7)),
     "qwen-sweep": ("qwen2.5-7b-shapes 50k-fact store (lognormal 8..96), R=100 x k=50, block 16",
                    lambda seed: _synth().sweep(_synth().QWEN25_7B, 100, 50, seed)),
     "mistral-sweep": ("mistral-7b-shapes 20k-fact store (lognormal 8..96; capped so store + "
@@ -294,6 +294,49 @@ def _cuda():
         return False
 
 
+def gpu_id(dev, local_rank: int) -> str:
+    """nvidia-smi --id for this device (its UUID), else the local rank."""
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(local_rank)
+
+
+def copy_probe(dev, elems: int = 1 << 30, reps: int = 10):
+    """Device copy bandwidth on this machine now (read + write bytes / time): the
+    best of reps single copies (the kind of figure the measured peak is) and
+    the average of ~0.8 s of copies back to back (a sustained figure, under
+    the same power cap as a long timed region).  Context for the roofline
+    fraction, not its denominator."""
+    import torch
+    a = torch.empty(elems, dtype=torch.bfloat16, device=dev)
+    b = torch.empty_like(a)
+    b.copy_(a)
+    best = float("inf")
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        b.copy_(a)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        best = min(best, e0.elapsed_time(e1))
+    # sustained: back to back for about as long as a timed region
+    n = max(1, int(800.0 / best))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        b.copy_(a)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    sustained = n * 2 * elems * 2 / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del a, b
+    torch.cuda.empty_cache()
+    return 2 * elems * 2 / (best / 1e3) / 1e9, sustained
+
+
 def h2d_probe(dev, nbytes: int = 1 << 30, reps: int = 5) -> float:
     """Pinned host -> device copy bandwidth (GB/s), CUDA events."""
     import torch
@@ -323,6 +366,142 @@ def max_over_ranks(values, world):
     return t.cpu().tolist()
 
 
+def run_offload(args, rank, world, local_rank):
+    """Host-tier store: a stream of 8 different Zipf batches, cycled.  Static
+    hot set (top 20% by rank, device-index entry point) or LRU hot set (same
+    HBM capacity in 48-token slots, host-index entry point, which promotes each
+    batch's cold facts before injecting)."""
+    import psutil
+    import torch
+
+    import synth
+    from gpu_common import make_cache, make_store
+    from kv_cache_injection_gather_b200 import binding as B
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    n_facts = 100_000
+    avail = psutil.virtual_memory().available
+    while n_facts * 32 * synth.QWEN25_7B.bytes_per_token > 0.6 * avail and n_facts > 5_000:
+        n_facts = int(n_facts * 0.8)
+    wl = WORKLOADS["offload"][1](rank, n_facts)
+    m, b0 = wl.model, wl.batch
+    hot = wl.notes["hot"]
+    hot_tokens = int(wl.fact_lens[hot].sum())
+    store = make_store(wl, on_device_gen=True, device=local_rank, host_tier=True,
+                       hot_capacity_tokens=hot_tokens)
+    lru = args.hot_policy == "lru"
+    if lru:
+        store.set_hot_policy(True, 48)  # slots of the longest fact, same HBM tokens
+    else:
+        store.set_hot(hot)
+    batches = [b0] + [synth.Batch(b0.req_offsets, ids, b0.start_pos, b0.block_tables,
+                                  b0.block_size, b0.num_blocks) for ids in wl.notes["more_ids"]]
+    ntoks = [int(wl.fact_lens[bb.fact_ids].sum()) for bb in batches]
+    kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False)
+    stream = torch.cuda.current_stream(dev)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
+    dvc = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)  # noqa: E731
+    host_b = [(pin(bb.req_offsets), pin(bb.fact_ids), pin(bb.start_pos), pin(bb.block_tables))
+              for bb in batches]
+    dev_b = [(dvc(bb.req_offsets), dvc(bb.fact_ids), dvc(bb.start_pos), dvc(bb.block_tables))
+             for bb in batches]
+    d_slots = torch.empty(max(ntoks), dtype=torch.int64, device=dev)
+    h_slots = torch.empty(max(ntoks), dtype=torch.int64).pin_memory()
+
+    def step(i):
+        j = i % len(batches)
+        if lru:
+            rc = store.inject_host(*host_b[j], desc, h_slots[:ntoks[j]], stream.cuda_stream)
+            if rc != 0:
+                raise RuntimeError(f"inject_host failed: {B.status_string(rc)}")
+        else:
+            store.inject(*dev_b[j], desc, d_slots[:ntoks[j]], stream.cuda_stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    st0 = store.lru_stats() if lru else None
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(gpu_id(dev, local_rank))
+    clocks.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    rc, _ = store.last_error()
+    if rc != 0:
+        raise RuntimeError(f"inject failed: {B.status_string(rc)}")
+    st1 = store.lru_stats() if lru else None
+    store.set_timing(True)
+    store.kernel_time()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    torch.cuda.synchronize(dev)
+    kern_ms, kern_n = store.kernel_time()
+    store.set_timing(False)
+    ms, kern_avg_ms = max_over_ranks([ms, kern_ms / max(kern_n, 1)], world)
+    tok_run = sum(ntoks[(args.warmup + i) % len(batches)] for i in range(args.steps))
+    value = world * tok_run / (ms / 1e3)
+    bpt = m.bytes_per_token
+    peak, peak_kind = hbm_peak()
+    link = h2d_probe(dev)
+    if lru:
+        prom_tok = st1["promoted_tokens"] - st0["promoted_tokens"]
+        link_bytes = prom_tok * bpt
+        hbm_bytes = (2 * tok_run + prom_tok) * bpt
+        t_min = max(link_bytes / (link * 1e9), hbm_bytes / (peak * 1e9))
+        hits = st1["hits"] - st0["hits"]
+        misses = st1["misses"] - st0["misses"]
+        detail = {"id_hit_fraction": hits / max(hits + misses, 1),
+                  "promoted_tokens_per_step": prom_tok / args.steps}
+        measured_s = ms / 1e3
+    else:
+        is_hot = np.zeros(len(wl.fact_lens), bool)
+        is_hot[hot] = True
+        t_min, link_bytes, hit_tok = 0.0, 0, 0
+        for i in range(args.steps):
+            bb = batches[(args.warmup + i) % len(batches)]
+            per = wl.fact_lens[bb.fact_ids].astype(np.int64)
+            hit = int(per[is_hot[bb.fact_ids]].sum())
+            miss_b = (int(per.sum()) - hit) * bpt
+            t_min += max(miss_b / (link * 1e9), (hit + int(per.sum())) * bpt / (peak * 1e9))
+            link_bytes += miss_b
+            hit_tok += hit
+        hbm_bytes = (hit_tok + tok_run) * bpt
+        detail = {"hit_token_fraction": hit_tok / max(tok_run, 1)}
+        measured_s = kern_avg_ms * args.steps / 1e3
+    algo = 2 * tok_run * bpt
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": workload_config(wl, "offload", {
+            "facts_note": f"{n_facts} facts (host memory available {avail / 1e9:.0f} GB)",
+            "hot_policy": args.hot_policy, "hot_tokens_per_plane": hot_tokens,
+            "batches": f"{len(batches)} Zipf batches cycled", "parallelism": f"replicas x{world}"}),
+        "us_per_batch": ms / args.steps * 1e3, "kernel_us": kern_avg_ms * 1e3, "clocks": clk,
+        "gpu_launches": (4 if lru else 2) * args.steps,
+        "roofline": {"bound": "host_link+hbm", "achieved": algo / measured_s / 1e9,
+                     "peak": algo / t_min / 1e9, "unit": "GB/s", "frac": t_min / measured_s,
+                     "peak_source": f"pinned H2D probe {link:.1f} GB/s for {link_bytes / 1e9:.2f} GB "
+                                    f"over the host link; {peak_kind} hbm_gbs {peak} for "
+                                    f"{hbm_bytes / 1e9:.1f} GB in HBM; per step the slower bounds",
+                     "timed": "whole step (promotion + plan + inject)" if lru else
+                              "inject kernel (plan excluded)", **detail},
+        "cpu_baseline": None,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    store.close()
+    return 0
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -334,31 +513,15 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("bench.py needs a CUDA device (the inject path has no CPU fallback)")
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    offload = args.workload == "offload"
+    if args.workload == "offload":
+        return run_offload(args, rank, world, local_rank)
     extra_cfg = {}
-    if offload:
-        # the store must fit in pinned host memory: scale the fact count down
-        # (keeping the 20% hot ratio) when the host has less than it needs
-        import psutil
-        import synth as _s
-        n_facts = 100_000
-        avail = psutil.virtual_memory().available
-        while n_facts * 32 * _s.QWEN25_7B.bytes_per_token > 0.6 * avail and n_facts > 5_000:
-            n_facts = int(n_facts * 0.8)
-        wl = WORKLOADS["offload"][1](rank, n_facts)
-        hot = wl.notes["hot"]
-        hot_tokens = int(wl.fact_lens[hot].sum())
-        extra_cfg = {"facts_note": f"{n_facts} facts (host memory available "
-                                   f"{avail / 1e9:.0f} GB)",
-                     "hot_facts": int(len(hot)), "hot_tokens_per_plane": hot_tokens}
-        store = make_store(wl, on_device_gen=True, device=local_rank, host_tier=True,
-                           hot_capacity_tokens=hot_tokens)
-        store.set_hot(hot)
-    else:
-        wl = WORKLOADS[args.workload][1](rank)
-        store = make_store(wl, on_device_gen=True, device=local_rank)
+    wl = WORKLOADS[args.workload][1](rank)
+    store = make_store(wl, on_device_gen=True, device=local_rank)
     m, b = wl.model, wl.batch
-    kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False)
+    kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False, head_major=args.head_major)
+    extra_cfg["cache_layout"] = "[L][num_blocks][H][B][D]" if args.head_major else "[L][num_blocks][B][H][D]"
+    copy_ref, copy_sus = copy_probe(dev)
     ro, ids, sp, bt = batch_tensors(b, local_rank)
     n_tok = wl.tokens()
     slots = torch.empty(n_tok, dtype=torch.int64, device=dev)
@@ -378,11 +541,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    try:
-        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        gpu_id = str(local_rank)
-    clocks = ClockSampler(gpu_id)
+    clocks = ClockSampler(gpu_id(dev, local_rank))
     # ---- device-resident timed region (the value)
     barrier()
     clocks.start()
@@ -440,34 +599,16 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = hbm_peak()
     achieved = algo_bytes / (kern_avg_ms / 1e3) / 1e9
     traffic_pt, rec = recorded_traffic(2 * m.bytes_per_token)
-    if args.workload != "llama-batch":
+    if args.workload != "llama-batch" or args.head_major:
         traffic_pt = None  # the committed counters are for the benchmark workload
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                "same_box_copy_gbs": copy_ref, "frac_of_same_box_copy": achieved / copy_ref,
+                "same_box_sustained_copy_gbs": copy_sus,
+                "frac_of_same_box_sustained_copy": achieved / copy_sus,
                 "traffic": None if traffic_pt is None else traffic_pt * n_tok,
                 "algorithmic_bytes": algo_bytes,
                 "kernel": "inject_kernel (plan_kernel excluded)"}
-    if offload:
-        # reads of cold facts cross the host link, hits and all writes are HBM
-        is_hot = np.zeros(len(wl.fact_lens), bool)
-        is_hot[wl.notes["hot"]] = True
-        per_id = wl.fact_lens[b.fact_ids].astype(np.int64)
-        hit_tok = int(per_id[is_hot[b.fact_ids]].sum())
-        miss_bytes = (n_tok - hit_tok) * m.bytes_per_token
-        hbm_bytes = hit_tok * m.bytes_per_token + n_tok * m.bytes_per_token
-        link = h2d_probe(dev)
-        # the kernel overlaps host-link reads with HBM traffic: the slower of
-        # the two bounds the batch
-        t_min = max(miss_bytes / (link * 1e9), hbm_bytes / (peak * 1e9))
-        roofline = {"bound": "host_link+hbm", "achieved": achieved,
-                    "peak": algo_bytes / t_min / 1e9, "unit": "GB/s",
-                    "frac": t_min / (kern_avg_ms / 1e3),
-                    "peak_source": f"pinned H2D probe {link:.1f} GB/s for the {miss_bytes / 1e9:.3f} GB "
-                                   f"of cold-fact reads + {peak_kind} hbm_gbs {peak} for the "
-                                   f"{hbm_bytes / 1e9:.2f} GB of hot reads and writes",
-                    "traffic": None, "algorithmic_bytes": algo_bytes,
-                    "hit_token_fraction": hit_tok / max(n_tok, 1),
-                    "kernel": "inject_kernel host-tier variant (plan_kernel excluded)"}
     baseline = cpu_baseline(wl, local_rank) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if rank != 0:
         store.close()
@@ -502,6 +643,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hot-policy", choices=["static", "lru"], default="static",
+                    help="offload workload: static top-20%% hot set or LRU promotion")
+    ap.add_argument("--head-major", action="store_true",
+                    help="cache layout [L][num_blocks][H][B][D] instead of [L][num_blocks][B][H][D]")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama-batch",
                     help="llama-batch is the benchmark; the others are smaller cases for "
                          "profiling and latency")

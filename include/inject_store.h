@@ -124,6 +124,18 @@ void is_store_destroy(is_store_t* store);
 int is_store_put_fact(is_store_t* store, const void* k_pre, const void* v, int32_t len,
                       int32_t* fact_id_out);
 
+/* Append one fact from its context-window encoding (technical summary,
+ * Offline phase, "Context-Window Encoding": each fact is encoded with a
+ * window of w preceding turns and only the fact's KV is kept).  k_pre and v
+ * are bf16 [L][H][window_len + fact_len][D] (host or device) -- the pre-RoPE
+ * keys and raw values the encoder produced for the window followed by the
+ * fact -- and only the last fact_len tokens of every plane are stored.  The
+ * window tokens are dropped; positions play no part (keys are pre-RoPE).
+ * Synchronous.  Errors as for is_store_put_fact, and INVALID_ARG for
+ * window_len < 0. */
+int is_store_put_fact_window(is_store_t* store, const void* k_pre, const void* v,
+                             int32_t window_len, int32_t fact_len, int32_t* fact_id_out);
+
 /* Number of facts, and a fact's token offset in every plane and length. */
 int is_store_num_facts(const is_store_t* store, int32_t* num_facts_out);
 int is_store_fact_info(const is_store_t* store, int32_t fact_id, int64_t* offset_out,
@@ -140,10 +152,38 @@ int is_store_read_fact(is_store_t* store, int32_t fact_id, void* k_out, void* v_
  * host DRAM when GPU memory is too small).  fact_ids (host array, n
  * entries; repeats ignored) replaces the previous hot set; the facts are
  * copied in list order.  Waits for the device to go idle first, so no batch
- * reads a half-updated set.  Errors: NOT_SUPPORTED (device tier),
+ * reads a half-updated set.  Errors: NOT_SUPPORTED (device tier, or the
+ * LRU policy),
  * BAD_FACT_ID, CAPACITY (more tokens than the hot arenas hold; the old set
  * is kept), INVALID_ARG, CUDA. */
 int is_store_set_hot(is_store_t* store, const int32_t* fact_ids, int32_t n);
+
+/* Hot-set policy of a host-tier store.
+ *   IS_HOT_STATIC  the caller names the hot facts (is_store_set_hot).
+ *   IS_HOT_LRU     the hot arenas are cut into slots of slot_tokens tokens;
+ *                  is_store_touch (called by is_inject_batch_host for its
+ *                  batch) promotes requested cold facts of at most
+ *                  slot_tokens tokens into the least recently used slot not
+ *                  used by that call, so the batch reads them from HBM.
+ * Either way the set starts empty.  Waits for the device to go idle.
+ * Errors: NOT_SUPPORTED (device tier), INVALID_ARG, CUDA. */
+#define IS_HOT_STATIC 0
+#define IS_HOT_LRU 1
+int is_store_set_hot_policy(is_store_t* store, int policy, int32_t slot_tokens);
+
+/* IS_HOT_LRU: mark fact_ids (host array) as used now and promote the cold
+ * ones (see above).  The copies (host link -> HBM) and the hot-table update
+ * are queued on `stream`; work queued after them on the same stream reads
+ * the new set.  Ids outside the store are ignored here.  *promoted_out (may
+ * be NULL) receives the number of facts promoted.  First waits until the
+ * previous touch's queued copies have finished (their lists are reused). */
+int is_store_touch(is_store_t* store, const int32_t* fact_ids, int32_t n, void* stream,
+                   int32_t* promoted_out);
+
+/* IS_HOT_LRU counters since the policy was set: ids found hot, ids found
+ * cold (each counted once per touch), facts promoted and their tokens. */
+int is_store_lru_stats(const is_store_t* store, int64_t* hits_out, int64_t* misses_out,
+                       int64_t* promoted_out, int64_t* promoted_tokens_out);
 
 /* Tier of the store, hot-arena capacity and use (tokens per plane), and the
  * number of hot facts (0 for a device-tier store). */

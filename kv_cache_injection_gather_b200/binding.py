@@ -31,6 +31,8 @@ IS_SCALING_NONE = 0
 IS_SCALING_LLAMA3 = 1
 IS_TIER_DEVICE = 0
 IS_TIER_HOST = 1
+IS_HOT_STATIC = 0
+IS_HOT_LRU = 1
 
 IS_NOALLOC_MAX_REQUESTS = 1024
 IS_NOALLOC_MAX_FACT_IDS = 65536
@@ -76,6 +78,7 @@ _SIGNATURES = {
                                        ctypes.POINTER(_P)]),
     "is_store_destroy": (None, [_P]),
     "is_store_put_fact": (ctypes.c_int, [_P, _P, _P, _I32, ctypes.POINTER(_I32)]),
+    "is_store_put_fact_window": (ctypes.c_int, [_P, _P, _P, _I32, _I32, ctypes.POINTER(_I32)]),
     "is_store_num_facts": (ctypes.c_int, [_P, ctypes.POINTER(_I32)]),
     "is_store_fact_info": (ctypes.c_int, [_P, _I32, ctypes.POINTER(_I64), ctypes.POINTER(_I32)]),
     "is_store_read_fact": (ctypes.c_int, [_P, _I32, _P, _P]),
@@ -90,6 +93,10 @@ _SIGNATURES = {
     "is_store_kernel_time": (ctypes.c_int, [_P, ctypes.POINTER(_F64), ctypes.POINTER(_I64)]),
     "is_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "is_store_set_hot": (ctypes.c_int, [_P, _P, _I32]),
+    "is_store_set_hot_policy": (ctypes.c_int, [_P, ctypes.c_int, _I32]),
+    "is_store_touch": (ctypes.c_int, [_P, _P, _I32, _P, ctypes.POINTER(_I32)]),
+    "is_store_lru_stats": (ctypes.c_int, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64),
+                                          ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
     "is_store_tier_info": (ctypes.c_int, [_P, ctypes.POINTER(_I32), ctypes.POINTER(_I64),
                                           ctypes.POINTER(_I64), ctypes.POINTER(_I32)]),
     "is_inject_batch_noalloc": (ctypes.c_int, [ctypes.POINTER(is_store_config_t), _P, _P, _I64,
@@ -131,6 +138,14 @@ def is_store_put_fact(store: int, k_pre_ptr: int, v_ptr: int, length: int) -> in
     fid = _I32()
     check(_lib.is_store_put_fact(store, k_pre_ptr, v_ptr, length, ctypes.byref(fid)),
           "is_store_put_fact")
+    return fid.value
+
+
+def is_store_put_fact_window(store: int, k_pre_ptr: int, v_ptr: int, window_len: int,
+                             fact_len: int) -> int:
+    fid = _I32()
+    check(_lib.is_store_put_fact_window(store, k_pre_ptr, v_ptr, window_len, fact_len,
+                                        ctypes.byref(fid)), "is_store_put_fact_window")
     return fid.value
 
 
@@ -206,6 +221,24 @@ def is_status_string(status: int) -> str:
 
 def is_store_set_hot(store: int, fact_ids_host_ptr: int, n: int) -> None:
     check(_lib.is_store_set_hot(store, fact_ids_host_ptr, n), "is_store_set_hot")
+
+
+def is_store_set_hot_policy(store: int, policy: int, slot_tokens: int = 0) -> None:
+    check(_lib.is_store_set_hot_policy(store, policy, slot_tokens), "is_store_set_hot_policy")
+
+
+def is_store_touch(store: int, fact_ids_host_ptr: int, n: int, stream: int = 0) -> int:
+    promoted = _I32()
+    check(_lib.is_store_touch(store, fact_ids_host_ptr, n, stream, ctypes.byref(promoted)),
+          "is_store_touch")
+    return promoted.value
+
+
+def is_store_lru_stats(store: int) -> tuple[int, int, int, int]:
+    h, m, p, t = _I64(), _I64(), _I64(), _I64()
+    check(_lib.is_store_lru_stats(store, ctypes.byref(h), ctypes.byref(m), ctypes.byref(p),
+                                  ctypes.byref(t)), "is_store_lru_stats")
+    return h.value, m.value, p.value, t.value
 
 
 def is_store_tier_info(store: int) -> tuple[int, int, int, int]:

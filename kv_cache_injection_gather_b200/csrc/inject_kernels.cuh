@@ -312,6 +312,7 @@ struct InjectArgs {
   uint16_t* v_cache;
   int64_t ls, bs, ts, hs;    // cache strides (elements)
   int32_t num_blocks, B;
+  int32_t vec_order;         // 0: (slot, head) rows, 1: (head, slot) rows
   int64_t* slot_out;
   const int32_t* seg;
   const long long* req_tok0;
@@ -449,6 +450,30 @@ struct Divisor {
 
 __device__ __forceinline__ int ilog2(int x) { return 31 - __clz(x); }
 
+// Vector order inside one layer of a block (rem = the vector's index in the
+// layer; a head row is D/8 consecutive vectors, so rotate-half partners stay
+// in one warp).  Sets the slot o and hv = head * D/8 + word.
+//   order 0: rows in (slot, head) order, head fastest;
+//   order 1: rows in (head, slot) order, slot fastest.
+// The launch picks the order whose fastest row index has the larger cache
+// stride, so the rows a wave of threads writes are spread over the block's
+// run of the cache while each head plane of the store is still read in
+// runs of consecutive rows (measured on B200: 97.6% vs 96.0% of the copy
+// peak on the token-major cache, 98.7% vs 96.2% on the head-major cache).
+template <bool POW2>
+__device__ __forceinline__ void split_vec(int rem, int order, const Divisor<POW2>& by_row,
+                                          const Divisor<POW2>& by_hrow, int vpr, int log_vpr,
+                                          int& o, int& hv) {
+  if (order == 0) {
+    o = by_row.div(rem);
+    hv = by_row.mod(rem);
+  } else {
+    const int h = by_hrow.div(rem), r2 = by_hrow.mod(rem);
+    o = r2 >> log_vpr;
+    hv = (h << log_vpr) + (r2 & (vpr - 1));
+  }
+}
+
 // Persistent gather-rotate-scatter kernel.  Work unit u covers global block
 // gb = u % total_blocks and layers [lg * lpu, min(L, (lg + 1) * lpu)),
 // lg = u / total_blocks, so CTAs running side by side read neighbouring
@@ -487,6 +512,8 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   const int vecs_layer = B * row_vecs;  // vectors per block and layer
   const Divisor<POW2> by_layer{vecs_layer, POW2 ? ilog2(vecs_layer) : 0};
   const Divisor<POW2> by_row{row_vecs, POW2 ? ilog2(row_vecs) : 0};
+  const Divisor<POW2> by_hrow{B * VPR, POW2 ? ilog2(B * VPR) : 0};
+  const int order = a.vec_order;
 
   int next = 0;
   if (tid == 0) next = int(atomicAdd(&a.hdr->next_unit, 1u));
@@ -565,7 +592,8 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
         const int v = base + q * NT + tid;
         const int l = l0 + by_layer.div(v);
         const int rem = by_layer.mod(v);
-        const int o = by_row.div(rem), hv = by_row.mod(rem);
+        int o, hv;
+        split_vec<POW2>(rem, order, by_row, by_hrow, VPR, LOG_VPR, o, hv);
         const long long src = v < total ? s_src[o] : -1;
         kv[q] = make_uint4(0, 0, 0, 0);
         vv[q] = kv[q];
@@ -587,7 +615,9 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
         const int v = base + q * NT + tid;
         const int l = l0 + by_layer.div(v);
         const int rem = by_layer.mod(v);
-        const int o = v < total ? by_row.div(rem) : 0, hv = by_row.mod(rem);
+        int o, hv;
+        split_vec<POW2>(rem, order, by_row, by_hrow, VPR, LOG_VPR, o, hv);
+        if (v >= total) o = 0;
         const int c = hv & (VPR - 1);
         const uint4 kr = rotate_vec<D, STYLE>(kv[q], c, s_cs4 + o * (D / 4));
         if (v < total && s_src[o] >= 0) {
@@ -599,6 +629,44 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
       }
     }
   }
+}
+
+// Host tier, least-recently-used hot set: copy newly promoted facts from the
+// pinned (device-mapped) host arenas into their HBM slots.  Promotion i moves
+// fact rows [src_tok, src_tok + len) of every (layer, head) plane to rows
+// [dst_tok, dst_tok + len) of the hot planes; 16 bytes per thread-step.
+struct Promotion {
+  long long src_tok;  // token offset in the host planes
+  long long dst_tok;  // token offset in the hot planes
+  int32_t len;
+  int32_t pad;
+};
+
+__global__ void promote_kernel(const Promotion* __restrict__ list, int32_t n, int32_t planes,
+                               int32_t vec_per_row, const uint16_t* __restrict__ k_host,
+                               const uint16_t* __restrict__ v_host, long long host_plane,
+                               uint16_t* __restrict__ k_hot, uint16_t* __restrict__ v_hot,
+                               long long hot_plane) {
+  for (int32_t i = blockIdx.y; i < n; i += gridDim.y) {
+    const Promotion pr = list[i];
+    const long long per_plane = (long long)pr.len * vec_per_row;
+    const long long total = per_plane * planes;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+      const long long p = e / per_plane, r = e % per_plane;
+      const long long so = p * host_plane + pr.src_tok * vec_per_row * 8 + r * 8;
+      const long long dso = p * hot_plane + pr.dst_tok * vec_per_row * 8 + r * 8;
+      *reinterpret_cast<uint4*>(k_hot + dso) = ld_stream(k_host + so);
+      *reinterpret_cast<uint4*>(v_hot + dso) = ld_stream(v_host + so);
+    }
+  }
+}
+
+// Hot-table changes: entry pairs (fact, token offset in the hot planes or -1).
+__global__ void hot_table_kernel(int64_t* __restrict__ hot_off, const int64_t* __restrict__ pairs,
+                                 int32_t n) {
+  const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) hot_off[pairs[2 * i]] = pairs[2 * i + 1];
 }
 
 // RoPE frequencies, fp64: inv_freq_i = theta^(-2i/D), optionally with the

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <list>
 #include <new>
 #include <vector>
 
@@ -56,6 +57,23 @@ struct is_store {
   int32_t hot_facts = 0;
   int64_t* d_hot = nullptr;
   std::vector<int64_t> h_hot;
+  // least-recently-used hot set (IS_HOT_LRU): fixed slots of slot_tokens
+  int hot_policy = IS_HOT_STATIC;
+  int32_t slot_tokens = 0;
+  std::vector<int32_t> slot_owner;                   // fact in each slot, -1 free
+  std::vector<uint64_t> slot_tick;                   // last touch that used it
+  std::list<int32_t> lru;                            // slots, most recent first
+  std::vector<std::list<int32_t>::iterator> lru_at;  // position of each slot
+  std::vector<uint64_t> fact_tick;                   // last touch that asked for it
+  uint64_t tick = 0;
+  int64_t lru_hits = 0, lru_misses = 0, lru_promoted = 0, lru_promoted_tokens = 0;
+  // promotion staging: pinned host list + device copy, reused after `touch_done`
+  isk::Promotion* h_promo = nullptr;
+  isk::Promotion* d_promo = nullptr;
+  int64_t* h_pairs = nullptr;
+  int64_t* d_pairs = nullptr;
+  size_t promo_cap = 0;
+  cudaEvent_t touch_done = nullptr;
   // fact table
   int64_t* d_off = nullptr;
   int32_t* d_len = nullptr;
@@ -130,6 +148,11 @@ void free_store(is_store* s) {
   cudaFree(s->k_hot);
   cudaFree(s->v_hot);
   cudaFree(s->d_hot);
+  cudaFreeHost(s->h_promo);
+  cudaFreeHost(s->h_pairs);
+  cudaFree(s->d_promo);
+  cudaFree(s->d_pairs);
+  if (s->touch_done) cudaEventDestroy(s->touch_done);
   if (s->host_arena) {
     cudaFreeHost(s->k);
     cudaFreeHost(s->v);
@@ -203,6 +226,11 @@ int grow_stage(is_store* s, size_t elems, int64_t slot_elems) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Vector order of the inject kernel for a cache layout: the row index with
+// the larger cache stride runs fastest (token-major: slots; head-major:
+// heads).
+int vec_order_for(int64_t token_stride, int64_t head_stride) { return token_stride > head_stride ? 1 : 0; }
 
 }  // namespace
 
@@ -336,24 +364,28 @@ void is_store_destroy(is_store_t* s) {
   free_store(s);
 }
 
-int is_store_put_fact(is_store_t* s, const void* k_pre, const void* v, int32_t len,
-                      int32_t* fact_id_out) {
-  if (!s || !k_pre || !v || len <= 0) return IS_ERR_INVALID_ARG;
+int is_store_put_fact_window(is_store_t* s, const void* k_pre, const void* v, int32_t window_len,
+                             int32_t len, int32_t* fact_id_out) {
+  if (!s || !k_pre || !v || len <= 0 || window_len < 0) return IS_ERR_INVALID_ARG;
   if (s->num_facts >= s->cfg.max_facts || s->used_tokens + len > s->cfg.capacity_tokens)
     return IS_ERR_CAPACITY;
   DeviceGuard guard(s->device);
   const is_store_config_t& c = s->cfg;
   const size_t row = size_t(c.head_dim) * sizeof(uint16_t);
-  const size_t width = size_t(len) * row;                    // one fact run of one plane
-  const size_t dpitch = size_t(c.capacity_tokens) * row;     // distance between planes
+  const size_t width = size_t(len) * row;                          // one fact run of one plane
+  const size_t spitch = size_t(window_len + len) * row;            // caller's plane stride
+  const size_t dpitch = size_t(c.capacity_tokens) * row;           // store's plane stride
   const size_t height = size_t(c.num_layers) * size_t(c.num_kv_heads);
   const size_t off_bytes = size_t(s->used_tokens) * row;
+  const size_t skip = size_t(window_len) * row;                    // the window's rows
   char* kd = reinterpret_cast<char*>(s->k) + off_bytes;
   char* vd = reinterpret_cast<char*>(s->v) + off_bytes;
   const int32_t id = s->num_facts;
   const int64_t off = s->used_tokens;
-  if (cudaMemcpy2D(kd, dpitch, k_pre, width, width, height, cudaMemcpyDefault) != cudaSuccess ||
-      cudaMemcpy2D(vd, dpitch, v, width, width, height, cudaMemcpyDefault) != cudaSuccess ||
+  if (cudaMemcpy2D(kd, dpitch, static_cast<const char*>(k_pre) + skip, spitch, width, height,
+                   cudaMemcpyDefault) != cudaSuccess ||
+      cudaMemcpy2D(vd, dpitch, static_cast<const char*>(v) + skip, spitch, width, height,
+                   cudaMemcpyDefault) != cudaSuccess ||
       cudaMemcpy(s->d_off + id, &off, sizeof(off), cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(s->d_len + id, &len, sizeof(len), cudaMemcpyHostToDevice) != cudaSuccess) {
     cudaGetLastError();
@@ -365,6 +397,11 @@ int is_store_put_fact(is_store_t* s, const void* k_pre, const void* v, int32_t l
   s->used_tokens = off + len;
   if (fact_id_out) *fact_id_out = id;
   return IS_OK;
+}
+
+int is_store_put_fact(is_store_t* s, const void* k_pre, const void* v, int32_t len,
+                      int32_t* fact_id_out) {
+  return is_store_put_fact_window(s, k_pre, v, 0, len, fact_id_out);
 }
 
 int is_store_num_facts(const is_store_t* s, int32_t* out) {
@@ -410,7 +447,7 @@ int is_store_arena(const is_store_t* s, void** k, void** v, int64_t* plane_token
 
 int is_store_set_hot(is_store_t* s, const int32_t* fact_ids, int32_t n) {
   if (!s || n < 0 || (n > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
-  if (!s->host_arena) return IS_ERR_NOT_SUPPORTED;
+  if (!s->host_arena || s->hot_policy != IS_HOT_STATIC) return IS_ERR_NOT_SUPPORTED;
   std::vector<int64_t> hot(size_t(s->cfg.max_facts), -1);
   int64_t used = 0;
   int32_t count = 0;
@@ -445,6 +482,132 @@ int is_store_set_hot(is_store_t* s, const int32_t* fact_ids, int32_t n) {
   s->h_hot.swap(hot);
   s->hot_used = used;
   s->hot_facts = count;
+  return IS_OK;
+}
+
+int is_store_set_hot_policy(is_store_t* s, int policy, int32_t slot_tokens) {
+  if (!s || (policy != IS_HOT_STATIC && policy != IS_HOT_LRU)) return IS_ERR_INVALID_ARG;
+  if (!s->host_arena) return IS_ERR_NOT_SUPPORTED;
+  if (policy == IS_HOT_LRU && (slot_tokens < 1 || slot_tokens > s->hot_cap)) return IS_ERR_INVALID_ARG;
+  DeviceGuard guard(s->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return IS_ERR_CUDA;  // no batch may read the old set
+  // every fact cold
+  if (cudaMemset(s->d_hot, 0xFF, sizeof(int64_t) * size_t(s->cfg.max_facts)) != cudaSuccess) return IS_ERR_CUDA;
+  std::fill(s->h_hot.begin(), s->h_hot.end(), int64_t(-1));
+  s->hot_used = 0;
+  s->hot_facts = 0;
+  s->hot_policy = policy;
+  s->slot_tokens = policy == IS_HOT_LRU ? slot_tokens : 0;
+  const size_t nslots = policy == IS_HOT_LRU ? size_t(s->hot_cap / slot_tokens) : 0;
+  s->slot_owner.assign(nslots, -1);
+  s->slot_tick.assign(nslots, 0);
+  s->lru.clear();
+  s->lru_at.assign(nslots, s->lru.end());
+  for (size_t i = 0; i < nslots; ++i) s->lru_at[i] = s->lru.insert(s->lru.end(), int32_t(i));
+  s->fact_tick.assign(size_t(s->cfg.max_facts), 0);
+  s->tick = 0;
+  s->lru_hits = s->lru_misses = s->lru_promoted = s->lru_promoted_tokens = 0;
+  if (!s->touch_done && cudaEventCreateWithFlags(&s->touch_done, cudaEventDisableTiming) != cudaSuccess)
+    return IS_ERR_CUDA;
+  return IS_OK;
+}
+
+// LRU promotion of the listed facts: hits move to the front; misses that fit
+// a slot take the least recently used slot not used by this call.  The data
+// moves on `stream` (promote_kernel reads the mapped host arenas), then the
+// hot table is patched; later work on the stream sees the new set.
+int is_store_touch(is_store_t* s, const int32_t* fact_ids, int32_t n, void* stream, int32_t* promoted_out) {
+  if (!s || n < 0 || (n > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
+  if (!s->host_arena || s->hot_policy != IS_HOT_LRU) return IS_ERR_NOT_SUPPORTED;
+  DeviceGuard guard(s->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The staging of the previous touch must have been consumed.
+  if (cudaEventSynchronize(s->touch_done) != cudaSuccess) return IS_ERR_CUDA;
+  const uint64_t tick = ++s->tick;
+  std::vector<isk::Promotion> promo;
+  std::vector<int64_t> pairs;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t f = fact_ids[i];
+    if (f < 0 || f >= s->num_facts) continue;  // the batch itself reports it
+    if (s->fact_tick[size_t(f)] == tick) continue;  // listed twice in this call
+    s->fact_tick[size_t(f)] = tick;
+    const int64_t ho = s->h_hot[size_t(f)];
+    if (ho >= 0) {
+      const int32_t slot = int32_t(ho / s->slot_tokens);
+      s->lru.splice(s->lru.begin(), s->lru, s->lru_at[size_t(slot)]);
+      s->slot_tick[size_t(slot)] = tick;
+      ++s->lru_hits;
+      continue;
+    }
+    ++s->lru_misses;
+    if (s->lru.empty() || s->h_len[size_t(f)] > s->slot_tokens) continue;  // served from host
+    const int32_t slot = s->lru.back();
+    if (s->slot_tick[size_t(slot)] == tick) continue;  // every slot serves this call
+    const int32_t old = s->slot_owner[size_t(slot)];
+    if (old >= 0) {
+      s->h_hot[size_t(old)] = -1;
+      pairs.push_back(old);
+      pairs.push_back(-1);
+    } else {
+      ++s->hot_facts;
+    }
+    const int64_t dst = int64_t(slot) * s->slot_tokens;
+    s->slot_owner[size_t(slot)] = f;
+    s->slot_tick[size_t(slot)] = tick;
+    s->h_hot[size_t(f)] = dst;
+    s->lru.splice(s->lru.begin(), s->lru, s->lru_at[size_t(slot)]);
+    pairs.push_back(f);
+    pairs.push_back(dst);
+    promo.push_back(isk::Promotion{s->h_off[size_t(f)], dst, s->h_len[size_t(f)], 0});
+    s->lru_promoted_tokens += s->h_len[size_t(f)];
+  }
+  s->lru_promoted += int64_t(promo.size());
+  s->hot_used = int64_t(s->hot_facts) * s->slot_tokens;
+  if (promoted_out) *promoted_out = int32_t(promo.size());
+  if (promo.empty()) return IS_OK;
+  const size_t np = promo.size(), nq = pairs.size() / 2;
+  if (np > s->promo_cap || nq > s->promo_cap) {
+    const size_t cap = std::max(np, nq) * 2;
+    cudaFreeHost(s->h_promo);
+    cudaFreeHost(s->h_pairs);
+    cudaFree(s->d_promo);
+    cudaFree(s->d_pairs);
+    s->h_promo = nullptr;
+    s->h_pairs = nullptr;
+    s->d_promo = nullptr;
+    s->d_pairs = nullptr;
+    s->promo_cap = 0;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&s->h_promo), cap * sizeof(isk::Promotion), 0) != cudaSuccess ||
+        cudaHostAlloc(reinterpret_cast<void**>(&s->h_pairs), cap * 2 * sizeof(int64_t), 0) != cudaSuccess ||
+        dalloc(&s->d_promo, cap) != cudaSuccess || dalloc(&s->d_pairs, cap * 2) != cudaSuccess)
+      return IS_ERR_OOM;
+    s->promo_cap = cap;
+  }
+  std::memcpy(s->h_promo, promo.data(), np * sizeof(isk::Promotion));
+  std::memcpy(s->h_pairs, pairs.data(), pairs.size() * sizeof(int64_t));
+  const is_store_config_t& c = s->cfg;
+  if (cudaMemcpyAsync(s->d_promo, s->h_promo, np * sizeof(isk::Promotion), cudaMemcpyHostToDevice, st) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(s->d_pairs, s->h_pairs, pairs.size() * sizeof(int64_t), cudaMemcpyHostToDevice, st) !=
+          cudaSuccess)
+    return IS_ERR_CUDA;
+  const int vpr = c.head_dim / 8;
+  dim3 grid(unsigned(std::max(1, s->sm_count / 2)), unsigned(std::min<size_t>(np, 65535)));
+  isk::promote_kernel<<<grid, 256, 0, st>>>(s->d_promo, int32_t(np), c.num_layers * c.num_kv_heads, vpr,
+                                             s->k_view, s->v_view, int64_t(c.capacity_tokens) * c.head_dim,
+                                             s->k_hot, s->v_hot, s->hot_cap * c.head_dim);
+  isk::hot_table_kernel<<<unsigned((nq + 255) / 256), 256, 0, st>>>(s->d_hot, s->d_pairs, int32_t(nq));
+  if (cudaEventRecord(s->touch_done, st) != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
+  return IS_OK;
+}
+
+int is_store_lru_stats(const is_store_t* s, int64_t* hits, int64_t* misses, int64_t* promoted,
+                       int64_t* promoted_tokens) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  if (hits) *hits = s->lru_hits;
+  if (misses) *misses = s->lru_misses;
+  if (promoted) *promoted = s->lru_promoted;
+  if (promoted_tokens) *promoted_tokens = s->lru_promoted_tokens;
   return IS_OK;
 }
 
@@ -507,7 +670,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.st = s->d_status;
   isk::plan_kernel<kPlanThreads><<<1, kPlanThreads, 0, st>>>(pa);
 
-  isk::InjectArgs ia;
+  isk::InjectArgs ia{};
   ia.k_store = s->k_view;
   ia.v_store = s->v_view;
   ia.k_hot = s->k_hot;
@@ -533,6 +696,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.hs = c.head_stride;
   ia.num_blocks = c.num_blocks;
   ia.B = c.block_size;
+  ia.vec_order = vec_order_for(c.token_stride, c.head_stride);
   ia.slot_out = slot_out;
   ia.seg = s->ws_seg;
   ia.req_tok0 = s->ws_tok0;
@@ -591,6 +755,10 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
   const int64_t n_slots = slot_out ? slot_cap : 0;
   int rc = grow_stage(s, n_off + n_ids + n_sp + n_bt + 4, n_slots);
   if (rc != IS_OK) return rc;
+  if (s->hot_policy == IS_HOT_LRU) {  // promote this batch's cold facts first
+    rc = is_store_touch(s, fact_ids, num_ids, stream, nullptr);
+    if (rc != IS_OK) return rc;
+  }
   // Pack the four index arrays into one pinned buffer: one host-to-device copy.
   int32_t* h = s->host_stage;
   std::memcpy(h, req_off, n_off * 4);
@@ -827,7 +995,7 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   pa.st = status;
   isk::plan_kernel<kPlanThreads><<<1, kPlanThreads, 0, st>>>(pa);
 
-  isk::InjectArgs ia;
+  isk::InjectArgs ia{};
   ia.k_store = static_cast<const uint16_t*>(k_store);
   ia.v_store = static_cast<const uint16_t*>(v_store);
   ia.plane = plane_tokens * c.head_dim;
@@ -849,6 +1017,7 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   ia.hs = k.head_stride;
   ia.num_blocks = k.num_blocks;
   ia.B = k.block_size;
+  ia.vec_order = vec_order_for(k.token_stride, k.head_stride);
   ia.slot_out = slot_out;
   ia.seg = pa.seg;
   ia.req_tok0 = pa.req_tok0;

@@ -106,6 +106,21 @@ class FactStore:
         k_pre, v = k_pre.contiguous(), v.contiguous()
         return B.is_store_put_fact(self.handle, k_pre.data_ptr(), v.data_ptr(), k_pre.shape[2])
 
+    def put_fact_window(self, k_pre: torch.Tensor, v: torch.Tensor, window_len: int) -> int:
+        """K/V of an encoded [window | fact], bf16 [L][H][window_len + len][D]:
+        store only the fact's tokens (context-window encoding)."""
+        if k_pre.shape != v.shape or k_pre.dim() != 4 or k_pre.shape[0] != self.L \
+                or k_pre.shape[1] != self.H or k_pre.shape[3] != self.D:
+            raise ValueError("encoding must be [L][H][window_len + len][D]")
+        if k_pre.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bf16")
+        n = k_pre.shape[2] - window_len
+        if window_len < 0 or n <= 0:
+            raise ValueError("window_len must leave at least one fact token")
+        k_pre, v = k_pre.contiguous(), v.contiguous()
+        return B.is_store_put_fact_window(self.handle, k_pre.data_ptr(), v.data_ptr(),
+                                          window_len, n)
+
     @property
     def num_facts(self) -> int:
         return B.is_store_num_facts(self.handle)
@@ -135,6 +150,23 @@ class FactStore:
         import numpy as np
         ids = np.ascontiguousarray(np.asarray(fact_ids, dtype=np.int32))
         B.is_store_set_hot(self.handle, ids.ctypes.data, ids.size)
+
+    def set_hot_policy(self, lru: bool, slot_tokens: int = 0) -> None:
+        """Host tier: LRU hot set with slots of slot_tokens, or back to static."""
+        B.is_store_set_hot_policy(self.handle, B.IS_HOT_LRU if lru else B.IS_HOT_STATIC,
+                                  slot_tokens)
+
+    def touch(self, fact_ids, stream: int | None = None) -> int:
+        """LRU: promote these facts (host ints) on the stream; returns how many."""
+        import numpy as np
+        ids = np.ascontiguousarray(np.asarray(fact_ids, dtype=np.int32))
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device).cuda_stream
+        return B.is_store_touch(self.handle, ids.ctypes.data, ids.size, stream)
+
+    def lru_stats(self) -> dict:
+        h, m, p, t = B.is_store_lru_stats(self.handle)
+        return dict(hits=h, misses=m, promoted=p, promoted_tokens=t)
 
     def tier_info(self) -> dict:
         t, cap, used, nf = B.is_store_tier_info(self.handle)

@@ -266,11 +266,12 @@ def sweep(model: Model, R: int, k: int, seed: int = 0, num_facts: int = 50_000) 
 
 def offload(seed: int = 0, num_facts: int = 100_000, R: int = 100, k: int = 50,
             zipf_s: float = 1.1, hot_fraction: float = 0.2,
-            slots_per_request: int = 4096) -> Workload:
+            slots_per_request: int = 4096, extra_batches: int = 0) -> Workload:
     """Qwen2.5-7B shapes; facts of 16..48 tokens (mean 32) in pinned host
     memory; requests draw k distinct facts by Zipf(zipf_s) over a seeded rank
     order; the hot set is the top hot_fraction of facts by rank.  The hot fact
-    ids go to notes["hot"]."""
+    ids go to notes["hot"]; notes["more_ids"] holds extra_batches further
+    draws of the same shape (CSR ids, same offsets) for streams of batches."""
     rng = np.random.default_rng(seed)
     lens = uniform_lengths(rng, num_facts, 16, 48)
     rank_to_fact = rng.permutation(num_facts).astype(np.int32)
@@ -280,9 +281,11 @@ def offload(seed: int = 0, num_facts: int = 100_000, R: int = 100, k: int = 50,
     mb = slots_per_request // 16
     batch = make_batch(rng, ids, 64, 16, R * mb, mb)
     n_hot = int(round(hot_fraction * num_facts))
+    more = [np.concatenate([zipf_distinct_ids(rng, rank_to_fact, probs, k) for _ in range(R)])
+            for _ in range(extra_batches)]
     return Workload(f"{QWEN25_7B.name} offload R={R} k={k}", QWEN25_7B, lens, batch, seed,
                     notes=dict(hot=rank_to_fact[:n_hot].copy(), zipf_s=zipf_s,
-                               hot_fraction=hot_fraction))
+                               hot_fraction=hot_fraction, more_ids=more))
 
 
 # ---------------------------------------------------------------------------

@@ -79,3 +79,68 @@ def test_set_hot_errors_keep_previous_set():
     assert e.value.status == B.IS_ERR_NOT_SUPPORTED
     assert dev.tier_info()["tier"] == B.IS_TIER_DEVICE
     dev.close()
+
+
+def _host_inject(store, wl):
+    from gpu_common import make_cache
+    from test_gpu_parity import to_bits
+    b = wl.batch
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
+    k, v, desc = make_cache(wl)
+    n_tok = wl.tokens()
+    slots = torch.empty(max(n_tok, 1), dtype=torch.int64).pin_memory()
+    rc = store.inject_host(pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos), pin(b.block_tables),
+                           desc, slots[:n_tok])
+    return rc, slots[:n_tok].numpy().copy(), to_bits(k), to_bits(v)
+
+
+def test_lru_hot_set_parity_and_promotion():
+    """LRU policy: the host entry point promotes each batch's cold facts into
+    HBM slots before injecting; results equal the oracle's every time, the
+    second pass over the same ids finds them hot, and a slot that is too
+    small for a fact leaves it on the host."""
+    _need_gpu()
+    model = synth.Model("qwen-like", 2, 4, 128, 1e6)
+    wl = _ragged(model, seed=31, R=5, max_k=8, lens=(1, 40), num_facts=30)
+    lens = wl.fact_lens
+    slot = 32
+    store = make_store(wl, host_tier=True, hot_capacity_tokens=slot * 6)
+    store.set_hot_policy(True, slot)
+    want = oracle_run(wl)
+    for rep in range(3):
+        rc, slots, gk, gv = _host_inject(store, wl)
+        assert_parity(want, (rc, slots, gk, gv))
+    st = store.lru_stats()
+    ids = wl.batch.fact_ids
+    assert st["promoted"] >= 1 and st["hits"] >= 1
+    assert st["hits"] + st["misses"] == 3 * len(np.unique(ids))  # each call counts distinct ids
+    info = store.tier_info()
+    assert info["hot_facts"] <= 6 and info["hot_used"] == info["hot_facts"] * slot
+    # explicit touch of facts that fit: all become hot (6 slots, 3 facts)
+    fit = [int(f) for f in np.flatnonzero(lens <= slot)[:3]]
+    store.touch(fit)
+    torch.cuda.synchronize()
+    assert_parity(want, _host_inject(store, wl))
+    with pytest.raises(B.InjectError):
+        store.set_hot([0])  # static API refused under LRU
+    store.close()
+
+
+def test_lru_eviction_keeps_results_exact():
+    """Far more distinct facts than slots: every batch evicts; results stay
+    exact."""
+    _need_gpu()
+    model = synth.Model("llama-like", 2, 8, 128, 5e5, llama3=True)
+    rng = np.random.default_rng(5)
+    lens = rng.integers(4, 20, 60).astype(np.int32)
+    store = None
+    for rep in range(4):
+        ids = [rng.choice(60, 6, replace=False) for _ in range(3)]
+        batch = synth.make_batch(rng, ids, [0, 17, 40], 16, 3 * 12, 12)
+        wl = synth.Workload("lru", model, lens, batch, seed=4)
+        if store is None:
+            store = make_store(wl, host_tier=True, hot_capacity_tokens=20 * 5)
+            store.set_hot_policy(True, 20)
+        assert_parity(oracle_run(wl), _host_inject(store, wl))
+    assert store.lru_stats()["promoted"] > 5
+    store.close()

@@ -232,3 +232,59 @@ def test_gpu_injected_cache_serves_the_query():
     err = np.abs(got - want).max()
     assert err < 3e-2 * np.abs(want).max()
     assert err < 0.1 * np.abs(causal - want).max()
+
+
+@pytest.mark.gpu
+def test_gpu_window_encoding_through_the_store_equals_prompt_injection():
+    """Context-window encoding end to end on the CUDA path: each fact is
+    encoded after everything before it (at an arbitrary offset), the encoder's
+    K/V of [window | fact] go to is_store_put_fact_window (window dropped), the
+    GPU injects, the query is prefilled against the cache.  The output equals
+    the ordinary causal prefill at bf16 level."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from kv_cache_injection_gather_b200 import FactStore, RopeConfig, cache_desc
+
+    model = TinyDecoder(seed=8)
+    prefix, facts, query = _setup(seed=9, lens=(5, 3, 6))
+    P, Q, L, H, D = len(prefix), len(query), model.L, model.nkv, model.D
+    lens = [len(f) for f in facts]
+    seq = [prefix] + facts
+    store = FactStore(L, H, D, RopeConfig(theta=1e4), sum(lens), len(facts))
+    to_bf = lambda a: torch.from_numpy(oracle.f64_to_bf16(a).view(np.int16)).view(torch.bfloat16)  # noqa: E731
+    for j, f in enumerate(facts):
+        enc = np.concatenate(seq[: j + 1] + [f])
+        n = len(enc)
+        _, caps = model.run(enc, 31 + np.arange(n), np.tril(np.ones((n, n), bool)))
+        k = np.ascontiguousarray(np.stack([c[0] for c in caps]).transpose(0, 2, 1, 3))
+        v = np.ascontiguousarray(np.stack([c[1] for c in caps]).transpose(0, 2, 1, 3))
+        kt, vt = to_bf(k), to_bf(v)
+        fid = store.put_fact_window(kt.cuda() if j % 2 else kt, vt.cuda() if j % 2 else vt, n - len(f))
+        kr, vr = store.read_fact(fid)  # only the fact's rows were kept
+        assert torch.equal(kr.cpu(), kt[:, :, n - len(f):]) and torch.equal(vr.cpu(), vt[:, :, n - len(f):])
+    B, NB = 16, 4
+    bt = torch.tensor([[2, 0, 3, 1]], dtype=torch.int32, device="cuda")
+    kc = torch.zeros((L, NB, B, H, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    store.inject(torch.tensor([0, 3], dtype=torch.int32, device="cuda"),
+                 torch.arange(3, dtype=torch.int32, device="cuda"),
+                 torch.tensor([P], dtype=torch.int32, device="cuda"), bt, cache_desc(kc, vc))
+    assert store.last_error()[0] == 0
+    store.close()
+    S = sum(lens)
+    pos = np.arange(P, P + S)
+    slot = torch.from_numpy(bt[0].cpu().numpy()[pos // B] * B + pos % B).cuda()
+    to64 = lambda t: oracle.bf16_to_f64(t.view(torch.int16).cpu().numpy().view(np.uint16))  # noqa: E731
+    kinj = to64(kc.view(L, NB * B, H, D)[:, slot])
+    vinj = to64(vc.view(L, NB * B, H, D)[:, slot])
+    _, pre_caps = model.run(prefix, np.arange(P), np.tril(np.ones((P, P), bool)))
+    past = [(np.concatenate([pre_caps[l][2], kinj[l]]), np.concatenate([pre_caps[l][1], vinj[l]]))
+            for l in range(L)]
+    allowed = np.concatenate([np.ones((Q, P + S), bool), np.tril(np.ones((Q, Q), bool))], axis=1)
+    got, _ = model.run(query, np.arange(P + S, P + S + Q), allowed, past=past)
+    want, _ = _prefill(model, prefix, facts, query, "causal")
+    local, _ = _prefill(model, prefix, facts, query, "local")
+    err = np.abs(got - want).max()
+    assert err < 3e-2 * np.abs(want).max()
+    assert err < 0.1 * np.abs(local - want).max()
