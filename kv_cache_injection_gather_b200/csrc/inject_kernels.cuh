@@ -28,6 +28,10 @@
 #ifndef IS_UNITS_PER_CTA
 #define IS_UNITS_PER_CTA 256
 #endif
+// 1: the copy loop keeps two half-chunks in flight (software pipeline).
+#ifndef IS_PIPELINE
+#define IS_PIPELINE 1
+#endif
 
 namespace isk {
 
@@ -585,10 +589,12 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
     const int total = (l1 - l0) * vecs_layer;
     const uint16_t* kst = a.k_store;
     const uint16_t* vst = a.v_store;
-    for (int base = 0; base < total; base += NT * VPT) {
-      uint4 kv[VPT], vv[VPT];
+    constexpr int HV = IS_PIPELINE ? VPT / 2 : VPT;  // vectors per thread per stage
+
+    // One stage: vectors base + q*NT + tid, q < HV, of the unit's flat range.
+    auto load_stage = [&](uint4 (&kv)[HV], uint4 (&vv)[HV], int base) {
 #pragma unroll
-      for (int q = 0; q < VPT; ++q) {
+      for (int q = 0; q < HV; ++q) {
         const int v = base + q * NT + tid;
         const int l = l0 + by_layer.div(v);
         const int rem = by_layer.mod(v);
@@ -610,8 +616,10 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
           }
         }
       }
+    };
+    auto store_stage = [&](const uint4 (&kv)[HV], const uint4 (&vv)[HV], int base) {
 #pragma unroll
-      for (int q = 0; q < VPT; ++q) {
+      for (int q = 0; q < HV; ++q) {
         const int v = base + q * NT + tid;
         const int l = l0 + by_layer.div(v);
         const int rem = by_layer.mod(v);
@@ -627,7 +635,28 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
           st_stream(a.v_cache + dst, vv[q]);
         }
       }
+    };
+
+#if IS_PIPELINE
+    // Two stages in flight: the next stage's loads are issued before the
+    // current stage is rotated and stored (stage control is uniform).
+    const int step = NT * HV;
+    uint4 ka[HV], va[HV], kb[HV], vb[HV];
+    if (total > 0) load_stage(ka, va, 0);
+    for (int base = 0; base < total; base += 2 * step) {
+      if (base + step < total) load_stage(kb, vb, base + step);
+      store_stage(ka, va, base);
+      if (base + step >= total) break;
+      if (base + 2 * step < total) load_stage(ka, va, base + 2 * step);
+      store_stage(kb, vb, base + step);
     }
+#else
+    for (int base = 0; base < total; base += NT * HV) {
+      uint4 kv[HV], vv[HV];
+      load_stage(kv, vv, base);
+      store_stage(kv, vv, base);
+    }
+#endif
   }
 }
 
