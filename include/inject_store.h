@@ -257,6 +257,13 @@ int is_inject_batch_host(is_store_t* store, int32_t num_requests,
  * NULL, receives the offending index (request, CSR entry or block). */
 int is_last_error(is_store_t* store, void* stream, int64_t* detail_out);
 
+/* As is_last_error, but waits at most timeout_ms for `stream` (polling,
+ * never blocking the calling thread longer): IS_ERR_TIMEOUT if the stream's
+ * work has not finished by then (nothing is cleared; call again later).  For
+ * callers that must not hang on a stalled stream. */
+int is_last_error_timeout(is_store_t* store, void* stream, int32_t timeout_ms,
+                          int64_t* detail_out);
+
 /* ---- measurement -------------------------------------------------------- */
 
 /* Enable (1) or disable (0) CUDA-event timing of the inject kernel itself

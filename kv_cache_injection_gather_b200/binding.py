@@ -89,6 +89,7 @@ _SIGNATURES = {
     "is_inject_batch_host": (ctypes.c_int, [_P, _I32, _P, _P, _I32, _P, _P, _I32,
                                             ctypes.POINTER(is_cache_t), _P, _I64, _P]),
     "is_last_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(_I64)]),
+    "is_last_error_timeout": (ctypes.c_int, [_P, _P, _I32, ctypes.POINTER(_I64)]),
     "is_store_set_timing": (ctypes.c_int, [_P, ctypes.c_int]),
     "is_store_kernel_time": (ctypes.c_int, [_P, ctypes.POINTER(_F64), ctypes.POINTER(_I64)]),
     "is_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -201,6 +202,12 @@ def is_inject_batch_host(store: int, num_requests: int, req_fact_offsets: int, f
 def is_last_error(store: int, stream: int = 0) -> tuple[int, int]:
     detail = _I64()
     rc = _lib.is_last_error(store, stream, ctypes.byref(detail))
+    return rc, detail.value
+
+
+def is_last_error_timeout(store: int, stream: int, timeout_ms: int) -> tuple[int, int]:
+    detail = _I64()
+    rc = _lib.is_last_error_timeout(store, stream, timeout_ms, ctypes.byref(detail))
     return rc, detail.value
 
 

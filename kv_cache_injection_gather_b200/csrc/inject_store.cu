@@ -3,10 +3,12 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <list>
 #include <new>
+#include <thread>
 #include <vector>
 
 #include "inject_store.h"
@@ -798,6 +800,21 @@ int is_last_error(is_store_t* s, void* stream, int64_t* detail) {
   if (h.code != 0 && cudaMemset(s->d_status, 0, sizeof(h)) != cudaSuccess) return IS_ERR_CUDA;
   if (detail) *detail = h.detail;
   return h.code;
+}
+
+int is_last_error_timeout(is_store_t* s, void* stream, int32_t timeout_ms, int64_t* detail) {
+  if (!s || timeout_ms < 0) return IS_ERR_INVALID_ARG;
+  DeviceGuard guard(s->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
+  for (;;) {
+    const cudaError_t q = cudaStreamQuery(st);
+    if (q == cudaSuccess) break;
+    if (q != cudaErrorNotReady) return IS_ERR_CUDA;
+    if (std::chrono::steady_clock::now() >= deadline) return IS_ERR_TIMEOUT;
+    std::this_thread::sleep_for(std::chrono::microseconds(200));
+  }
+  return is_last_error(s, stream, detail);
 }
 
 int is_store_set_timing(is_store_t* s, int enable) {

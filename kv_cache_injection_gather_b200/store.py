@@ -214,6 +214,12 @@ class FactStore:
             stream = torch.cuda.current_stream(self.device).cuda_stream
         return B.is_last_error(self.handle, stream)
 
+    def last_error_timeout(self, timeout_ms: int, stream: int | None = None) -> tuple[int, int]:
+        """As last_error, waiting at most timeout_ms (IS_ERR_TIMEOUT otherwise)."""
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device).cuda_stream
+        return B.is_last_error_timeout(self.handle, stream, timeout_ms)
+
     def set_timing(self, enable: bool) -> None:
         B.is_store_set_timing(self.handle, enable)
 

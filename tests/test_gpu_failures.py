@@ -1,0 +1,83 @@
+"""Failure detection without a GPU fault: a stream held back by a short
+device sleep on another stream (the GPU stays responsive), ids and tables
+that the device-side checks reject; every wait is bounded.  No kernel of
+this library spins or waits on another."""
+from __future__ import annotations
+
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_common import batch_tensors, make_cache, make_store
+from kv_cache_injection_gather_b200 import binding as B
+
+pytestmark = pytest.mark.gpu
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def test_bounded_wait_times_out_then_recovers():
+    _need_gpu()
+    from kv_cache_injection_gather_b200 import binding
+    wl = synth.tiny(0)
+    store = make_store(wl)
+    k, v, desc = make_cache(wl)
+    ro, ids, sp, bt = batch_tensors(wl.batch)
+    s = torch.cuda.Stream()
+    # the batch's stream waits for a bounded device sleep (~0.3 s at ~2 GHz)
+    # queued on another stream
+    gate = torch.cuda.Event()
+    blocker = torch.cuda.Stream()
+    with torch.cuda.stream(blocker):
+        torch.cuda._sleep(int(6e8))
+        gate.record(blocker)
+    s.wait_event(gate)
+    with torch.cuda.stream(s):
+        store.inject(ro, ids, sp, bt, desc, stream=s.cuda_stream)
+    t0 = time.perf_counter()
+    rc, _ = store.last_error_timeout(50, s.cuda_stream)
+    waited = time.perf_counter() - t0
+    assert rc == binding.IS_ERR_TIMEOUT and waited < 0.25
+    rc, _ = store.last_error_timeout(30_000, s.cuda_stream)
+    assert rc == binding.IS_OK
+    store.close()
+
+
+def test_device_status_is_cleared_after_reading():
+    _need_gpu()
+    wl = synth.tiny(0)
+    store = make_store(wl)
+    k, v, desc = make_cache(wl)
+    ro, ids, sp, bt = batch_tensors(wl.batch)
+    bad = ids.clone()
+    bad[0] = 10_000
+    store.inject(ro, bad, sp, bt, desc)
+    rc, detail = store.last_error()
+    assert rc == B.IS_ERR_BAD_FACT_ID and detail == 0  # request 0
+    assert store.last_error()[0] == B.IS_OK          # read once, then cleared
+    store.inject(ro, ids, sp, bt, desc)               # the store keeps working
+    assert store.last_error()[0] == B.IS_OK
+    store.close()
+
+
+def test_host_entry_point_reports_device_errors():
+    _need_gpu()
+    wl = synth.tiny(0)
+    store = make_store(wl)
+    k, v, desc = make_cache(wl)
+    b = wl.batch
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
+    bt = b.block_tables.copy()
+    bt[0, 2] = 9999  # the first fact's tokens start at position 32: block 2
+    rc = store.inject_host(pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos), pin(bt), desc)
+    assert rc == B.IS_ERR_BAD_BLOCK
+    rc = store.inject_host(pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos),
+                           pin(b.block_tables), desc)
+    assert rc == B.IS_OK
+    store.close()
