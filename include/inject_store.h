@@ -264,10 +264,16 @@ int is_last_error(is_store_t* store, void* stream, int64_t* detail_out);
 int is_last_error_timeout(is_store_t* store, void* stream, int32_t timeout_ms,
                           int64_t* detail_out);
 
+/* Batches with at most max_requests requests (0..8; default 8) and at most
+ * 256 fact ids run as one kernel that composes the batch in every CTA
+ * instead of a plan kernel followed by the inject kernel (lower latency for
+ * small batches; same results).  0 always uses the two-kernel path. */
+int is_store_set_small_batch_limit(is_store_t* store, int32_t max_requests);
+
 /* ---- measurement -------------------------------------------------------- */
 
 /* Enable (1) or disable (0) CUDA-event timing of the inject kernel itself
- * (the plan kernel excluded).  While enabled each batch records two events
+ * (the plan kernel excluded; for small batches the single kernel).  While enabled each batch records two events
  * on its stream around the inject kernel. */
 int is_store_set_timing(is_store_t* store, int enable);
 

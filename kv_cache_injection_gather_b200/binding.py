@@ -91,6 +91,7 @@ _SIGNATURES = {
     "is_last_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(_I64)]),
     "is_last_error_timeout": (ctypes.c_int, [_P, _P, _I32, ctypes.POINTER(_I64)]),
     "is_store_set_timing": (ctypes.c_int, [_P, ctypes.c_int]),
+    "is_store_set_small_batch_limit": (ctypes.c_int, [_P, _I32]),
     "is_store_kernel_time": (ctypes.c_int, [_P, ctypes.POINTER(_F64), ctypes.POINTER(_I64)]),
     "is_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "is_store_set_hot": (ctypes.c_int, [_P, _P, _I32]),
@@ -209,6 +210,10 @@ def is_last_error_timeout(store: int, stream: int, timeout_ms: int) -> tuple[int
     detail = _I64()
     rc = _lib.is_last_error_timeout(store, stream, timeout_ms, ctypes.byref(detail))
     return rc, detail.value
+
+
+def is_store_set_small_batch_limit(store: int, max_requests: int) -> None:
+    check(_lib.is_store_set_small_batch_limit(store, max_requests), "is_store_set_small_batch_limit")
 
 
 def is_store_set_timing(store: int, enable: bool) -> None:

@@ -76,6 +76,26 @@ __device__ __forceinline__ void record_error(DevStatus* st, int32_t code, long l
 
 // ---------------------------------------------------------------- plan kernel
 
+// Work-unit size (layers per unit lpu, units per block upb).  A batch whose
+// one-layer units fit in about one wave of the grid uses one layer per unit:
+// everything is in flight at once (latency).  Larger batches aim at
+// ~IS_UNITS_PER_CTA units per CTA, so the dynamic schedule's tail (at most
+// one unit) stays short, with at least two layers per unit so a unit's
+// set-up (slot walk, cos/sin table) is shared by more than one layer.
+__device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32_t grid_ctas,
+                                          int32_t& lpu, int32_t& upb) {
+  const long long grid = grid_ctas;
+  upb = 1;
+  if (total_blocks > 0 && (long long)total_blocks * L <= 2 * grid) {
+    upb = L;
+  } else if (total_blocks > 0) {
+    const long long want = (grid * IS_UNITS_PER_CTA + total_blocks - 1) / total_blocks;
+    upb = int32_t(max(1LL, min(want, (long long)max(1, L / 2))));
+  }
+  lpu = (L + upb - 1) / upb;
+  upb = (L + lpu - 1) / lpu;
+}
+
 struct PlanArgs {
   int32_t R;
   const int32_t* req_off;    // [R+1]
@@ -230,22 +250,8 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   const bool over_blocks = total_blocks > a.max_batch_blocks;
 
   if (tid == 0) {
-    // Work-unit size (layers per unit).  A batch whose one-layer units fit in
-    // about one wave of the grid uses one layer per unit: everything is in
-    // flight at once (latency).  Larger batches aim at ~IS_UNITS_PER_CTA
-    // units per CTA, so the dynamic schedule's tail (at most one unit) stays
-    // short, with at least two layers per unit so a unit's set-up (slot walk,
-    // cos/sin table) is shared by more than one layer's copy.
-    const long long grid = a.grid_ctas;
-    int32_t upb = 1;
-    if (total_blocks > 0 && (long long)total_blocks * a.L <= 2 * grid) {
-      upb = a.L;
-    } else if (total_blocks > 0) {
-      const long long want = (grid * IS_UNITS_PER_CTA + total_blocks - 1) / total_blocks;
-      upb = int32_t(max(1LL, min(want, (long long)max(1, a.L / 2))));
-    }
-    const int32_t lpu = (a.L + upb - 1) / upb;
-    upb = (a.L + lpu - 1) / lpu;
+    int32_t lpu, upb;
+    unit_size(total_blocks, a.L, a.grid_ctas, lpu, upb);
     a.hdr->layers_per_unit = lpu;
     a.hdr->units_per_block = upb;
     a.hdr->total_blocks = total_blocks;
@@ -317,6 +323,7 @@ struct InjectArgs {
   int64_t ls, bs, ts, hs;    // cache strides (elements)
   int32_t num_blocks, B;
   int32_t vec_order;         // 0: (slot, head) rows, 1: (head, slot) rows
+  int32_t fact_len_count;    // number of facts (small-batch kernel's id check)
   int64_t* slot_out;
   const int32_t* seg;
   const long long* req_tok0;
@@ -478,38 +485,31 @@ __device__ __forceinline__ void split_vec(int rem, int order, const Divisor<POW2
   }
 }
 
-// Persistent gather-rotate-scatter kernel.  Work unit u covers global block
-// gb = u % total_blocks and layers [lg * lpu, min(L, (lg + 1) * lpu)),
-// lg = u / total_blocks, so CTAs running side by side read neighbouring
-// tokens of the same layers.  Units are taken from an atomic counter; the
-// next unit is fetched while the current one is copied.
-//
-// Inside a unit the vectors are numbered v = ((l - l0) * B + o) * H * D/8 +
-// h * D/8 + c (layer, in-block slot, head, 16-byte vector of the row), so
-// consecutive threads write consecutive 16-byte words of the token-major
-// cache and read whole 256-byte head rows of the store.  POW2: H and B are
-// powers of two (all index splits are shifts).  HOST_TIER: the store lives
-// in pinned host memory read over the host link, except the facts that also
-// sit in the HBM hot arenas; the source of every slot is chosen per fact.
-template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER>
-__global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
+// Shared-memory state of a CTA of the inject kernels, reused unit after unit.
+template <bool HOST_TIER>
+struct UnitShared {
+  long long src[kMaxBlockSize];  // store token of each in-block slot (-1: none)
+  // host tier: per-slot K/V row bases (token offset applied) and plane stride
+  const uint16_t* kb[HOST_TIER ? kMaxBlockSize : 1];
+  const uint16_t* vb[HOST_TIER ? kMaxBlockSize : 1];
+  long long pl[HOST_TIER ? kMaxBlockSize : 1];
+};
+
+// One work unit: cache block b (logical, of request r) x layers [l0, l1).
+// j is the CSR index of the first fact with a token in the block, seg[] the
+// facts' segment offsets (global or shared memory), j1 the end of the
+// request's CSR range, len_r its segment length, tok0 its first slot-mapping
+// index.  The slot mapping is written when write_slots.  Vector order inside
+// a layer: split_vec.  Every thread of the CTA calls this with the same
+// arguments; the caller puts a barrier between units.
+template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER>
+__device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TIER>& sm,
+                                         float4* s_cs4, int r, int b, int j_first,
+                                         const int32_t* seg, int j1, int start, int len_r,
+                                         long long tok0, int l0, int l1, bool write_slots) {
   constexpr int VPR = D / 8;  // 16-byte vectors per head row
   constexpr int LOG_VPR = (VPR == 4) ? 2 : (VPR == 8) ? 3 : (VPR == 16) ? 4 : 5;
-  extern __shared__ float4 s_cs4[];            // [B * D/4] cos/sin of the block
-  __shared__ long long s_src[kMaxBlockSize];  // store token of each slot (-1: none)
-  // host tier: per-slot K/V row bases (token offset applied) and plane stride
-  __shared__ const uint16_t* s_kb[HOST_TIER ? kMaxBlockSize : 1];
-  __shared__ const uint16_t* s_vb[HOST_TIER ? kMaxBlockSize : 1];
-  __shared__ long long s_pl[HOST_TIER ? kMaxBlockSize : 1];
-  __shared__ int s_unit;
-
   const int tid = threadIdx.x;
-  // When launched as a programmatic dependent of the plan kernel, wait here
-  // for its results; without such a launch this returns at once.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int total_units = a.hdr->total_units;
-  const int total_blocks = a.hdr->total_blocks;
-  const int lpu = a.hdr->layers_per_unit;
   const int B = a.B;
   const int H = a.H;
   const int row_vecs = H * VPR;         // vectors per token (all heads)
@@ -518,73 +518,57 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   const Divisor<POW2> by_row{row_vecs, POW2 ? ilog2(row_vecs) : 0};
   const Divisor<POW2> by_hrow{B * VPR, POW2 ? ilog2(B * VPR) : 0};
   const int order = a.vec_order;
+  long long* s_src = sm.src;
+  const uint16_t** s_kb = sm.kb;
+  const uint16_t** s_vb = sm.vb;
+  long long* s_pl = sm.pl;
 
-  int next = 0;
-  if (tid == 0) next = int(atomicAdd(&a.hdr->next_unit, 1u));
-  for (;;) {
-    __syncthreads();  // the previous unit's tables are no longer read
-    if (tid == 0) {
-      s_unit = next;
-      if (next < total_units) next = int(atomicAdd(&a.hdr->next_unit, 1u));
-    }
-    __syncthreads();
-    const int u = s_unit;
-    if (u >= total_units) break;
-    const int gb = u % total_blocks;
-    const int lg = u / total_blocks;
-    const BlockDesc d = a.desc[gb];
-    const int r = d.r;
-    const int start = a.start_pos[r];
-    const int j1 = a.req_off[r + 1];
-    const long long tok0 = a.req_tok0[r];
-    const int len_r = int(a.req_tok0[r + 1] - tok0);
-    const int blk_pos = d.b * B;                       // position of in-block slot 0
-    const int o_lo = max(start - blk_pos, 0);
-    const int o_hi = min(start + len_r - blk_pos, B);  // exclusive
-    const int phys = a.block_tables[(long long)r * a.max_blocks + d.b];
-    const bool phys_ok = phys >= 0 && phys < a.num_blocks;
-    const int l0 = lg * lpu, l1 = min(a.L, l0 + lpu);
+  const int blk_pos = b * B;                         // position of in-block slot 0
+  const int o_lo = max(start - blk_pos, 0);
+  const int o_hi = min(start + len_r - blk_pos, B);  // exclusive
+  const int phys = a.block_tables[(long long)r * a.max_blocks + b];
+  const bool phys_ok = phys >= 0 && phys < a.num_blocks;
 
-    // Store token of each in-block slot: walk forward from the block's
-    // first fact (facts cover consecutive segment ranges).
-    if (tid < B) {
-      const int o = tid;
-      long long src = -1;
-      if (o >= o_lo && o < o_hi) {
-        const int i = blk_pos + o - start;  // segment index
-        int j = d.j;
-        while (j + 1 < j1 && a.seg[j + 1] <= i) ++j;
-        const int f = a.fact_ids[j];
-        const int t = i - a.seg[j];
-        src = a.fact_off[f] + t;
-        if (HOST_TIER) {
-          const long long ho = a.hot_off[f];
-          if (ho >= 0) {
-            s_kb[o] = a.k_hot + (ho + t) * D;
-            s_vb[o] = a.v_hot + (ho + t) * D;
-            s_pl[o] = a.hot_plane;
-          } else {
-            s_kb[o] = a.k_store + src * D;
-            s_vb[o] = a.v_store + src * D;
-            s_pl[o] = a.plane;
-          }
+  // Store token of each in-block slot: walk forward from the block's first
+  // fact (facts cover consecutive segment ranges).
+  if (tid < B) {
+    const int o = tid;
+    long long src = -1;
+    if (o >= o_lo && o < o_hi) {
+      const int i = blk_pos + o - start;  // segment index
+      int j = j_first;
+      while (j + 1 < j1 && seg[j + 1] <= i) ++j;
+      const int f = a.fact_ids[j];
+      const int t = i - seg[j];
+      src = a.fact_off[f] + t;
+      if (HOST_TIER) {
+        const long long ho = a.hot_off[f];
+        if (ho >= 0) {
+          s_kb[o] = a.k_hot + (ho + t) * D;
+          s_vb[o] = a.v_hot + (ho + t) * D;
+          s_pl[o] = a.hot_plane;
+        } else {
+          s_kb[o] = a.k_store + src * D;
+          s_vb[o] = a.v_store + src * D;
+          s_pl[o] = a.plane;
         }
-        if (lg == 0 && a.slot_out) a.slot_out[tok0 + i] = phys_ok ? (long long)phys * B + o : -1;
       }
-      s_src[o] = src;
+      if (write_slots && a.slot_out) a.slot_out[tok0 + i] = phys_ok ? (long long)phys * B + o : -1;
     }
-    if (!phys_ok) {
-      if (tid == 0 && lg == 0) record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + d.b);
-      continue;  // uniform; the loop top holds the barrier
-    }
-    // cos/sin of every (slot, frequency): fp64 angle and sincos, kept fp32.
-    for (int e = tid; e < B * (D / 2); e += NT) {
-      const int o = e / (D / 2), i = e % (D / 2);
-      double sn, cn;
-      sincos(double(blk_pos + o) * a.inv_freq[i], &sn, &cn);
-      reinterpret_cast<float2*>(s_cs4)[cs_index<D, STYLE>(o, i)] = make_float2(float(cn), float(sn));
-    }
-    __syncthreads();
+    s_src[o] = src;
+  }
+  if (!phys_ok) {
+    if (tid == 0 && write_slots) record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
+    return;  // uniform; the caller's barrier follows
+  }
+  // cos/sin of every (slot, frequency): fp64 angle and sincos, kept fp32.
+  for (int e = tid; e < B * (D / 2); e += NT) {
+    const int o = e / (D / 2), i = e % (D / 2);
+    double sn, cn;
+    sincos(double(blk_pos + o) * a.inv_freq[i], &sn, &cn);
+    reinterpret_cast<float2*>(s_cs4)[cs_index<D, STYLE>(o, i)] = make_float2(float(cn), float(sn));
+  }
+  __syncthreads();
 
     const int total = (l1 - l0) * vecs_layer;
     const uint16_t* kst = a.k_store;
@@ -657,6 +641,189 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
       store_stage(kv, vv, base);
     }
 #endif
+}
+
+// Persistent gather-rotate-scatter kernel.  Work unit u covers global block
+// gb = u % total_blocks and layers [lg * lpu, min(L, (lg + 1) * lpu)),
+// lg = u / total_blocks, so CTAs running side by side read neighbouring
+// tokens of the same layers.  Units are taken from an atomic counter; the
+// next unit is fetched while the current one is copied.  POW2: H and B are
+// powers of two (all index splits are shifts).  HOST_TIER: the store lives
+// in pinned host memory read over the host link, except the facts that also
+// sit in the HBM hot arenas; the source of every slot is chosen per fact.
+template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER>
+__global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
+  extern __shared__ float4 s_cs4[];  // [B * D/4] cos/sin of the block
+  __shared__ UnitShared<HOST_TIER> sm;
+  __shared__ int s_unit;
+
+  const int tid = threadIdx.x;
+  // When launched as a programmatic dependent of the plan kernel, wait here
+  // for its results; without such a launch this returns at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int total_units = a.hdr->total_units;
+  const int total_blocks = a.hdr->total_blocks;
+  const int lpu = a.hdr->layers_per_unit;
+
+  int next = 0;
+  if (tid == 0) next = int(atomicAdd(&a.hdr->next_unit, 1u));
+  for (;;) {
+    __syncthreads();  // the previous unit's tables are no longer read
+    if (tid == 0) {
+      s_unit = next;
+      if (next < total_units) next = int(atomicAdd(&a.hdr->next_unit, 1u));
+    }
+    __syncthreads();
+    const int u = s_unit;
+    if (u >= total_units) break;
+    const int gb = u % total_blocks;
+    const int lg = u / total_blocks;
+    const BlockDesc d = a.desc[gb];
+    const int r = d.r;
+    const long long tok0 = a.req_tok0[r];
+    const int l0 = lg * lpu;
+    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER>(a, sm, s_cs4, r, d.b, d.j, a.seg, a.req_off[r + 1],
+                                                 a.start_pos[r], int(a.req_tok0[r + 1] - tok0), tok0,
+                                                 l0, min(a.L, l0 + lpu), lg == 0);
+  }
+}
+
+// Small batches (at most kSmallRequests requests and kSmallIds fact ids):
+// one kernel.  Every CTA of the persistent grid composes the batch itself in
+// shared memory -- the same definitions as plan_kernel (CSR check, lengths,
+// segment offsets, validity, token and block prefixes, work-unit size) --
+// and takes units u = blockIdx.x, blockIdx.x + gridDim.x, ...  CTA 0 alone
+// records batch- and request-level errors and the -1 slots of invalid
+// requests.  No work space, no second launch.
+constexpr int kSmallRequests = 8;
+constexpr int kSmallIds = 256;
+
+struct SmallPlan {
+  int32_t len[kSmallIds];      // fact length per CSR entry, -1 for an id outside the store
+  int32_t seg[kSmallIds];      // segment offset of each entry inside its request
+  int32_t pref[kSmallIds + 1]; // exclusive prefix of valid lengths over the whole batch
+  int32_t roff[kSmallRequests + 1];
+  int32_t start[kSmallRequests];
+  int32_t err[kSmallRequests];
+  int32_t nblk[kSmallRequests];
+  int32_t blk0[kSmallRequests + 1];
+  int32_t bad, total_units, total_blocks, lpu;
+};
+
+template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER>
+__global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, int32_t R, int32_t num_ids,
+                                                                int64_t slot_cap, int32_t grid_ctas,
+                                                                int32_t max_batch_blocks) {
+  static_assert(NT == kSmallIds, "one thread per fact id");
+  extern __shared__ float4 s_cs4[];
+  __shared__ UnitShared<HOST_TIER> sm;
+  __shared__ SmallPlan p;
+  __shared__ int32_t s_wsum[NT / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool reporter = blockIdx.x == 0;
+
+  // CSR: starts at 0, ends at num_ids, never decreases.
+  if (tid <= R) p.roff[tid] = a.req_off[tid];
+  if (tid < R) p.start[tid] = a.start_pos[tid];
+  if (tid == 0) p.bad = 0;
+  __syncthreads();
+  if ((tid < R && p.roff[tid + 1] < p.roff[tid]) || (tid == 0 && (p.roff[0] != 0 || p.roff[R] != num_ids)))
+    p.bad = 1;
+  __syncthreads();
+  if (p.bad) {
+    if (reporter && tid == 0) record_error(a.st, kErrInvalidArg, -1);
+    return;
+  }
+  // Lengths, and their exclusive prefix over the batch (invalid ids count 0).
+  int32_t len = 0;
+  if (tid < num_ids) {
+    const int32_t f = a.fact_ids[tid];
+    const bool ok = f >= 0 && f < a.fact_len_count;
+    p.len[tid] = ok ? a.fact_len[f] : -1;
+    len = ok ? p.len[tid] : 0;
+  }
+  int32_t x = len;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, d);
+    if (lane >= d) x += y;
+  }
+  if (lane == 31) s_wsum[warp] = x;
+  __syncthreads();
+  int32_t wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += s_wsum[w];
+  p.pref[tid] = wbase + x - len;
+  if (tid == NT - 1) p.pref[NT] = wbase + x;  // so p.pref[num_ids] is the batch total
+  __syncthreads();
+  // Per request: validity and touched blocks.
+  if (tid < R) {
+    const int r = tid, j0 = p.roff[r], j1 = p.roff[r + 1];
+    const long long S = p.pref[j1] - p.pref[j0];
+    int32_t err = kOk;
+    for (int j = j0; j < j1; ++j)
+      if (p.len[j] < 0) { err = kErrBadFactId; break; }
+    if (err == kOk && p.start[r] < 0) err = kErrInvalidArg;
+    if (err == kOk && (long long)p.start[r] + S > (long long)a.max_blocks * a.B) err = kErrPosition;
+    p.err[r] = err;
+    p.nblk[r] = (err == kOk && S > 0) ? int32_t((p.start[r] + S - 1) / a.B - p.start[r] / a.B + 1) : 0;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int32_t acc = 0;
+    for (int r = 0; r < R; ++r) { p.blk0[r] = acc; acc += p.nblk[r]; }
+    p.blk0[R] = acc;
+    const long long total_tokens = p.pref[num_ids];
+    // the same limits as the two-kernel path, so results never depend on
+    // which path a batch takes
+    const bool over = (a.slot_out != nullptr && total_tokens > slot_cap) || acc > max_batch_blocks;
+    int32_t lpu, upb;
+    unit_size(acc, a.L, grid_ctas, lpu, upb);
+    p.lpu = lpu;
+    p.total_blocks = acc;
+    p.total_units = over ? 0 : acc * upb;
+    if (reporter) {
+      for (int r = 0; r < R; ++r)
+        if (p.err[r] != kOk) record_error(a.st, p.err[r], r);
+      if (over) record_error(a.st, kErrCapacity, total_tokens);
+    }
+  }
+  // Segment offsets inside each request.
+  if (tid < num_ids) {
+    int r = 0;
+    while (r + 1 < R && p.roff[r + 1] <= tid) ++r;
+    p.seg[tid] = p.pref[tid] - p.pref[p.roff[r]];
+  }
+  __syncthreads();
+  // -1 slots for the tokens of invalid requests (nothing at all on capacity).
+  const bool over_cap =
+      (a.slot_out != nullptr && p.pref[num_ids] > slot_cap) || p.blk0[R] > max_batch_blocks;
+  if (reporter && a.slot_out && !over_cap) {
+    for (int r = 0; r < R; ++r) {
+      if (p.err[r] == kOk) continue;
+      const int32_t S = p.pref[p.roff[r + 1]] - p.pref[p.roff[r]];
+      for (int32_t i = tid; i < S; i += NT) a.slot_out[p.pref[p.roff[r]] + i] = -1;
+    }
+  }
+
+  const int total_units = p.total_units, total_blocks = p.total_blocks, lpu = p.lpu;
+  for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+    __syncthreads();  // the previous unit's tables are no longer read
+    const int gb = u % total_blocks, lg = u / total_blocks;
+    int r = 0;
+    while (r + 1 < R && p.blk0[r + 1] <= gb) ++r;
+    const int start = p.start[r];
+    const int b = start / a.B + (gb - p.blk0[r]);
+    const int j0 = p.roff[r], j1 = p.roff[r + 1];
+    const int i_first = max(0, b * a.B - start);
+    int lo = j0, hi = j1 - 1;  // last fact with seg <= i_first
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.seg[mid] <= i_first) lo = mid; else hi = mid - 1;
+    }
+    const int l0 = lg * lpu;
+    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER>(a, sm, s_cs4, r, b, lo, p.seg, j1, start,
+                                                 p.pref[j1] - p.pref[j0], p.pref[j0], l0,
+                                                 min(a.L, l0 + lpu), lg == 0);
   }
 }
 

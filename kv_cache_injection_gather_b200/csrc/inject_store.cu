@@ -109,6 +109,7 @@ struct is_store {
   size_t events_used = 0;
   // kernel configuration
   int inject_grid = 0;
+  int32_t small_limit = isk::kSmallRequests;  // batches up to this many requests: one kernel
 };
 
 namespace {
@@ -177,6 +178,23 @@ void* inject_fn() {
       &isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER>);
 }
 
+template <int D, int STYLE, bool POW2, bool HOST_TIER>
+void* small_fn() {
+  return reinterpret_cast<void*>(
+      &isk::small_inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER>);
+}
+
+template <bool POW2, bool HOST_TIER = false>
+void* pick_small_t(int D, int style) {
+  switch (D) {
+    case 32: return style ? small_fn<32, 1, POW2, HOST_TIER>() : small_fn<32, 0, POW2, HOST_TIER>();
+    case 64: return style ? small_fn<64, 1, POW2, HOST_TIER>() : small_fn<64, 0, POW2, HOST_TIER>();
+    case 128: return style ? small_fn<128, 1, POW2, HOST_TIER>() : small_fn<128, 0, POW2, HOST_TIER>();
+    case 256: return style ? small_fn<256, 1, POW2, HOST_TIER>() : small_fn<256, 0, POW2, HOST_TIER>();
+    default: return nullptr;
+  }
+}
+
 template <bool POW2, bool HOST_TIER = false>
 void* pick_inject_t(int D, int style) {
   switch (D) {
@@ -197,6 +215,13 @@ void* pick_inject(int D, int style, int H, int B, bool host_tier = false) {
   const bool p2 = is_pow2(H) && is_pow2(B);
   if (host_tier) return p2 ? pick_inject_t<true, true>(D, style) : pick_inject_t<false, true>(D, style);
   return p2 ? pick_inject_t<true>(D, style) : pick_inject_t<false>(D, style);
+}
+
+// The single-kernel variant for small batches, same selection.
+void* pick_small(int D, int style, int H, int B, bool host_tier) {
+  const bool p2 = is_pow2(H) && is_pow2(B);
+  if (host_tier) return p2 ? pick_small_t<true, true>(D, style) : pick_small_t<false, true>(D, style);
+  return p2 ? pick_small_t<true>(D, style) : pick_small_t<false>(D, style);
 }
 
 size_t cs_smem_bytes(int D, int B) { return size_t(B) * size_t(D / 2) * sizeof(float2); }
@@ -343,9 +368,12 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
   // Persistent inject grid: resident CTAs per SM x SMs, for the largest
   // cos/sin table (B = 128) so one grid size serves every block size.
   const size_t smem_max = cs_smem_bytes(c.head_dim, isk::kMaxBlockSize);
-  void* variants[4] = {pick_inject_t<true>(c.head_dim, c.rope_style), pick_inject_t<false>(c.head_dim, c.rope_style),
+  void* variants[8] = {pick_inject_t<true>(c.head_dim, c.rope_style), pick_inject_t<false>(c.head_dim, c.rope_style),
                        pick_inject_t<true, true>(c.head_dim, c.rope_style),
-                       pick_inject_t<false, true>(c.head_dim, c.rope_style)};
+                       pick_inject_t<false, true>(c.head_dim, c.rope_style),
+                       pick_small_t<true>(c.head_dim, c.rope_style), pick_small_t<false>(c.head_dim, c.rope_style),
+                       pick_small_t<true, true>(c.head_dim, c.rope_style),
+                       pick_small_t<false, true>(c.head_dim, c.rope_style)};
   for (void* f : variants) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
   void* fn = pick_inject_t<true>(c.head_dim, c.rope_style);
   int per_sm = 0;
@@ -670,7 +698,8 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.desc = s->ws_desc;
   pa.hdr = s->ws_hdr;
   pa.st = s->d_status;
-  isk::plan_kernel<kPlanThreads><<<1, kPlanThreads, 0, st>>>(pa);
+  const bool small = R <= s->small_limit && num_ids <= isk::kSmallIds;
+  if (!small) isk::plan_kernel<kPlanThreads><<<1, kPlanThreads, 0, st>>>(pa);
 
   isk::InjectArgs ia{};
   ia.k_store = s->k_view;
@@ -705,7 +734,12 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.desc = s->ws_desc;
   ia.hdr = s->ws_hdr;
   ia.st = s->d_status;
-  void* fn = pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena);
+  ia.fact_len_count = s->num_facts;
+  void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena)
+                   : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena);
+  int32_t small_R = R, small_ids = num_ids, small_grid = s->inject_grid, small_blocks = s->max_blocks;
+  int64_t small_cap = slot_cap;
+  void* small_args[] = {&ia, &small_R, &small_ids, &small_cap, &small_grid, &small_blocks};
   void* args[] = {&ia};
   TimedLaunch* ev = nullptr;
   if (s->timing && s->events_used < size_t(kMaxTimedLaunches)) {
@@ -717,19 +751,21 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
     if (s->events_used < s->events.size()) ev = &s->events[s->events_used++];
   }
   cudaError_t e;
-  if (ev) {
+  const size_t smem = cs_smem_bytes(cf.head_dim, c.block_size);
+  if (ev) cudaEventRecord(ev->start, st);
+  if (small) {
+    // One kernel composes and injects the whole small batch.
+    e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), small_args, smem, st);
+  } else if (ev) {
     // Timed: events bracket the inject kernel alone (no early launch).
-    cudaEventRecord(ev->start, st);
-    e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), args,
-                         cs_smem_bytes(cf.head_dim, c.block_size), st);
-    cudaEventRecord(ev->stop, st);
+    e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), args, smem, st);
   } else {
     // Programmatic dependent launch: the inject grid becomes resident while
     // the plan kernel runs and starts work when the plan's results are ready.
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(unsigned(s->inject_grid));
     lc.blockDim = dim3(kInjectThreads);
-    lc.dynamicSmemBytes = cs_smem_bytes(cf.head_dim, c.block_size);
+    lc.dynamicSmemBytes = smem;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -738,6 +774,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
     lc.numAttrs = 1;
     e = cudaLaunchKernelExC(&lc, fn, args);
   }
+  if (ev) cudaEventRecord(ev->stop, st);
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
   return IS_OK;
 }
@@ -815,6 +852,12 @@ int is_last_error_timeout(is_store_t* s, void* stream, int32_t timeout_ms, int64
     std::this_thread::sleep_for(std::chrono::microseconds(200));
   }
   return is_last_error(s, stream, detail);
+}
+
+int is_store_set_small_batch_limit(is_store_t* s, int32_t max_requests) {
+  if (!s || max_requests < 0 || max_requests > isk::kSmallRequests) return IS_ERR_INVALID_ARG;
+  s->small_limit = max_requests;
+  return IS_OK;
 }
 
 int is_store_set_timing(is_store_t* s, int enable) {

@@ -220,6 +220,10 @@ class FactStore:
             stream = torch.cuda.current_stream(self.device).cuda_stream
         return B.is_last_error_timeout(self.handle, stream, timeout_ms)
 
+    def set_small_batch_limit(self, max_requests: int) -> None:
+        """Batches up to max_requests (<= 8) requests run as one kernel; 0: never."""
+        B.is_store_set_small_batch_limit(self.handle, max_requests)
+
     def set_timing(self, enable: bool) -> None:
         B.is_store_set_timing(self.handle, enable)
 

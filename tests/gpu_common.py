@@ -20,7 +20,8 @@ def rope_of(model: synth.Model, style: int = 0) -> RopeConfig:
 
 
 def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = None,
-               device: int = 0, extra_tokens: int = 0, **limits) -> FactStore:
+               device: int = 0, extra_tokens: int = 0, small_limit: int | None = None,
+               **limits) -> FactStore:
     """Put every fact of the workload, in id order (ids equal indices).
 
     Small stores are generated on the host (numpy) and copied; large ones are
@@ -29,6 +30,8 @@ def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = 
     total = int(wl.fact_lens.sum()) + extra_tokens
     store = FactStore(m.num_layers, m.num_kv_heads, m.head_dim, rope_of(m, style), total,
                       len(wl.fact_lens), device=device, **limits)
+    if small_limit is not None:  # 0: always the plan + inject kernels
+        store.set_small_batch_limit(small_limit)
     if on_device_gen is None:
         on_device_gen = total * m.bytes_per_token > (64 << 20)
     dev = torch.device("cuda", device)

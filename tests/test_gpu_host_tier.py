@@ -23,13 +23,15 @@ def _need_gpu():
         pytest.skip("no CUDA device")
 
 
+@pytest.mark.parametrize("path", ["fused", "two-kernel"])
 @pytest.mark.parametrize("hot_part", ["none", "some", "all"])
-def test_host_tier_parity(hot_part):
+def test_host_tier_parity(hot_part, path):
     _need_gpu()
     model = synth.Model("qwen-like", 2, 4, 128, 1e6)
     wl = _ragged(model, seed=21, R=6, max_k=8, lens=(1, 40), num_facts=30)
     total = int(wl.fact_lens.sum())
-    store = make_store(wl, host_tier=True, hot_capacity_tokens=total)
+    store = make_store(wl, host_tier=True, hot_capacity_tokens=total,
+                       small_limit=None if path == "fused" else 0)
     if hot_part == "some":
         store.set_hot(np.arange(0, 30, 3))
     elif hot_part == "all":

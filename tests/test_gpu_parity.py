@@ -49,11 +49,17 @@ def oracle_run(wl: synth.Workload, style=0, head_major=False, slot_capacity=None
     return rc, slots, kc, vc, kref
 
 
-def gpu_run(wl: synth.Workload, style=0, head_major=False, slot_capacity=None, store=None):
+# Small batches run as one kernel by default; "two-kernel" forces the plan +
+# inject path on the same inputs.
+PATHS = {"fused": None, "two-kernel": 0}
+
+
+def gpu_run(wl: synth.Workload, style=0, head_major=False, slot_capacity=None, store=None,
+            path="fused"):
     _need_gpu()
     own = store is None
     if own:
-        store = make_store(wl, style)
+        store = make_store(wl, style, small_limit=PATHS[path])
     k, v, desc = make_cache(wl, head_major=head_major)
     ro, ids, sp, bt = batch_tensors(wl.batch)
     n_tok = int(wl.fact_lens[wl.batch.fact_ids[(wl.batch.fact_ids >= 0) &
@@ -98,11 +104,12 @@ def test_device_generator_matches_host():
     assert np.array_equal(t.cpu().numpy().view(np.uint16), host)
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("style", [0, 1])
 @pytest.mark.parametrize("start", [32, 37, 0])
-def test_tiny_parity(start, style):
+def test_tiny_parity(start, style, path):
     wl = synth.tiny(0, start_pos=start)
-    assert_parity(oracle_run(wl, style), gpu_run(wl, style))
+    assert_parity(oracle_run(wl, style), gpu_run(wl, style, path=path))
 
 
 def _ragged(model, seed, B=16, R=7, max_k=9, lens=(1, 40), num_facts=40, starts=None,
@@ -133,33 +140,48 @@ SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
-def test_ragged_batches_parity(shape):
+def test_ragged_batches_parity(shape, path):
     name, L, H, D, theta, ll3, B_, style, hm = shape
     model = synth.Model(name, L, H, D, theta, llama3=ll3)
     wl = _ragged(model, seed=sum(name.encode()), B=B_)
-    assert_parity(oracle_run(wl, style, hm), gpu_run(wl, style, hm))
+    assert_parity(oracle_run(wl, style, hm), gpu_run(wl, style, hm, path=path))
 
 
-def test_long_segments_many_blocks():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_many_requests_many_ids(path):
+    """Past the single-kernel limits (9 requests; 300 ids): the two-kernel
+    path in both settings."""
+    model = synth.Model("m", 2, 4, 64, 1e4)
+    wl = _ragged(model, seed=77, R=9, max_k=9, lens=(1, 12), num_facts=50)
+    assert_parity(oracle_run(wl), gpu_run(wl, path=path))
+    wl2 = _ragged(model, seed=78, R=6, max_k=150, lens=(1, 6), num_facts=400, spare_blocks=1)
+    assert len(wl2.batch.fact_ids) > 256
+    assert_parity(oracle_run(wl2), gpu_run(wl2, path=path))
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_long_segments_many_blocks(path):
     """Facts longer than several blocks; positions up to ~5k (fp32 angle range
     the kernel must handle with fp64 angles)."""
     model = synth.Model("long", 2, 2, 128, 5e5, llama3=True)
     wl = _ragged(model, seed=3, R=3, max_k=6, lens=(100, 400), num_facts=12,
                  starts=[0, 3000, 4097])
-    assert_parity(oracle_run(wl), gpu_run(wl))
+    assert_parity(oracle_run(wl), gpu_run(wl, path=path))
 
 
-def test_empty_batch_and_empty_requests():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_empty_batch_and_empty_requests(path):
     model = synth.Model("e", 1, 2, 64, 1e4)
     rng = np.random.default_rng(0)
     fl = rng.integers(1, 20, 10).astype(np.int32)
     b0 = synth.make_batch(rng, [], np.zeros(0), 16, 4, 1)
     wl0 = synth.Workload("empty", model, fl, b0)
-    assert_parity(oracle_run(wl0), gpu_run(wl0))
+    assert_parity(oracle_run(wl0), gpu_run(wl0, path=path))
     b1 = synth.make_batch(rng, [np.zeros(0, int)] * 3, [5, 0, 16], 16, 6, 2)
     wl1 = synth.Workload("empty-requests", model, fl, b1)
-    assert_parity(oracle_run(wl1), gpu_run(wl1))
+    assert_parity(oracle_run(wl1), gpu_run(wl1, path=path))
 
 
 def _error_wl(kind):
@@ -188,19 +210,21 @@ def _error_wl(kind):
     return synth.Workload("err-" + kind, wl.model, wl.fact_lens, batch, wl.seed)
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("kind", ["bad_fact", "position", "bad_block", "negative_block",
                                   "negative_start", "csr", "csr_range"])
-def test_device_errors_match_oracle(kind):
+def test_device_errors_match_oracle(kind, path):
     wl = _error_wl(kind)
     o = oracle_run(wl)
     assert o[0] != oracle.OK
-    assert_parity(o, gpu_run(wl))
+    assert_parity(o, gpu_run(wl, path=path))
 
 
-def test_slot_capacity_error_writes_nothing():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_slot_capacity_error_writes_nothing(path):
     wl = synth.tiny(0)
     o = oracle_run(wl, slot_capacity=3)
-    g = gpu_run(wl, slot_capacity=3)
+    g = gpu_run(wl, slot_capacity=3, path=path)
     assert o[0] == g[0] == oracle.ERR_CAPACITY
     assert np.array_equal(g[2], o[2]) and np.array_equal(g[3], o[3])
 
