@@ -62,7 +62,7 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic(bytes_per_token_algo: float):
+def recorded_traffic():
     """DRAM bytes per injected token of the inject kernel from the committed
     ncu summary, if it was taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "inject_kernel_traffic.json")
@@ -598,7 +598,7 @@ def run_ours(args, rank, world, local_rank):
     algo_bytes = n_tok * 2 * m.bytes_per_token   # read K+V + write K+V
     peak, peak_kind = hbm_peak()
     achieved = algo_bytes / (kern_avg_ms / 1e3) / 1e9
-    traffic_pt, rec = recorded_traffic(2 * m.bytes_per_token)
+    traffic_pt, rec = recorded_traffic()
     if args.workload != "llama-batch" or args.head_major:
         traffic_pt = None  # the committed counters are for the benchmark workload
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -1,24 +1,30 @@
 // Device code of the retrieve-and-inject path for sm_100a.
 //
-// Two kernels per batch (technical summary of "InferScale: GPU-Native KV
+// What a batch computes (technical summary of "InferScale: GPU-Native KV
 // Injection for Personalized LLM Serving", section "Methodology -- 2. Online
-// phase: Chunked RoPE and KV injection"):
+// phase: Chunked RoPE and KV injection"): each request's retrieved facts are
+// laid out as one contiguous segment at new serving positions ("Dynamic
+// rotation"), every stored pre-RoPE key is rotated to its token's position
+// (RoPE; fp64 angles, fp32 rotation, bf16 round-to-nearest-even), and K and
+// the raw V are scatter-copied into the paged KV cache ("Injection").
 //
-//   plan_kernel    one CTA.  Composes every request's retrieved facts into one
-//                  contiguous segment ("Dynamic rotation": the facts are laid
-//                  out as one segment at new serving positions), validates the
-//                  batch, and writes one descriptor per touched cache block.
-//   inject_kernel  persistent grid.  Per work unit (one cache block of one
-//                  request x a range of layers) it gathers the stored pre-RoPE
-//                  K and raw V rows of the block's tokens, rotates K to the
-//                  tokens' positions (RoPE, fp64 angles, fp32 rotation, bf16
-//                  round-to-nearest-even), and writes K and V into the paged
-//                  cache ("Injection": scatter-copy into the paged KV cache).
+// Kernels:
+//   plan_kernel          one CTA: composes the segments, validates the batch,
+//                        writes one descriptor per touched cache block.
+//   inject_kernel        persistent grid, launched as a programmatic
+//                        dependent of the plan: per work unit (one cache
+//                        block of one request x a range of layers) gathers
+//                        the block's K/V rows, rotates K, writes the cache.
+//   small_inject_kernel  small batches: every CTA composes the batch itself
+//                        in shared memory, then runs the same per-unit work.
+//   promote_kernel,      host-tier store, LRU hot set: copy promoted facts
+//   hot_table_kernel     into HBM slots, patch the hot table.
+//   inv_freq_kernel      RoPE frequencies (fp64, Llama-3.1 rule optional).
 //
 // The path is a copy with a small rotation: bandwidth-bound on HBM.  Every
-// global access is a 16-byte vector; a block's tokens of one layer are one
-// contiguous run of the cache (token-major layout), written by consecutive
-// threads.
+// global access is a 16-byte vector; stored rows are read in runs along
+// their token planes and each block's layer of the cache is one contiguous
+// run written by the whole CTA.
 #pragma once
 
 #include <cuda_runtime.h>

@@ -1,5 +1,7 @@
-// Host side of libinjectstore.so: the fact store, the C-ABI declared in
-// include/inject_store.h, and the launches of the plan and inject kernels.
+// Host side of libinjectstore.so: the fact store (device or pinned-host tier,
+// static or LRU hot set), the C-ABI declared in include/inject_store.h, the
+// launches of the kernels in inject_kernels.cuh, and the allocation-free
+// entry point at the end of the file.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -99,7 +101,6 @@ struct is_store {
   int32_t* stage = nullptr;
   size_t stage_elems = 0;
   int32_t* host_stage = nullptr;   // pinned mirror of `stage`
-  size_t host_stage_elems = 0;
   isk::DevStatus* host_status = nullptr;  // pinned
   int64_t* stage_slots = nullptr;
   int64_t stage_slot_elems = 0;

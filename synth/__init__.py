@@ -47,7 +47,6 @@ _M2 = np.uint64(0x94D049BB133111EB)
 # Stream tags: the high bits of a stream id name the tensor family.
 TAG_FACT = 1 << 40        # stream = TAG_FACT | (fact_id << 1) | is_value
 TAG_CACHE = 2 << 40       # stream = TAG_CACHE | is_value   (cache pre-fill)
-TAG_MODEL = 3 << 40       # tiny-model weights and activations in tests
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
