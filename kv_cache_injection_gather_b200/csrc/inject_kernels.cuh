@@ -466,6 +466,7 @@ struct Divisor {
 };
 
 __device__ __forceinline__ int ilog2(int x) { return 31 - __clz(x); }
+__host__ __device__ constexpr int clog2(int x) { return x <= 1 ? 0 : 1 + clog2(x / 2); }
 
 // Vector order inside one layer of a block (rem = the vector's index in the
 // layer; a head row is D/8 consecutive vectors, so rotate-half partners stay
@@ -508,7 +509,7 @@ struct UnitShared {
 // index.  The slot mapping is written when write_slots.  Vector order inside
 // a layer: split_vec.  Every thread of the CTA calls this with the same
 // arguments; the caller puts a barrier between units.
-template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER>
+template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER, int HC, int BC>
 __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TIER>& sm,
                                          float4* s_cs4, int r, int b, int j_first,
                                          const int32_t* seg, int j1, int start, int len_r,
@@ -516,13 +517,15 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
   constexpr int VPR = D / 8;  // 16-byte vectors per head row
   constexpr int LOG_VPR = (VPR == 4) ? 2 : (VPR == 8) ? 3 : (VPR == 16) ? 4 : 5;
   const int tid = threadIdx.x;
-  const int B = a.B;
-  const int H = a.H;
+  // HC / BC > 0: the KV head count / block size are compile-time constants
+  // (the common model shapes), which folds the per-vector index arithmetic.
+  const int B = BC > 0 ? BC : a.B;
+  const int H = HC > 0 ? HC : a.H;
   const int row_vecs = H * VPR;         // vectors per token (all heads)
   const int vecs_layer = B * row_vecs;  // vectors per block and layer
-  const Divisor<POW2> by_layer{vecs_layer, POW2 ? ilog2(vecs_layer) : 0};
-  const Divisor<POW2> by_row{row_vecs, POW2 ? ilog2(row_vecs) : 0};
-  const Divisor<POW2> by_hrow{B * VPR, POW2 ? ilog2(B * VPR) : 0};
+  const Divisor<POW2> by_layer{vecs_layer, POW2 ? (BC > 0 && HC > 0 ? clog2(BC * HC * VPR) : ilog2(vecs_layer)) : 0};
+  const Divisor<POW2> by_row{row_vecs, POW2 ? (HC > 0 ? clog2(HC * VPR) : ilog2(row_vecs)) : 0};
+  const Divisor<POW2> by_hrow{B * VPR, POW2 ? (BC > 0 ? clog2(BC * VPR) : ilog2(B * VPR)) : 0};
   const int order = a.vec_order;
   long long* s_src = sm.src;
   const uint16_t** s_kb = sm.kb;
@@ -657,7 +660,7 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
 // powers of two (all index splits are shifts).  HOST_TIER: the store lives
 // in pinned host memory read over the host link, except the facts that also
 // sit in the HBM hot arenas; the source of every slot is chosen per fact.
-template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER>
+template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
 __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   extern __shared__ float4 s_cs4[];  // [B * D/4] cos/sin of the block
   __shared__ UnitShared<HOST_TIER> sm;
@@ -688,7 +691,7 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
     const int r = d.r;
     const long long tok0 = a.req_tok0[r];
     const int l0 = lg * lpu;
-    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER>(a, sm, s_cs4, r, d.b, d.j, a.seg, a.req_off[r + 1],
+    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC>(a, sm, s_cs4, r, d.b, d.j, a.seg, a.req_off[r + 1],
                                                  a.start_pos[r], int(a.req_tok0[r + 1] - tok0), tok0,
                                                  l0, min(a.L, l0 + lpu), lg == 0);
   }
@@ -716,7 +719,7 @@ struct SmallPlan {
   int32_t bad, total_units, total_blocks, lpu;
 };
 
-template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER>
+template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
 __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, int32_t R, int32_t num_ids,
                                                                 int64_t slot_cap, int32_t grid_ctas,
                                                                 int32_t max_batch_blocks) {
@@ -827,7 +830,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
       if (p.seg[mid] <= i_first) lo = mid; else hi = mid - 1;
     }
     const int l0 = lg * lpu;
-    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER>(a, sm, s_cs4, r, b, lo, p.seg, j1, start,
+    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC>(a, sm, s_cs4, r, b, lo, p.seg, j1, start,
                                                  p.pref[j1] - p.pref[j0], p.pref[j0], l0,
                                                  min(a.L, l0 + lpu), lg == 0);
   }

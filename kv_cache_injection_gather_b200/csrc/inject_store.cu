@@ -173,16 +173,18 @@ void free_store(is_store* s) {
 
 bool head_dim_supported(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
 
-template <int D, int STYLE, bool POW2, bool HOST_TIER>
+template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
 void* inject_fn() {
   return reinterpret_cast<void*>(
-      &isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER>);
+      &isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER, HC, BC>);
 }
 
-template <int D, int STYLE, bool POW2, bool HOST_TIER>
+
+
+template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
 void* small_fn() {
   return reinterpret_cast<void*>(
-      &isk::small_inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER>);
+      &isk::small_inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER, HC, BC>);
 }
 
 template <bool POW2, bool HOST_TIER = false>
@@ -194,6 +196,25 @@ void* pick_small_t(int D, int style) {
     case 256: return style ? small_fn<256, 1, POW2, HOST_TIER>() : small_fn<256, 0, POW2, HOST_TIER>();
     default: return nullptr;
   }
+}
+
+// Compile-time shapes for the common models (D = 128, block size 16, 4 or 8
+// KV heads: Llama-3.1-8B, Mistral-7B, Qwen2.5-7B): the per-vector index
+// arithmetic folds to constants.  Returns nullptr for other shapes.
+template <bool SMALL, bool HOST_TIER>
+void* pick_fixed(int D, int style, int H, int B) {
+#ifndef IS_NO_FIXED_SHAPES
+  if (D != 128 || B != 16) return nullptr;
+  if (H == 8)
+    return SMALL ? (style ? small_fn<128, 1, true, HOST_TIER, 8, 16>() : small_fn<128, 0, true, HOST_TIER, 8, 16>())
+                 : (style ? inject_fn<128, 1, true, HOST_TIER, 8, 16>() : inject_fn<128, 0, true, HOST_TIER, 8, 16>());
+  if (H == 4)
+    return SMALL ? (style ? small_fn<128, 1, true, HOST_TIER, 4, 16>() : small_fn<128, 0, true, HOST_TIER, 4, 16>())
+                 : (style ? inject_fn<128, 1, true, HOST_TIER, 4, 16>() : inject_fn<128, 0, true, HOST_TIER, 4, 16>());
+#else
+  (void)D; (void)style; (void)H; (void)B;
+#endif
+  return nullptr;
 }
 
 template <bool POW2, bool HOST_TIER = false>
@@ -213,6 +234,8 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 // when both are powers of two; the host-tier variant for stores in pinned
 // host memory.
 void* pick_inject(int D, int style, int H, int B, bool host_tier = false) {
+  if (void* f = host_tier ? pick_fixed<false, true>(D, style, H, B) : pick_fixed<false, false>(D, style, H, B))
+    return f;
   const bool p2 = is_pow2(H) && is_pow2(B);
   if (host_tier) return p2 ? pick_inject_t<true, true>(D, style) : pick_inject_t<false, true>(D, style);
   return p2 ? pick_inject_t<true>(D, style) : pick_inject_t<false>(D, style);
@@ -220,6 +243,8 @@ void* pick_inject(int D, int style, int H, int B, bool host_tier = false) {
 
 // The single-kernel variant for small batches, same selection.
 void* pick_small(int D, int style, int H, int B, bool host_tier) {
+  if (void* f = host_tier ? pick_fixed<true, true>(D, style, H, B) : pick_fixed<true, false>(D, style, H, B))
+    return f;
   const bool p2 = is_pow2(H) && is_pow2(B);
   if (host_tier) return p2 ? pick_small_t<true, true>(D, style) : pick_small_t<false, true>(D, style);
   return p2 ? pick_small_t<true>(D, style) : pick_small_t<false>(D, style);
@@ -376,6 +401,12 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
                        pick_small_t<true, true>(c.head_dim, c.rope_style),
                        pick_small_t<false, true>(c.head_dim, c.rope_style)};
   for (void* f : variants) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
+  for (int h : {4, 8})
+    for (void* f : {pick_fixed<false, false>(c.head_dim, c.rope_style, h, 16),
+                    pick_fixed<false, true>(c.head_dim, c.rope_style, h, 16),
+                    pick_fixed<true, false>(c.head_dim, c.rope_style, h, 16),
+                    pick_fixed<true, true>(c.head_dim, c.rope_style, h, 16)})
+      if (f) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
   void* fn = pick_inject_t<true>(c.head_dim, c.rope_style);
   int per_sm = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kInjectThreads, cs_smem_bytes(c.head_dim, 16));
