@@ -516,10 +516,26 @@ def run_ours(args, rank, world, local_rank):
     if args.workload == "offload":
         return run_offload(args, rank, world, local_rank)
     extra_cfg = {}
-    wl = WORKLOADS[args.workload][1](rank)
-    store = make_store(wl, on_device_gen=True, device=local_rank)
+    heads = None
+    if args.shard == "heads":
+        # KV-head shards (tensor-parallel serving): every rank holds heads
+        # [h0, h1) of every fact and of the cache and injects the same batch of
+        # 100 x world requests; per-GPU bytes stay those of the 1-GPU batch.
+        import synth
+        from kv_cache_injection_gather_b200 import shard
+        if args.workload != "llama-batch":
+            raise SystemExit("--shard heads is defined for the llama-batch workload")
+        wl = synth.llama_batch(0, R=100 * world)
+        heads = shard.head_shard(wl.model.num_kv_heads, world, rank)
+        extra_cfg["kv_heads_per_rank"] = heads[1] - heads[0]
+    else:
+        wl = WORKLOADS[args.workload][1](rank)
+    store = make_store(wl, on_device_gen=True, device=local_rank, heads=heads)
     m, b = wl.model, wl.batch
-    kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False, head_major=args.head_major)
+    if heads is not None:
+        m = synth.Model(m.name, m.num_layers, heads[1] - heads[0], m.head_dim, m.rope_theta, m.llama3)
+    kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False, head_major=args.head_major,
+                                      num_kv_heads=None if heads is None else heads[1] - heads[0])
     extra_cfg["cache_layout"] = "[L][num_blocks][H][B][D]" if args.head_major else "[L][num_blocks][B][H][D]"
     copy_ref, copy_sus = copy_probe(dev)
     ro, ids, sp, bt = batch_tensors(b, local_rank)
@@ -593,7 +609,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- max over ranks
     ms, e2e_ms, kern_avg_ms = max_over_ranks([ms, e2e_ms, kern_ms / max(kern_n, 1)], world)
     ms_step = ms / args.steps
-    tokens_all = n_tok * world
+    tokens_all = n_tok * (1 if heads is not None else world)
     value = tokens_all / (ms_step / 1e3)
     algo_bytes = n_tok * 2 * m.bytes_per_token   # read K+V + write K+V
     peak, peak_kind = hbm_peak()
@@ -619,7 +635,8 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": workload_config(wl, args.workload,
-                                  dict(extra_cfg, parallelism=f"replicas x{world}")),
+                                  dict(extra_cfg, parallelism=(f"kv-head shards x{world}" if heads
+                                                               else f"replicas x{world}"))),
         "us_per_batch": ms_step * 1e3,
         "gbs_per_gpu": algo_bytes / (ms_step / 1e3) / 1e9,
         "kernel_us": kern_avg_ms * 1e3,
@@ -645,6 +662,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-policy", choices=["static", "lru"], default="static",
                     help="offload workload: static top-20%% hot set or LRU promotion")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="multi-GPU: independent replicas (default) or KV-head shards of one "
+                         "batch of 100 x N requests (both weak scaling, no collective)")
     ap.add_argument("--head-major", action="store_true",
                     help="cache layout [L][num_blocks][H][B][D] instead of [L][num_blocks][B][H][D]")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama-batch",

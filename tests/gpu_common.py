@@ -21,12 +21,16 @@ def rope_of(model: synth.Model, style: int = 0) -> RopeConfig:
 
 def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = None,
                device: int = 0, extra_tokens: int = 0, small_limit: int | None = None,
-               **limits) -> FactStore:
+               heads: tuple[int, int] | None = None, **limits) -> FactStore:
     """Put every fact of the workload, in id order (ids equal indices).
 
     Small stores are generated on the host (numpy) and copied; large ones are
-    generated on the device by the same counter-based definition."""
-    m = wl.model
+    generated on the device by the same counter-based definition.  heads =
+    (h0, h1) keeps KV heads [h0, h1) of every fact (a head-sharded store; the
+    workload's model then names the full head count)."""
+    full = wl.model
+    m = full if heads is None else synth.Model(full.name, full.num_layers, heads[1] - heads[0],
+                                               full.head_dim, full.rope_theta, full.llama3)
     total = int(wl.fact_lens.sum()) + extra_tokens
     store = FactStore(m.num_layers, m.num_kv_heads, m.head_dim, rope_of(m, style), total,
                       len(wl.fact_lens), device=device, **limits)
@@ -37,22 +41,28 @@ def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = 
     dev = torch.device("cuda", device)
     if on_device_gen:
         maxlen = int(wl.fact_lens.max())
-        kbuf = torch.empty(m.num_layers * m.num_kv_heads * maxlen * m.head_dim,
+        kbuf = torch.empty(full.num_layers * full.num_kv_heads * maxlen * full.head_dim,
                            dtype=torch.bfloat16, device=dev)
         vbuf = torch.empty_like(kbuf)
         stream = torch.cuda.current_stream(dev).cuda_stream
         for f, n in enumerate(wl.fact_lens):
             n = int(n)
-            cnt = m.num_layers * m.num_kv_heads * n * m.head_dim
+            cnt = full.num_layers * full.num_kv_heads * n * full.head_dim
             synth.fill_device(kbuf.data_ptr(), cnt, wl.seed, synth.fact_stream(f, False), 0, stream)
             synth.fill_device(vbuf.data_ptr(), cnt, wl.seed, synth.fact_stream(f, True), 0, stream)
-            shape = (m.num_layers, m.num_kv_heads, n, m.head_dim)
-            fid = store.put_fact(kbuf[:cnt].view(shape), vbuf[:cnt].view(shape))
+            shape = (full.num_layers, full.num_kv_heads, n, full.head_dim)
+            k, v = kbuf[:cnt].view(shape), vbuf[:cnt].view(shape)
+            if heads is not None:
+                k, v = k[:, heads[0]:heads[1]], v[:, heads[0]:heads[1]]
+            fid = store.put_fact(k, v)
             assert fid == f
         torch.cuda.synchronize(dev)
     else:
         for f, n in enumerate(wl.fact_lens):
-            k, v = synth.fact_kv(wl.seed, f, m.num_layers, m.num_kv_heads, int(n), m.head_dim)
+            k, v = synth.fact_kv(wl.seed, f, full.num_layers, full.num_kv_heads, int(n), full.head_dim)
+            if heads is not None:
+                k, v = k[:, heads[0]:heads[1]], v[:, heads[0]:heads[1]]
+            k, v = np.ascontiguousarray(k), np.ascontiguousarray(v)
             kt = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16)
             vt = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16)
             assert store.put_fact(kt, vt) == f
@@ -66,10 +76,15 @@ def cache_shape(wl: synth.Workload, head_major: bool = False):
     return (m.num_layers, b.num_blocks, b.block_size, m.num_kv_heads, m.head_dim)
 
 
-def make_cache(wl: synth.Workload, device: int = 0, fill: bool = True, head_major: bool = False):
+def make_cache(wl: synth.Workload, device: int = 0, fill: bool = True, head_major: bool = False,
+               num_kv_heads: int | None = None):
     """K and V caches (bf16, device); filled with seeded values so untouched
-    slots can be checked, or left uninitialised."""
-    shape = cache_shape(wl, head_major)
+    slots can be checked, or left uninitialised.  num_kv_heads overrides the
+    model's (a head-sharded cache)."""
+    shape = list(cache_shape(wl, head_major))
+    if num_kv_heads is not None:
+        shape[2 if head_major else 3] = num_kv_heads
+    shape = tuple(shape)
     dev = torch.device("cuda", device)
     k = torch.empty(shape, dtype=torch.bfloat16, device=dev)
     v = torch.empty(shape, dtype=torch.bfloat16, device=dev)

@@ -321,3 +321,27 @@ def test_llama_single_request_full_store():
     rc, slots = oracle.inject_batch(st, f, b.req_offsets, b.fact_ids, b.start_pos, b.block_tables,
                                     kc, vc, b.block_size, k_ref=kref)
     assert_parity((rc, slots, kc, vc, kref), g)
+
+
+def test_head_sharded_stores_reproduce_the_full_cache():
+    """KV-head shards (the multi-GPU tensor-parallel partition): a store and
+    cache holding heads [h0, h1) only, fed the whole batch, produce exactly
+    the oracle's full cache restricted to those heads."""
+    _need_gpu()
+    from gpu_common import make_cache
+    model = synth.Model("llama-like", 2, 8, 128, 5e5, llama3=True)
+    wl = _ragged(model, seed=41, R=5)
+    orc, oslots, okc, ovc, kref = oracle_run(wl)
+    for h0, h1 in ((0, 4), (4, 8), (6, 8)):
+        store = make_store(wl, heads=(h0, h1))
+        k, v, desc = make_cache(wl, num_kv_heads=h1 - h0)
+        ro, ids, sp, bt = batch_tensors(wl.batch)
+        store.inject(ro, ids, sp, bt, desc)
+        assert store.last_error()[0] == orc
+        gk, gv = to_bits(k), to_bits(v)
+        assert np.array_equal(gv, ovc[:, :, :, h0:h1])
+        w = ~np.isnan(kref[:, :, :, h0:h1])
+        assert np.array_equal(gk[~w], okc[:, :, :, h0:h1][~w])
+        err = np.abs(oracle.bf16_to_f64(gk[w]) - kref[:, :, :, h0:h1][w])
+        assert np.all(err <= REL * np.abs(kref[:, :, :, h0:h1][w]) + ABS)
+        store.close()
