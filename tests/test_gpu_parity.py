@@ -16,6 +16,7 @@ import oracle
 import synth
 from gpu_common import (CACHE_FILL_SEED, batch_tensors, make_cache, make_store, to_bits)
 from kv_cache_injection_gather_b200 import binding as B
+from kv_cache_injection_gather_b200 import cache_desc
 
 pytestmark = pytest.mark.gpu
 
@@ -332,9 +333,14 @@ def test_head_sharded_stores_reproduce_the_full_cache():
     model = synth.Model("llama-like", 2, 8, 128, 5e5, llama3=True)
     wl = _ragged(model, seed=41, R=5)
     orc, oslots, okc, ovc, kref = oracle_run(wl)
+    kfull, vfull, _ = make_cache(wl)  # the oracle's fill, all heads
     for h0, h1 in ((0, 4), (4, 8), (6, 8)):
         store = make_store(wl, heads=(h0, h1))
-        k, v, desc = make_cache(wl, num_kv_heads=h1 - h0)
+        # The shard's cache starts as the full cache's head slice, so its
+        # untouched slots hold the values the oracle's cache holds there.
+        k = kfull[:, :, :, h0:h1].contiguous()
+        v = vfull[:, :, :, h0:h1].contiguous()
+        desc = cache_desc(k, v)
         ro, ids, sp, bt = batch_tensors(wl.batch)
         store.inject(ro, ids, sp, bt, desc)
         assert store.last_error()[0] == orc
