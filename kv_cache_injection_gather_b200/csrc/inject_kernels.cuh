@@ -405,11 +405,27 @@ __device__ __forceinline__ int cs_index(int o, int i) {
   }
 }
 
-// Rotate one 16-byte vector (8 bf16) of a key row.
-//   own: this lane's vector; c: its index in the row (0 .. D/8-1)
-//   cs: cos/sin table of this token (float4 words as laid out above)
+// The cos/sin words one lane needs to rotate its vector c of a key row (the
+// table of its token, float4 words as laid out above): rotate-half uses
+// t[0..3] (elements 2q, 2q+1 of the half row), interleaved t[0..1].
 template <int D, int STYLE>
-__device__ __forceinline__ uint4 rotate_vec(const uint4 own, int c, const float4* cs_tok) {
+__device__ __forceinline__ void load_cs(const float4* cs_tok, int c, float4 (&t)[4]) {
+  if (STYLE == 0) {
+    constexpr int VH = D / 16;
+    const int cp = c < VH ? c : c - VH;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) t[q] = cs_tok[q * VH + cp];
+  } else {
+    t[0] = cs_tok[c];
+    t[1] = cs_tok[D / 8 + c];
+    t[2] = t[3] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Rotate one 16-byte vector (8 bf16) of a key row with its cos/sin words.
+//   own: this lane's vector; c: its index in the row (0 .. D/8-1)
+template <int D, int STYLE>
+__device__ __forceinline__ uint4 rotate_regs(const uint4 own, int c, const float4 (&t)[4]) {
   const uint32_t w[4] = {own.x, own.y, own.z, own.w};
   float x[8];
 #pragma unroll
@@ -425,25 +441,22 @@ __device__ __forceinline__ uint4 rotate_vec(const uint4 own, int c, const float4
 #pragma unroll
     for (int q = 0; q < 4; ++q) { p[2 * q] = bf_lo(pw[q]); p[2 * q + 1] = bf_hi(pw[q]); }
     const bool first = c < VH;
-    const int cp = first ? c : c - VH;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 t = cs_tok[q * VH + cp];  // {cos, sin} of elements 2q, 2q+1
-      const float s0 = first ? -t.y : t.y, s1 = first ? -t.w : t.w;
+      const float s0 = first ? -t[q].y : t[q].y, s1 = first ? -t[q].w : t[q].w;
       // first half:  x cos - partner sin;  second half: x cos + partner sin
-      y[2 * q] = fmaf(x[2 * q], t.x, p[2 * q] * s0);
-      y[2 * q + 1] = fmaf(x[2 * q + 1], t.z, p[2 * q + 1] * s1);
+      y[2 * q] = fmaf(x[2 * q], t[q].x, p[2 * q] * s0);
+      y[2 * q + 1] = fmaf(x[2 * q + 1], t[q].z, p[2 * q + 1] * s1);
     }
   } else {
     // Pairs (2m, 2m+1) inside the vector.
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const float4 t = cs_tok[h * (D / 8) + c];  // pairs 2h and 2h+1 of this vector
       const int a0 = 4 * h, a1 = 4 * h + 2;
-      y[a0] = fmaf(x[a0], t.x, -(x[a0 + 1] * t.y));
-      y[a0 + 1] = fmaf(x[a0 + 1], t.x, x[a0] * t.y);
-      y[a1] = fmaf(x[a1], t.z, -(x[a1 + 1] * t.w));
-      y[a1 + 1] = fmaf(x[a1 + 1], t.z, x[a1] * t.w);
+      y[a0] = fmaf(x[a0], t[h].x, -(x[a0 + 1] * t[h].y));
+      y[a0 + 1] = fmaf(x[a0 + 1], t[h].x, x[a0] * t[h].y);
+      y[a1] = fmaf(x[a1], t[h].z, -(x[a1 + 1] * t[h].w));
+      y[a1 + 1] = fmaf(x[a1 + 1], t[h].z, x[a1] * t[h].w);
     }
   }
   uint4 out;
@@ -452,6 +465,13 @@ __device__ __forceinline__ uint4 rotate_vec(const uint4 own, int c, const float4
   out.z = pack_bf16(y[4], y[5]);
   out.w = pack_bf16(y[6], y[7]);
   return out;
+}
+
+template <int D, int STYLE>
+__device__ __forceinline__ uint4 rotate_vec(const uint4 own, int c, const float4* cs_tok) {
+  float4 t[4];
+  load_cs<D, STYLE>(cs_tok, c, t);
+  return rotate_regs<D, STYLE>(own, c, t);
 }
 
 constexpr int kMaxBlockSize = 128;
@@ -509,7 +529,7 @@ struct UnitShared {
 // index.  The slot mapping is written when write_slots.  Vector order inside
 // a layer: split_vec.  Every thread of the CTA calls this with the same
 // arguments; the caller puts a barrier between units.
-template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER, int HC, int BC>
+template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER, int HC, int BC, bool FAST>
 __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TIER>& sm,
                                          float4* s_cs4, int r, int b, int j_first,
                                          const int32_t* seg, int j1, int start, int len_r,
@@ -579,6 +599,70 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
   }
   __syncthreads();
 
+  // FAST: compile-time H and B with one head's block row of vectors (B * D/8)
+  // equal to the CTA, slot-fastest rows (token-major cache; the launch picks
+  // FAST only for vector order 1), device tier.  Each thread then owns one
+  // (slot o, word c) for every head and layer of the unit: its source row,
+  // cache address and cos/sin words are set up once per unit, and each
+  // vector costs one plane step.
+  if constexpr (FAST) {
+    static_assert(HC > 0 && BC > 0 && BC * VPR == NT && !HOST_TIER, "fast path shape");
+    {
+      const int o = tid / VPR, c = tid % VPR;
+      const long long src = s_src[o];
+      const bool act = src >= 0;
+      float4 cs[4];
+      load_cs<D, STYLE>(s_cs4 + o * (D / 4), c, cs);
+      const uint16_t* kp = a.k_store + (act ? src : 0) * D + c * 8 + (long long)l0 * HC * a.plane;
+      const uint16_t* vp = a.v_store + (act ? src : 0) * D + c * 8 + (long long)l0 * HC * a.plane;
+      uint16_t* kd = a.k_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
+      uint16_t* vd = a.v_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
+      const int nw = (l1 - l0) * HC;  // (layer, head) rows of this thread, in plane order
+      constexpr int HW = IS_PIPELINE ? VPT / 2 : VPT;
+      auto load_w = [&](uint4 (&kv)[HW], uint4 (&vv)[HW], int w0) {
+#pragma unroll
+        for (int q = 0; q < HW; ++q) {
+          const int w = w0 + q;
+          kv[q] = make_uint4(0, 0, 0, 0);
+          vv[q] = kv[q];
+          if (act && w < nw) {
+            kv[q] = ld_stream(kp + (long long)w * a.plane);
+            vv[q] = ld_stream(vp + (long long)w * a.plane);
+          }
+        }
+      };
+      auto store_w = [&](const uint4 (&kv)[HW], const uint4 (&vv)[HW], int w0) {
+#pragma unroll
+        for (int q = 0; q < HW; ++q) {
+          const int w = w0 + q;
+          const uint4 kr = rotate_regs<D, STYLE>(kv[q], c, cs);
+          if (act && w < nw) {
+            const int l = l0 + w / HC, h = w % HC;
+            const long long off = (long long)l * a.ls + (long long)h * a.hs;
+            st_stream(kd + off, kr);
+            st_stream(vd + off, vv[q]);
+          }
+        }
+      };
+#if IS_PIPELINE
+      uint4 ka[HW], va[HW], kb[HW], vb[HW];
+      if (nw > 0) load_w(ka, va, 0);
+      for (int w0 = 0; w0 < nw; w0 += 2 * HW) {
+        if (w0 + HW < nw) load_w(kb, vb, w0 + HW);
+        store_w(ka, va, w0);
+        if (w0 + HW >= nw) break;
+        if (w0 + 2 * HW < nw) load_w(ka, va, w0 + 2 * HW);
+        store_w(kb, vb, w0 + HW);
+      }
+#else
+      for (int w0 = 0; w0 < nw; w0 += HW) {
+        uint4 kv[HW], vv[HW];
+        load_w(kv, vv, w0);
+        store_w(kv, vv, w0);
+      }
+#endif
+    }
+  } else {
     const int total = (l1 - l0) * vecs_layer;
     const uint16_t* kst = a.k_store;
     const uint16_t* vst = a.v_store;
@@ -650,6 +734,7 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
       store_stage(kv, vv, base);
     }
 #endif
+  }
 }
 
 // Persistent gather-rotate-scatter kernel.  Work unit u covers global block
@@ -660,7 +745,8 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
 // powers of two (all index splits are shifts).  HOST_TIER: the store lives
 // in pinned host memory read over the host link, except the facts that also
 // sit in the HBM hot arenas; the source of every slot is chosen per fact.
-template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
+template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0,
+          bool FAST = false>
 __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   extern __shared__ float4 s_cs4[];  // [B * D/4] cos/sin of the block
   __shared__ UnitShared<HOST_TIER> sm;
@@ -691,7 +777,7 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
     const int r = d.r;
     const long long tok0 = a.req_tok0[r];
     const int l0 = lg * lpu;
-    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC>(a, sm, s_cs4, r, d.b, d.j, a.seg, a.req_off[r + 1],
+    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC, FAST>(a, sm, s_cs4, r, d.b, d.j, a.seg, a.req_off[r + 1],
                                                  a.start_pos[r], int(a.req_tok0[r + 1] - tok0), tok0,
                                                  l0, min(a.L, l0 + lpu), lg == 0);
   }
@@ -719,7 +805,8 @@ struct SmallPlan {
   int32_t bad, total_units, total_blocks, lpu;
 };
 
-template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
+template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0,
+          bool FAST = false>
 __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, int32_t R, int32_t num_ids,
                                                                 int64_t slot_cap, int32_t grid_ctas,
                                                                 int32_t max_batch_blocks) {
@@ -830,7 +917,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
       if (p.seg[mid] <= i_first) lo = mid; else hi = mid - 1;
     }
     const int l0 = lg * lpu;
-    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC>(a, sm, s_cs4, r, b, lo, p.seg, j1, start,
+    run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC, FAST>(a, sm, s_cs4, r, b, lo, p.seg, j1, start,
                                                  p.pref[j1] - p.pref[j0], p.pref[j0], l0,
                                                  min(a.L, l0 + lpu), lg == 0);
   }

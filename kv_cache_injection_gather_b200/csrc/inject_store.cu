@@ -173,18 +173,18 @@ void free_store(is_store* s) {
 
 bool head_dim_supported(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
 
-template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
+template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0, bool FAST = false>
 void* inject_fn() {
-  return reinterpret_cast<void*>(
-      &isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER, HC, BC>);
+  return reinterpret_cast<void*>(&isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread,
+                                                     kInjectMinBlocks, POW2, HOST_TIER, HC, BC, FAST>);
 }
 
 
 
-template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0>
+template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0, bool FAST = false>
 void* small_fn() {
-  return reinterpret_cast<void*>(
-      &isk::small_inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread, kInjectMinBlocks, POW2, HOST_TIER, HC, BC>);
+  return reinterpret_cast<void*>(&isk::small_inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread,
+                                                           kInjectMinBlocks, POW2, HOST_TIER, HC, BC, FAST>);
 }
 
 template <bool POW2, bool HOST_TIER = false>
@@ -201,18 +201,25 @@ void* pick_small_t(int D, int style) {
 // Compile-time shapes for the common models (D = 128, block size 16, 4 or 8
 // KV heads: Llama-3.1-8B, Mistral-7B, Qwen2.5-7B): the per-vector index
 // arithmetic folds to constants.  Returns nullptr for other shapes.
+template <bool SMALL, bool HOST_TIER, int HC, bool FAST>
+void* fixed_fn(int style) {
+  return SMALL ? (style ? small_fn<128, 1, true, HOST_TIER, HC, 16, FAST>()
+                        : small_fn<128, 0, true, HOST_TIER, HC, 16, FAST>())
+               : (style ? inject_fn<128, 1, true, HOST_TIER, HC, 16, FAST>()
+                        : inject_fn<128, 0, true, HOST_TIER, HC, 16, FAST>());
+}
+
+// order: the launch's vector order (1: slot-fastest, the FAST copy loop on
+// the device tier).
 template <bool SMALL, bool HOST_TIER>
-void* pick_fixed(int D, int style, int H, int B) {
+void* pick_fixed(int D, int style, int H, int B, int order) {
 #ifndef IS_NO_FIXED_SHAPES
   if (D != 128 || B != 16) return nullptr;
-  if (H == 8)
-    return SMALL ? (style ? small_fn<128, 1, true, HOST_TIER, 8, 16>() : small_fn<128, 0, true, HOST_TIER, 8, 16>())
-                 : (style ? inject_fn<128, 1, true, HOST_TIER, 8, 16>() : inject_fn<128, 0, true, HOST_TIER, 8, 16>());
-  if (H == 4)
-    return SMALL ? (style ? small_fn<128, 1, true, HOST_TIER, 4, 16>() : small_fn<128, 0, true, HOST_TIER, 4, 16>())
-                 : (style ? inject_fn<128, 1, true, HOST_TIER, 4, 16>() : inject_fn<128, 0, true, HOST_TIER, 4, 16>());
+  const bool fast = order == 1 && !HOST_TIER;
+  if (H == 8) return fast ? fixed_fn<SMALL, HOST_TIER, 8, !HOST_TIER>(style) : fixed_fn<SMALL, HOST_TIER, 8, false>(style);
+  if (H == 4) return fast ? fixed_fn<SMALL, HOST_TIER, 4, !HOST_TIER>(style) : fixed_fn<SMALL, HOST_TIER, 4, false>(style);
 #else
-  (void)D; (void)style; (void)H; (void)B;
+  (void)D; (void)style; (void)H; (void)B; (void)order;
 #endif
   return nullptr;
 }
@@ -233,8 +240,8 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 // The inject kernel for a head dim, RoPE style and (H, B): the shift variant
 // when both are powers of two; the host-tier variant for stores in pinned
 // host memory.
-void* pick_inject(int D, int style, int H, int B, bool host_tier = false) {
-  if (void* f = host_tier ? pick_fixed<false, true>(D, style, H, B) : pick_fixed<false, false>(D, style, H, B))
+void* pick_inject(int D, int style, int H, int B, bool host_tier = false, int order = 0) {
+  if (void* f = host_tier ? pick_fixed<false, true>(D, style, H, B, order) : pick_fixed<false, false>(D, style, H, B, order))
     return f;
   const bool p2 = is_pow2(H) && is_pow2(B);
   if (host_tier) return p2 ? pick_inject_t<true, true>(D, style) : pick_inject_t<false, true>(D, style);
@@ -242,8 +249,8 @@ void* pick_inject(int D, int style, int H, int B, bool host_tier = false) {
 }
 
 // The single-kernel variant for small batches, same selection.
-void* pick_small(int D, int style, int H, int B, bool host_tier) {
-  if (void* f = host_tier ? pick_fixed<true, true>(D, style, H, B) : pick_fixed<true, false>(D, style, H, B))
+void* pick_small(int D, int style, int H, int B, bool host_tier, int order) {
+  if (void* f = host_tier ? pick_fixed<true, true>(D, style, H, B, order) : pick_fixed<true, false>(D, style, H, B, order))
     return f;
   const bool p2 = is_pow2(H) && is_pow2(B);
   if (host_tier) return p2 ? pick_small_t<true, true>(D, style) : pick_small_t<false, true>(D, style);
@@ -402,11 +409,12 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
                        pick_small_t<false, true>(c.head_dim, c.rope_style)};
   for (void* f : variants) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
   for (int h : {4, 8})
-    for (void* f : {pick_fixed<false, false>(c.head_dim, c.rope_style, h, 16),
-                    pick_fixed<false, true>(c.head_dim, c.rope_style, h, 16),
-                    pick_fixed<true, false>(c.head_dim, c.rope_style, h, 16),
-                    pick_fixed<true, true>(c.head_dim, c.rope_style, h, 16)})
-      if (f) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
+    for (int order : {0, 1})
+      for (void* f : {pick_fixed<false, false>(c.head_dim, c.rope_style, h, 16, order),
+                      pick_fixed<false, true>(c.head_dim, c.rope_style, h, 16, order),
+                      pick_fixed<true, false>(c.head_dim, c.rope_style, h, 16, order),
+                      pick_fixed<true, true>(c.head_dim, c.rope_style, h, 16, order)})
+        if (f) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
   void* fn = pick_inject_t<true>(c.head_dim, c.rope_style);
   int per_sm = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kInjectThreads, cs_smem_bytes(c.head_dim, 16));
@@ -767,8 +775,10 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.hdr = s->ws_hdr;
   ia.st = s->d_status;
   ia.fact_len_count = s->num_facts;
-  void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena)
-                   : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena);
+  void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena,
+                              ia.vec_order)
+                   : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena,
+                                 ia.vec_order);
   int32_t small_R = R, small_ids = num_ids, small_grid = s->inject_grid, small_blocks = s->max_blocks;
   int64_t small_cap = slot_cap;
   void* small_args[] = {&ia, &small_R, &small_ids, &small_cap, &small_grid, &small_blocks};
@@ -1116,7 +1126,7 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   ia.desc = pa.desc;
   ia.hdr = hdr;
   ia.st = status;
-  void* fn = pick_inject(c.head_dim, c.rope_style, c.num_kv_heads, k.block_size);
+  void* fn = pick_inject(c.head_dim, c.rope_style, c.num_kv_heads, k.block_size, false, ia.vec_order);
   void* args[] = {&ia};
   if (cudaLaunchKernel(fn, dim3(unsigned(grid)), dim3(kInjectThreads), args,
                        cs_smem_bytes(c.head_dim, k.block_size), st) != cudaSuccess)
