@@ -16,7 +16,11 @@ layer and KV head (inject kernel).  Inputs are synthetic and seeded; the
 Multi-GPU (torchrun, one rank per GPU): every rank is an independent replica
 with its own store and batch (requests are independent; no collective on the
 data path), so the scaling is weak and the value is the sum over ranks of
-tokens divided by the slowest rank's time.
+tokens divided by the slowest rank's time.  ``--shard heads`` splits the KV
+heads of one larger batch over the ranks; ``--shard facts`` splits the facts
+over the ranks, each rank injecting 100 requests and reading the facts it
+does not hold from the peers' arenas over NVLink inside the inject kernel
+(roofline: those bytes at the peer-copy bandwidth).
 
 ``--impl reference`` times the CPU oracle (the plain fp64 C definition of the
 path) on the host cores, on a bounded sample of the same workload per step.
@@ -40,6 +44,9 @@ sys.path.insert(0, ROOT)
 sys.path.insert(0, os.path.join(ROOT, "tests"))
 
 METRIC = "injected KV tokens/s and achieved HBM GB/s (vs ~8 TB/s); per-batch inject µs"
+# NVLink 5 peer copy measured on this kind of node, per direction per GPU
+# (900 GB/s nominal): the bound of reads from a peer's arenas.
+NVLINK_PEER_GBS = 770.0
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["kv_cache_injection_gather_b200/csrc/inject_kernels.cuh",
                   "kv_cache_injection_gather_b200/csrc/inject_store.cu"]
@@ -517,7 +524,19 @@ def run_ours(args, rank, world, local_rank):
         return run_offload(args, rank, world, local_rank)
     extra_cfg = {}
     heads = None
-    if args.shard == "heads":
+    owner = None
+    if args.shard == "facts":
+        # Fact shards: one fact pool and one batch of 100 requests for every
+        # rank; rank p holds the facts g with g % N == p and injects the whole
+        # batch (global ids) into its own cache, reading the other ranks'
+        # facts from their arenas over NVLink inside the inject kernel.
+        from kv_cache_injection_gather_b200 import shard
+        if args.workload not in ("llama-batch", "llama-batch-small"):
+            raise SystemExit("--shard facts is defined for the llama-batch workloads")
+        wl = WORKLOADS[args.workload][1](0)
+        owner = shard.round_robin_owner(len(wl.fact_lens), world)
+        extra_cfg["facts_per_rank"] = int((owner == rank).sum())
+    elif args.shard == "heads":
         # KV-head shards (tensor-parallel serving): every rank holds heads
         # [h0, h1) of every fact and of the cache and injects the same batch of
         # 100 x world requests; per-GPU bytes stay those of the 1-GPU batch.
@@ -530,7 +549,16 @@ def run_ours(args, rank, world, local_rank):
         extra_cfg["kv_heads_per_rank"] = heads[1] - heads[0]
     else:
         wl = WORKLOADS[args.workload][1](rank)
-    store = make_store(wl, on_device_gen=True, device=local_rank, heads=heads)
+    store = make_store(wl, on_device_gen=True, device=local_rank, heads=heads,
+                       facts=None if owner is None else shard.owned_facts(owner, rank))
+    group = None
+    if owner is not None:
+        if world > 1:
+            group = shard.FactShardGroup(store, owner)
+        else:
+            info = [store.fact_info(i) for i in range(store.num_facts)]
+            store.attach_shards([store.arena_ptrs()], *shard.global_fact_table(
+                owner, [([o for o, _ in info], [n for _, n in info])]))
     m, b = wl.model, wl.batch
     if heads is not None:
         m = synth.Model(m.name, m.num_layers, heads[1] - heads[0], m.head_dim, m.rope_theta, m.llama3)
@@ -615,7 +643,7 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = hbm_peak()
     achieved = algo_bytes / (kern_avg_ms / 1e3) / 1e9
     traffic_pt, rec = recorded_traffic()
-    if args.workload != "llama-batch" or args.head_major:
+    if args.workload != "llama-batch" or args.head_major or owner is not None:
         traffic_pt = None  # the committed counters are for the benchmark workload
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
@@ -625,7 +653,22 @@ def run_ours(args, rank, world, local_rank):
                 "traffic": None if traffic_pt is None else traffic_pt * n_tok,
                 "algorithmic_bytes": algo_bytes,
                 "kernel": "inject_kernel (plan_kernel excluded)"}
+    if owner is not None and world > 1:
+        # Peer reads: rows of facts other ranks own cross NVLink once; the
+        # bound is those bytes at the measured peer-copy bandwidth.
+        ids_all = b.fact_ids
+        remote_tok = int(wl.fact_lens[ids_all[owner[ids_all] != rank]].sum())
+        link_bytes = remote_tok * m.bytes_per_token
+        link = link_bytes / (kern_avg_ms / 1e3) / 1e9
+        roofline = {"bound": "nvlink", "achieved": link, "peak": NVLINK_PEER_GBS,
+                    "unit": "GB/s", "frac": link / NVLINK_PEER_GBS,
+                    "peak_source": "measured peer copy per direction (pool reference)",
+                    "link_bytes": link_bytes, "hbm_achieved_gbs": achieved,
+                    "hbm_frac": achieved / peak, "traffic": None, "algorithmic_bytes": algo_bytes,
+                    "kernel": "inject_kernel (plan_kernel excluded)"}
     baseline = cpu_baseline(wl, local_rank) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if group is not None:
+        group.close()
     if rank != 0:
         store.close()
         return 0
@@ -635,8 +678,10 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": workload_config(wl, args.workload,
-                                  dict(extra_cfg, parallelism=(f"kv-head shards x{world}" if heads
-                                                               else f"replicas x{world}"))),
+                                  dict(extra_cfg, parallelism=(
+                                      f"kv-head shards x{world}" if heads is not None else
+                                      f"fact shards x{world} (peer reads over NVLink)" if owner is not None
+                                      else f"replicas x{world}"))),
         "us_per_batch": ms_step * 1e3,
         "gbs_per_gpu": algo_bytes / (ms_step / 1e3) / 1e9,
         "kernel_us": kern_avg_ms * 1e3,
@@ -662,9 +707,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-policy", choices=["static", "lru"], default="static",
                     help="offload workload: static top-20%% hot set or LRU promotion")
-    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
-                    help="multi-GPU: independent replicas (default) or KV-head shards of one "
-                         "batch of 100 x N requests (both weak scaling, no collective)")
+    ap.add_argument("--shard", choices=["replicas", "heads", "facts"], default="replicas",
+                    help="multi-GPU: independent replicas (default), KV-head shards of one "
+                         "batch of 100 x N requests (both weak scaling, no collective), or fact "
+                         "shards (each rank holds 1/N of the facts and injects 100 requests, "
+                         "reading the rest from peers over NVLink)")
     ap.add_argument("--head-major", action="store_true",
                     help="cache layout [L][num_blocks][H][B][D] instead of [L][num_blocks][B][H][D]")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama-batch",

@@ -196,6 +196,71 @@ int is_store_tier_info(const is_store_t* store, int32_t* tier_out, int64_t* hot_
 int is_store_arena(const is_store_t* store, void** k_arena_out, void** v_arena_out,
                    int64_t* plane_tokens_out);
 
+/* ---- fact-sharded stores (several GPUs) -------------------------------- */
+
+/* When the facts outgrow one GPU's memory (technical summary, Results,
+ * "Scalability" names that limit; its answer there is host DRAM, the host
+ * tier above), the store can instead be split by fact over the GPUs of a
+ * node: each GPU keeps a store holding its share of the facts, and every
+ * GPU injects its own requests reading each fact from the GPU that holds it
+ * -- its own HBM, or a peer's over NVLink -- inside the one inject kernel,
+ * with no staging copy.  The pages do not describe this partition; the
+ * method (positions, rotation, scatter) is unchanged.
+ *
+ * A view is attached to a device-tier store (its "home": batch work space,
+ * stream, status) and lists the shards' arenas and a global fact table.
+ * While it is attached, the store's batches take GLOBAL fact ids, in
+ * [0, num_global_facts), and read fact g's rows from arena fact_shard[g] at
+ * token fact_offset[g] of every plane.  Every arena has the home store's
+ * L, H and D and layout [L][H][plane_tokens][D] (another store's
+ * is_store_arena, this GPU's or a peer's opened with is_ipc_open).
+ *
+ * Arguments (host arrays, copied):
+ *   num_shards        >= 1
+ *   k_arenas, v_arenas  [num_shards] device addresses, 16-byte aligned
+ *   plane_tokens      [num_shards] tokens per plane of each arena
+ *   num_global_facts  >= 1
+ *   fact_shard        int32 [num_global_facts], in [0, num_shards)
+ *   fact_offset       int64 [num_global_facts], >= 0
+ *   fact_len          int32 [num_global_facts], >= 1, and
+ *                     fact_offset + fact_len <= plane_tokens[fact_shard]
+ * Replaces a previous view.  Waits for the device to go idle first.  The
+ * arenas must stay valid and unchanged while batches that read them run
+ * (for peers: keep their stores alive and stop putting facts until every
+ * GPU's batches are done).  Errors: INVALID_ARG (null, bad table entry;
+ * the previous view is kept), NOT_SUPPORTED (host-tier store), OOM, CUDA. */
+int is_store_attach_shards(is_store_t* store, int32_t num_shards, const void* const* k_arenas,
+                           const void* const* v_arenas, const int64_t* plane_tokens,
+                           int32_t num_global_facts, const int32_t* fact_shard,
+                           const int64_t* fact_offset, const int32_t* fact_len);
+
+/* Drop the view: the store's batches read its own facts again.  Waits for
+ * the device to go idle first.  A store with no view is left as it is. */
+int is_store_detach_shards(is_store_t* store);
+
+/* Number of shards of the attached view (0: none) and of its global facts. */
+int is_store_shard_info(const is_store_t* store, int32_t* num_shards_out,
+                        int32_t* num_global_facts_out);
+
+/* Inter-process handle of a device allocation (a cudaIpcMemHandle_t). */
+typedef struct {
+  unsigned char bytes[64];
+} is_ipc_handle_t;
+
+/* Handles of a device-tier store's K and V arenas, for other processes on
+ * this node to open with is_ipc_open, and its plane stride in tokens.
+ * Errors: INVALID_ARG, NOT_SUPPORTED (host-tier store), CUDA. */
+int is_store_export(const is_store_t* store, is_ipc_handle_t* k_handle_out,
+                    is_ipc_handle_t* v_handle_out, int64_t* plane_tokens_out);
+
+/* Map another process's exported arena into this process on `device`
+ * (peer access enabled when the arena is on another GPU); *ptr_out is its
+ * base address here.  is_ipc_close unmaps it: only after every batch that
+ * reads it has finished.  A handle from this same process is refused by
+ * CUDA (use is_store_arena instead).  Errors: INVALID_ARG, CUDA. */
+int is_ipc_open(int device, const is_ipc_handle_t* handle, void** ptr_out);
+int is_ipc_close(int device, void* ptr);
+
 /* ---- the hot path ------------------------------------------------------ */
 
 /* Inject one batch (technical summary, Online phase, "Dynamic rotation" and

@@ -60,6 +60,10 @@ class is_cache_t(ctypes.Structure):
     ]
 
 
+class is_ipc_handle_t(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64)]
+
+
 class InjectError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -101,6 +105,14 @@ _SIGNATURES = {
                                           ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
     "is_store_tier_info": (ctypes.c_int, [_P, ctypes.POINTER(_I32), ctypes.POINTER(_I64),
                                           ctypes.POINTER(_I64), ctypes.POINTER(_I32)]),
+    "is_store_attach_shards": (ctypes.c_int, [_P, _I32, _P, _P, _P, _I32, _P, _P, _P]),
+    "is_store_detach_shards": (ctypes.c_int, [_P]),
+    "is_store_shard_info": (ctypes.c_int, [_P, ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
+    "is_store_export": (ctypes.c_int, [_P, ctypes.POINTER(is_ipc_handle_t),
+                                       ctypes.POINTER(is_ipc_handle_t), ctypes.POINTER(_I64)]),
+    "is_ipc_open": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(is_ipc_handle_t),
+                                   ctypes.POINTER(_P)]),
+    "is_ipc_close": (ctypes.c_int, [ctypes.c_int, _P]),
     "is_inject_batch_noalloc": (ctypes.c_int, [ctypes.POINTER(is_store_config_t), _P, _P, _I64,
                                                _P, _P, _I32, _I32, _P, _P, _I32, _P, _P, _I32,
                                                ctypes.POINTER(is_cache_t), _P, _I64, _P, _P]),
@@ -173,6 +185,54 @@ def is_store_arena(store: int) -> tuple[int, int, int]:
     check(_lib.is_store_arena(store, ctypes.byref(k), ctypes.byref(v), ctypes.byref(t)),
           "is_store_arena")
     return k.value, v.value, t.value
+
+
+def is_store_attach_shards(store: int, k_arenas: list[int], v_arenas: list[int],
+                           plane_tokens: list[int], fact_shard, fact_offset, fact_len) -> None:
+    """fact_shard / fact_offset / fact_len: int32 / int64 / int32 sequences
+    of one length (host; copied)."""
+    n, nf = len(k_arenas), len(fact_shard)
+    if len(v_arenas) != n or len(plane_tokens) != n or len(fact_offset) != nf or len(fact_len) != nf:
+        raise ValueError("is_store_attach_shards: array lengths differ")
+    ka = (_P * max(n, 1))(*k_arenas)
+    va = (_P * max(n, 1))(*v_arenas)
+    pt = (_I64 * max(n, 1))(*plane_tokens)
+    fs = (_I32 * max(nf, 1))(*[int(x) for x in fact_shard])
+    fo = (_I64 * max(nf, 1))(*[int(x) for x in fact_offset])
+    fl = (_I32 * max(nf, 1))(*[int(x) for x in fact_len])
+    check(_lib.is_store_attach_shards(store, n, ka, va, pt, nf, fs, fo, fl), "is_store_attach_shards")
+
+
+def is_store_detach_shards(store: int) -> None:
+    check(_lib.is_store_detach_shards(store), "is_store_detach_shards")
+
+
+def is_store_shard_info(store: int) -> tuple[int, int]:
+    n, nf = _I32(), _I32()
+    check(_lib.is_store_shard_info(store, ctypes.byref(n), ctypes.byref(nf)), "is_store_shard_info")
+    return n.value, nf.value
+
+
+def is_store_export(store: int) -> tuple[bytes, bytes, int]:
+    """(K handle, V handle, plane tokens); handles as 64-byte strings."""
+    hk, hv, t = is_ipc_handle_t(), is_ipc_handle_t(), _I64()
+    check(_lib.is_store_export(store, ctypes.byref(hk), ctypes.byref(hv), ctypes.byref(t)),
+          "is_store_export")
+    return bytes(hk.bytes), bytes(hv.bytes), t.value
+
+
+def is_ipc_open(device: int, handle: bytes) -> int:
+    if len(handle) != 64:
+        raise ValueError("is_ipc_open: a handle is 64 bytes")
+    h = is_ipc_handle_t()
+    ctypes.memmove(h.bytes, handle, 64)
+    out = _P()
+    check(_lib.is_ipc_open(device, ctypes.byref(h), ctypes.byref(out)), "is_ipc_open")
+    return out.value
+
+
+def is_ipc_close(device: int, ptr: int) -> None:
+    check(_lib.is_ipc_close(device, ptr), "is_ipc_close")
 
 
 def is_inject_batch(store: int, num_requests: int, req_fact_offsets: int, fact_ids: int,

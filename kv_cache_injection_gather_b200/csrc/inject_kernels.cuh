@@ -342,6 +342,13 @@ struct InjectArgs {
   const uint16_t* v_hot;
   int64_t hot_plane;         // hot_cap * D
   const int64_t* hot_off;    // [num_facts], -1 when the fact is not in HBM
+  // fact-sharded view (per-slot source variant; shard_k == nullptr: none):
+  // fact f's rows sit in arena fact_shard[f] ([L][H][plane][D], this GPU's
+  // or a peer's memory) at token fact_off[f]
+  const uint16_t* const* shard_k;  // [num_shards]
+  const uint16_t* const* shard_v;
+  const int64_t* shard_plane;      // elements between (l,h) planes of each arena
+  const int32_t* fact_shard;       // [num_facts]
 };
 
 // Streaming 16-byte accesses: every store row is read once per batch and
@@ -516,7 +523,8 @@ __device__ __forceinline__ void split_vec(int rem, int order, const Divisor<POW2
 template <bool HOST_TIER>
 struct UnitShared {
   long long src[kMaxBlockSize];  // store token of each in-block slot (-1: none)
-  // host tier: per-slot K/V row bases (token offset applied) and plane stride
+  // per-slot sources (host tier, sharded view): K/V row bases (token offset
+  // applied) and plane stride
   const uint16_t* kb[HOST_TIER ? kMaxBlockSize : 1];
   const uint16_t* vb[HOST_TIER ? kMaxBlockSize : 1];
   long long pl[HOST_TIER ? kMaxBlockSize : 1];
@@ -570,7 +578,12 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
       const int f = a.fact_ids[j];
       const int t = i - seg[j];
       src = a.fact_off[f] + t;
-      if (HOST_TIER) {
+      if (HOST_TIER && a.shard_k) {
+        const int sh = a.fact_shard[f];
+        s_kb[o] = a.shard_k[sh] + src * D;
+        s_vb[o] = a.shard_v[sh] + src * D;
+        s_pl[o] = a.shard_plane[sh];
+      } else if (HOST_TIER) {
         const long long ho = a.hot_off[f];
         if (ho >= 0) {
           s_kb[o] = a.k_hot + (ho + t) * D;
@@ -601,20 +614,33 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
 
   // FAST: compile-time H and B with one head's block row of vectors (B * D/8)
   // equal to the CTA, slot-fastest rows (token-major cache; the launch picks
-  // FAST only for vector order 1), device tier.  Each thread then owns one
-  // (slot o, word c) for every head and layer of the unit: its source row,
-  // cache address and cos/sin words are set up once per unit, and each
-  // vector costs one plane step.
+  // FAST only for vector order 1).  Each thread then owns one (slot o, word
+  // c) for every head and layer of the unit: its source row and plane stride
+  // (the store's, or the slot's own with per-slot sources), cache address
+  // and cos/sin words are set up once per unit, and each vector costs one
+  // plane step.
   if constexpr (FAST) {
-    static_assert(HC > 0 && BC > 0 && BC * VPR == NT && !HOST_TIER, "fast path shape");
+    static_assert(HC > 0 && BC > 0 && BC * VPR == NT, "fast path shape");
     {
       const int o = tid / VPR, c = tid % VPR;
       const long long src = s_src[o];
       const bool act = src >= 0;
       float4 cs[4];
       load_cs<D, STYLE>(s_cs4 + o * (D / 4), c, cs);
-      const uint16_t* kp = a.k_store + (act ? src : 0) * D + c * 8 + (long long)l0 * HC * a.plane;
-      const uint16_t* vp = a.v_store + (act ? src : 0) * D + c * 8 + (long long)l0 * HC * a.plane;
+      const uint16_t* krow;
+      const uint16_t* vrow;
+      long long pl;
+      if constexpr (HOST_TIER) {
+        krow = act ? s_kb[o] : a.k_store;
+        vrow = act ? s_vb[o] : a.v_store;
+        pl = act ? s_pl[o] : 0;
+      } else {
+        krow = a.k_store + (act ? src : 0) * D;
+        vrow = a.v_store + (act ? src : 0) * D;
+        pl = a.plane;
+      }
+      const uint16_t* kp = krow + c * 8 + (long long)l0 * HC * pl;
+      const uint16_t* vp = vrow + c * 8 + (long long)l0 * HC * pl;
       uint16_t* kd = a.k_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
       uint16_t* vd = a.v_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
       const int nw = (l1 - l0) * HC;  // (layer, head) rows of this thread, in plane order
@@ -626,8 +652,8 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
           kv[q] = make_uint4(0, 0, 0, 0);
           vv[q] = kv[q];
           if (act && w < nw) {
-            kv[q] = ld_stream(kp + (long long)w * a.plane);
-            vv[q] = ld_stream(vp + (long long)w * a.plane);
+            kv[q] = ld_stream(kp + (long long)w * pl);
+            vv[q] = ld_stream(vp + (long long)w * pl);
           }
         }
       };
@@ -742,9 +768,11 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
 // lg = u / total_blocks, so CTAs running side by side read neighbouring
 // tokens of the same layers.  Units are taken from an atomic counter; the
 // next unit is fetched while the current one is copied.  POW2: H and B are
-// powers of two (all index splits are shifts).  HOST_TIER: the store lives
-// in pinned host memory read over the host link, except the facts that also
-// sit in the HBM hot arenas; the source of every slot is chosen per fact.
+// powers of two (all index splits are shifts).  HOST_TIER: the source of
+// every slot is chosen per fact — the store lives in pinned host memory read
+// over the host link, except the facts that also sit in the HBM hot arenas;
+// or, with a sharded view, facts live in several stores' arenas (peer GPUs'
+// memory read over NVLink, or this GPU's).
 template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0,
           bool FAST = false>
 __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {

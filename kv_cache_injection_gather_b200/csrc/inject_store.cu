@@ -108,6 +108,16 @@ struct is_store {
   bool timing = false;
   std::vector<TimedLaunch> events;
   size_t events_used = 0;
+  // fact-sharded view (is_store_attach_shards): arenas of several stores and
+  // a global fact table; batches take global ids while it is attached
+  int32_t shard_n = 0;
+  int32_t shard_facts = 0;
+  const uint16_t** d_shard_k = nullptr;
+  const uint16_t** d_shard_v = nullptr;
+  int64_t* d_shard_plane = nullptr;  // elements between (l,h) planes
+  int32_t* d_shard_of = nullptr;     // [shard_facts]
+  int64_t* d_shard_off = nullptr;
+  int32_t* d_shard_len = nullptr;
   // kernel configuration
   int inject_grid = 0;
   int32_t small_limit = isk::kSmallRequests;  // batches up to this many requests: one kernel
@@ -131,8 +141,36 @@ cudaError_t dalloc(T** p, size_t count) {
   return cudaMalloc(reinterpret_cast<void**>(p), std::max<size_t>(count, 1) * sizeof(T));
 }
 
+struct ShardView {
+  const uint16_t** k = nullptr;
+  const uint16_t** v = nullptr;
+  int64_t* plane = nullptr;
+  int32_t* of = nullptr;
+  int64_t* off = nullptr;
+  int32_t* len = nullptr;
+  void release() {
+    cudaFree(k);
+    cudaFree(v);
+    cudaFree(plane);
+    cudaFree(of);
+    cudaFree(off);
+    cudaFree(len);
+    *this = ShardView{};
+  }
+};
+
+void free_view(is_store* s) {
+  ShardView{s->d_shard_k, s->d_shard_v, s->d_shard_plane, s->d_shard_of, s->d_shard_off, s->d_shard_len}
+      .release();
+  s->d_shard_k = s->d_shard_v = nullptr;
+  s->d_shard_plane = s->d_shard_off = nullptr;
+  s->d_shard_of = s->d_shard_len = nullptr;
+  s->shard_n = s->shard_facts = 0;
+}
+
 void free_store(is_store* s) {
   if (!s) return;
+  free_view(s);
   cudaFree(s->d_off);
   cudaFree(s->d_len);
   cudaFree(s->d_inv_freq);
@@ -209,15 +247,14 @@ void* fixed_fn(int style) {
                         : inject_fn<128, 0, true, HOST_TIER, HC, 16, FAST>());
 }
 
-// order: the launch's vector order (1: slot-fastest, the FAST copy loop on
-// the device tier).
+// order: the launch's vector order (1: slot-fastest, the FAST copy loop).
 template <bool SMALL, bool HOST_TIER>
 void* pick_fixed(int D, int style, int H, int B, int order) {
 #ifndef IS_NO_FIXED_SHAPES
   if (D != 128 || B != 16) return nullptr;
-  const bool fast = order == 1 && !HOST_TIER;
-  if (H == 8) return fast ? fixed_fn<SMALL, HOST_TIER, 8, !HOST_TIER>(style) : fixed_fn<SMALL, HOST_TIER, 8, false>(style);
-  if (H == 4) return fast ? fixed_fn<SMALL, HOST_TIER, 4, !HOST_TIER>(style) : fixed_fn<SMALL, HOST_TIER, 4, false>(style);
+  const bool fast = order == 1;
+  if (H == 8) return fast ? fixed_fn<SMALL, HOST_TIER, 8, true>(style) : fixed_fn<SMALL, HOST_TIER, 8, false>(style);
+  if (H == 4) return fast ? fixed_fn<SMALL, HOST_TIER, 4, true>(style) : fixed_fn<SMALL, HOST_TIER, 4, false>(style);
 #else
   (void)D; (void)style; (void)H; (void)B; (void)order;
 #endif
@@ -515,6 +552,124 @@ int is_store_arena(const is_store_t* s, void** k, void** v, int64_t* plane_token
   return IS_OK;
 }
 
+int is_store_attach_shards(is_store_t* s, int32_t n, const void* const* k_arenas, const void* const* v_arenas,
+                           const int64_t* plane_tokens, int32_t nf, const int32_t* fact_shard,
+                           const int64_t* fact_offset, const int32_t* fact_len) {
+  if (!s || n < 1 || nf < 1 || !k_arenas || !v_arenas || !plane_tokens || !fact_shard || !fact_offset ||
+      !fact_len)
+    return IS_ERR_INVALID_ARG;
+  if (s->host_arena) return IS_ERR_NOT_SUPPORTED;
+  for (int32_t i = 0; i < n; ++i)
+    if (!k_arenas[i] || !v_arenas[i] || !aligned16(k_arenas[i]) || !aligned16(v_arenas[i]) ||
+        plane_tokens[i] < 1 || plane_tokens[i] > (int64_t(1) << 31) - 1)
+      return IS_ERR_INVALID_ARG;
+  for (int32_t g = 0; g < nf; ++g) {
+    const int32_t sh = fact_shard[g];
+    if (sh < 0 || sh >= n || fact_offset[g] < 0 || fact_len[g] < 1 ||
+        fact_offset[g] + fact_len[g] > plane_tokens[sh])
+      return IS_ERR_INVALID_ARG;
+  }
+  DeviceGuard guard(s->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return IS_ERR_CUDA;
+  const int64_t D = s->cfg.head_dim;
+  std::vector<const uint16_t*> hk(static_cast<size_t>(n)), hv(static_cast<size_t>(n));
+  std::vector<int64_t> hp(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) {
+    hk[size_t(i)] = static_cast<const uint16_t*>(k_arenas[i]);
+    hv[size_t(i)] = static_cast<const uint16_t*>(v_arenas[i]);
+    hp[size_t(i)] = plane_tokens[i] * D;
+  }
+  ShardView nv;
+  if (dalloc(&nv.k, size_t(n)) != cudaSuccess || dalloc(&nv.v, size_t(n)) != cudaSuccess ||
+      dalloc(&nv.plane, size_t(n)) != cudaSuccess || dalloc(&nv.of, size_t(nf)) != cudaSuccess ||
+      dalloc(&nv.off, size_t(nf)) != cudaSuccess || dalloc(&nv.len, size_t(nf)) != cudaSuccess) {
+    cudaGetLastError();
+    nv.release();
+    return IS_ERR_OOM;
+  }
+  if (cudaMemcpy(nv.k, hk.data(), sizeof(void*) * size_t(n), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(nv.v, hv.data(), sizeof(void*) * size_t(n), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(nv.plane, hp.data(), sizeof(int64_t) * size_t(n), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(nv.of, fact_shard, sizeof(int32_t) * size_t(nf), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(nv.off, fact_offset, sizeof(int64_t) * size_t(nf), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(nv.len, fact_len, sizeof(int32_t) * size_t(nf), cudaMemcpyHostToDevice) != cudaSuccess) {
+    nv.release();
+    return IS_ERR_CUDA;
+  }
+  free_view(s);
+  s->d_shard_k = nv.k;
+  s->d_shard_v = nv.v;
+  s->d_shard_plane = nv.plane;
+  s->d_shard_of = nv.of;
+  s->d_shard_off = nv.off;
+  s->d_shard_len = nv.len;
+  s->shard_n = n;
+  s->shard_facts = nf;
+  return IS_OK;
+}
+
+int is_store_detach_shards(is_store_t* s) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  if (s->shard_n == 0) return IS_OK;
+  DeviceGuard guard(s->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return IS_ERR_CUDA;
+  free_view(s);
+  return IS_OK;
+}
+
+int is_store_shard_info(const is_store_t* s, int32_t* num_shards, int32_t* num_global_facts) {
+  if (!s) return IS_ERR_INVALID_ARG;
+  if (num_shards) *num_shards = s->shard_n;
+  if (num_global_facts) *num_global_facts = s->shard_facts;
+  return IS_OK;
+}
+
+static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(is_ipc_handle_t), "IPC handle size");
+
+int is_store_export(const is_store_t* s, is_ipc_handle_t* k_handle, is_ipc_handle_t* v_handle,
+                    int64_t* plane_tokens) {
+  if (!s || !k_handle || !v_handle) return IS_ERR_INVALID_ARG;
+  if (s->host_arena) return IS_ERR_NOT_SUPPORTED;
+  DeviceGuard guard(s->device);
+  cudaIpcMemHandle_t hk, hv;
+  if (cudaIpcGetMemHandle(&hk, s->k) != cudaSuccess || cudaIpcGetMemHandle(&hv, s->v) != cudaSuccess) {
+    cudaGetLastError();
+    return IS_ERR_CUDA;
+  }
+  std::memcpy(k_handle->bytes, &hk, sizeof(hk));
+  std::memcpy(v_handle->bytes, &hv, sizeof(hv));
+  if (plane_tokens) *plane_tokens = s->cfg.capacity_tokens;
+  return IS_OK;
+}
+
+int is_ipc_open(int device, const is_ipc_handle_t* handle, void** ptr) {
+  if (!handle || !ptr) return IS_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return IS_ERR_INVALID_ARG;
+  DeviceGuard guard(device);
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle->bytes, sizeof(h));
+  if (cudaIpcOpenMemHandle(ptr, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();
+    *ptr = nullptr;
+    return IS_ERR_CUDA;
+  }
+  return IS_OK;
+}
+
+int is_ipc_close(int device, void* ptr) {
+  if (!ptr) return IS_ERR_INVALID_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return IS_ERR_INVALID_ARG;
+  DeviceGuard guard(device);
+  if (cudaIpcCloseMemHandle(ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return IS_ERR_CUDA;
+  }
+  return IS_OK;
+}
+
 int is_store_set_hot(is_store_t* s, const int32_t* fact_ids, int32_t n) {
   if (!s || n < 0 || (n > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
   if (!s->host_arena || s->hot_policy != IS_HOT_STATIC) return IS_ERR_NOT_SUPPORTED;
@@ -723,8 +878,11 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.max_blocks = max_blocks_per_req;
   pa.B = c.block_size;
   pa.L = cf.num_layers;
-  pa.fact_len = s->d_len;
-  pa.num_facts = s->num_facts;
+  // With a sharded view attached, ids are global: the view's fact table.
+  const bool view = s->shard_n > 0;
+  const int32_t nfacts = view ? s->shard_facts : s->num_facts;
+  pa.fact_len = view ? s->d_shard_len : s->d_len;
+  pa.num_facts = nfacts;
   pa.slot_out = slot_out;
   pa.slot_cap = slot_cap;
   pa.grid_ctas = s->inject_grid;
@@ -749,8 +907,12 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.hot_plane = s->hot_cap * cf.head_dim;
   ia.hot_off = s->d_hot;
   ia.plane = int64_t(cf.capacity_tokens) * cf.head_dim;
-  ia.fact_off = s->d_off;
-  ia.fact_len = s->d_len;
+  ia.fact_off = view ? s->d_shard_off : s->d_off;
+  ia.fact_len = view ? s->d_shard_len : s->d_len;
+  ia.shard_k = view ? s->d_shard_k : nullptr;
+  ia.shard_v = view ? s->d_shard_v : nullptr;
+  ia.shard_plane = s->d_shard_plane;
+  ia.fact_shard = s->d_shard_of;
   ia.inv_freq = s->d_inv_freq;
   ia.L = cf.num_layers;
   ia.H = cf.num_kv_heads;
@@ -774,10 +936,11 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.desc = s->ws_desc;
   ia.hdr = s->ws_hdr;
   ia.st = s->d_status;
-  ia.fact_len_count = s->num_facts;
-  void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena,
-                              ia.vec_order)
-                   : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, s->host_arena,
+  ia.fact_len_count = nfacts;
+  // Per-slot sources: the host tier, or the arenas of a sharded view.
+  const bool per_slot = s->host_arena || view;
+  void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, ia.vec_order)
+                   : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot,
                                  ia.vec_order);
   int32_t small_R = R, small_ids = num_ids, small_grid = s->inject_grid, small_blocks = s->max_blocks;
   int64_t small_cap = slot_cap;

@@ -145,6 +145,29 @@ class FactStore:
         v = torch.as_tensor(_DeviceArray(vp, shape, "<i2"), device=dev).view(torch.bfloat16)
         return k, v
 
+    # ---- fact-sharded view
+    def export(self) -> tuple[bytes, bytes, int]:
+        """IPC handles of the K and V arenas (for peers' is_ipc_open) and the
+        plane stride in tokens."""
+        return B.is_store_export(self.handle)
+
+    def arena_ptrs(self) -> tuple[int, int, int]:
+        """Device addresses of the K and V arenas and the plane stride."""
+        return B.is_store_arena(self.handle)
+
+    def attach_shards(self, arenas, fact_shard, fact_offset, fact_len) -> None:
+        """arenas: [(k_ptr, v_ptr, plane_tokens)] per shard; the global fact
+        table as three host sequences.  Batches then take global fact ids."""
+        B.is_store_attach_shards(self.handle, [a[0] for a in arenas], [a[1] for a in arenas],
+                                 [a[2] for a in arenas], fact_shard, fact_offset, fact_len)
+
+    def detach_shards(self) -> None:
+        B.is_store_detach_shards(self.handle)
+
+    def shard_info(self) -> tuple[int, int]:
+        """(shards, global facts) of the attached view; (0, 0) when none."""
+        return B.is_store_shard_info(self.handle)
+
     def set_hot(self, fact_ids) -> None:
         """Host tier: keep these facts (host int sequence) in the HBM hot arenas."""
         import numpy as np

@@ -21,19 +21,22 @@ def rope_of(model: synth.Model, style: int = 0) -> RopeConfig:
 
 def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = None,
                device: int = 0, extra_tokens: int = 0, small_limit: int | None = None,
-               heads: tuple[int, int] | None = None, **limits) -> FactStore:
+               heads: tuple[int, int] | None = None, facts=None, **limits) -> FactStore:
     """Put every fact of the workload, in id order (ids equal indices).
 
     Small stores are generated on the host (numpy) and copied; large ones are
     generated on the device by the same counter-based definition.  heads =
     (h0, h1) keeps KV heads [h0, h1) of every fact (a head-sharded store; the
-    workload's model then names the full head count)."""
+    workload's model then names the full head count).  facts = increasing
+    global ids keeps only those facts, local id i holding facts[i] (a
+    fact-sharded store)."""
     full = wl.model
     m = full if heads is None else synth.Model(full.name, full.num_layers, heads[1] - heads[0],
                                                full.head_dim, full.rope_theta, full.llama3)
-    total = int(wl.fact_lens.sum()) + extra_tokens
-    store = FactStore(m.num_layers, m.num_kv_heads, m.head_dim, rope_of(m, style), total,
-                      len(wl.fact_lens), device=device, **limits)
+    ids = np.arange(len(wl.fact_lens)) if facts is None else np.asarray(facts, np.int64)
+    total = int(wl.fact_lens[ids].sum()) + extra_tokens
+    store = FactStore(m.num_layers, m.num_kv_heads, m.head_dim, rope_of(m, style), max(total, 1),
+                      max(len(ids), 1), device=device, **limits)
     if small_limit is not None:  # 0: always the plan + inject kernels
         store.set_small_batch_limit(small_limit)
     if on_device_gen is None:
@@ -45,8 +48,8 @@ def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = 
                            dtype=torch.bfloat16, device=dev)
         vbuf = torch.empty_like(kbuf)
         stream = torch.cuda.current_stream(dev).cuda_stream
-        for f, n in enumerate(wl.fact_lens):
-            n = int(n)
+        for i, f in enumerate(ids):
+            f, n = int(f), int(wl.fact_lens[f])
             cnt = full.num_layers * full.num_kv_heads * n * full.head_dim
             synth.fill_device(kbuf.data_ptr(), cnt, wl.seed, synth.fact_stream(f, False), 0, stream)
             synth.fill_device(vbuf.data_ptr(), cnt, wl.seed, synth.fact_stream(f, True), 0, stream)
@@ -55,17 +58,18 @@ def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = 
             if heads is not None:
                 k, v = k[:, heads[0]:heads[1]], v[:, heads[0]:heads[1]]
             fid = store.put_fact(k, v)
-            assert fid == f
+            assert fid == i
         torch.cuda.synchronize(dev)
     else:
-        for f, n in enumerate(wl.fact_lens):
-            k, v = synth.fact_kv(wl.seed, f, full.num_layers, full.num_kv_heads, int(n), full.head_dim)
+        for i, f in enumerate(ids):
+            f, n = int(f), int(wl.fact_lens[f])
+            k, v = synth.fact_kv(wl.seed, f, full.num_layers, full.num_kv_heads, n, full.head_dim)
             if heads is not None:
                 k, v = k[:, heads[0]:heads[1]], v[:, heads[0]:heads[1]]
             k, v = np.ascontiguousarray(k), np.ascontiguousarray(v)
             kt = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16)
             vt = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16)
-            assert store.put_fact(kt, vt) == f
+            assert store.put_fact(kt, vt) == i
     return store
 
 

@@ -1,7 +1,9 @@
 """The multi-GPU partitions on CPU: world_size-2 gloo ranks, the CPU oracle
 standing in for each rank's GPU.  Head shards and request shards each
-reproduce the single-rank result with no data exchange; the benchmark's
-max-over-ranks timing reduction works across processes."""
+reproduce the single-rank result with no data exchange; the fact-shard
+view's set-up (table and handle swap, peer mapping, collective close)
+routes every global fact id to its rows; the benchmark's max-over-ranks
+timing reduction works across processes."""
 from __future__ import annotations
 
 import os
@@ -110,6 +112,120 @@ def test_partitions_reproduce_single_rank_with_gloo():
         v_u.reshape(flat_v.shape)[:, sr] = flat_v[:, sr]
     assert np.array_equal(k_u, kf) and np.array_equal(v_u, vf)
     assert list(mx) == [11.0, 3.0]
+
+
+class _HostShardStore:
+    """A rank's fact store for the fact-shard set-up test: the oracle's CPU
+    store behind the calls FactShardGroup makes (arena 'addresses' are
+    tokens naming the rank)."""
+
+    def __init__(self, rank, st):
+        self.rank, self.st, self.device = rank, st, 0
+        self.attached, self.detached = None, 0
+
+    @property
+    def num_facts(self):
+        return self.st.num_facts
+
+    def fact_info(self, i):
+        return int(self.st.off[i]), int(self.st.len[i])
+
+    def export(self):
+        pad = lambda b: b.ljust(64, b"\0")  # noqa: E731
+        return pad(b"K%d" % self.rank), pad(b"V%d" % self.rank), self.st.k.shape[2]
+
+    def arena_ptrs(self):
+        return 1000 + self.rank, 2000 + self.rank, self.st.k.shape[2]
+
+    def attach_shards(self, arenas, shard_of, off, ln):
+        self.attached = (list(arenas), np.asarray(shard_of), np.asarray(off), np.asarray(ln))
+
+    def detach_shards(self):
+        self.detached += 1
+
+
+def _fact_shard_worker(rank, world, port, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from kv_cache_injection_gather_b200 import shard
+        wl = _tiny_multi(seed=3)
+        m = wl.model
+        owner = shard.round_robin_owner(len(wl.fact_lens), world)
+        mine = shard.owned_facts(owner, rank)
+        st = oracle.Store(m.num_layers, m.num_kv_heads, m.head_dim,
+                          int(wl.fact_lens[mine].sum()) + 7 * rank, len(mine))
+        import synth
+        for g in mine:
+            st.put(*synth.fact_kv(wl.seed, int(g), m.num_layers, m.num_kv_heads,
+                                  int(wl.fact_lens[g]), m.head_dim))
+        fake = _HostShardStore(rank, st)
+        opened, closed = [], []
+
+        def ipc_open(dev, h):
+            ptr = {b"K": 1000, b"V": 2000}[h[:1]] + int(h[1:].rstrip(b"\0"))
+            opened.append(ptr)
+            return ptr
+
+        grp = shard.FactShardGroup(fake, owner, ipc_open=ipc_open,
+                                   ipc_close=lambda dev, p: closed.append(p))
+        arenas = [None] * world
+        dist.all_gather_object(arenas, (st.k, st.v))
+        grp.close()
+        out = {"attached": fake.attached, "opened": opened, "closed": closed,
+               "detached": fake.detached, "arenas": arenas}
+        np.save(os.path.join(out_dir, f"fs{rank}.npy"), np.array([out], dtype=object),
+                allow_pickle=True)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_fact_shard_view_routes_every_global_id_with_gloo():
+    """Fact shards, host side: over world-size-2 gloo ranks holding alternate
+    facts, every rank builds the same global table and arena list (its own
+    arena, the peer's through the IPC mapping), and each global id's entry
+    points at that fact's rows in its owner's arena."""
+    import synth
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_fact_shard_worker, args=(world, _free_port(), d), nprocs=world,
+                           join=True, start_method="spawn")
+        outs = [np.load(os.path.join(d, f"fs{r}.npy"), allow_pickle=True)[0] for r in range(world)]
+    wl = _tiny_multi(seed=3)
+    m = wl.model
+    for rank, o in enumerate(outs):
+        arenas, shard_of, off, ln = o["attached"]
+        assert [a[:2] for a in arenas] == [(1000 + p, 2000 + p) for p in range(world)]
+        assert sorted(o["opened"]) == sorted(o["closed"]) == [1000 + 1 - rank, 2000 + 1 - rank]
+        assert o["detached"] == 1
+        assert np.array_equal(shard_of, np.arange(len(wl.fact_lens)) % world)
+        assert np.array_equal(ln, wl.fact_lens)
+        for g in range(len(wl.fact_lens)):
+            kp, vp, plane = arenas[shard_of[g]]
+            ka, va = o["arenas"][kp - 1000][0], o["arenas"][vp - 2000][1]
+            assert plane == ka.shape[2] and off[g] + ln[g] <= plane
+            k, v = synth.fact_kv(wl.seed, g, m.num_layers, m.num_kv_heads, int(ln[g]), m.head_dim)
+            assert np.array_equal(ka[:, :, off[g]:off[g] + ln[g]], k)
+            assert np.array_equal(va[:, :, off[g]:off[g] + ln[g]], v)
+    for a, b in zip(outs[0]["attached"][1:], outs[1]["attached"][1:]):
+        assert np.array_equal(a, b)
+
+
+def test_global_fact_table_rejects_mismatched_owners():
+    from kv_cache_injection_gather_b200 import shard
+    owner = shard.round_robin_owner(5, 2)
+    assert list(owner) == [0, 1, 0, 1, 0]
+    assert list(shard.owned_facts(owner, 1)) == [1, 3]
+    s, o, n = shard.global_fact_table(owner, [([0, 10, 20], [10, 10, 5]), ([0, 7], [7, 3])])
+    assert list(s) == [0, 1, 0, 1, 0] and list(o) == [0, 0, 10, 7, 20] and list(n) == [10, 7, 10, 3, 5]
+    with pytest.raises(ValueError):
+        shard.global_fact_table(owner, [([0, 10], [10, 10]), ([0, 7], [7, 3])])
+    with pytest.raises(ValueError):
+        shard.global_fact_table([0, 2], [([0], [1]), ([0], [1])])
 
 
 def test_contiguous_ranges_cover_everything():
