@@ -69,7 +69,7 @@ struct PlanHeader {
 };
 
 // One touched cache block of one request.
-struct BlockDesc {
+struct __align__(16) BlockDesc {
   int32_t r;     // request
   int32_t b;     // logical block index in the request's table
   int32_t j;     // CSR index of the first fact with a token in the block
@@ -83,17 +83,20 @@ __device__ __forceinline__ void record_error(DevStatus* st, int32_t code, long l
 // ---------------------------------------------------------------- plan kernel
 
 // Work-unit size (layers per unit lpu, units per block upb).  A batch whose
-// one-layer units fit in about one wave of the grid uses one layer per unit:
-// everything is in flight at once (latency).  Larger batches aim at
-// ~IS_UNITS_PER_CTA units per CTA, so the dynamic schedule's tail (at most
-// one unit) stays short, with at least two layers per unit so a unit's
-// set-up (slot walk, cos/sin table) is shared by more than one layer.
+// one-layer units fit in about two waves of the grid takes the fewest layers
+// per unit that fit one wave (one layer when they already do): everything is
+// in flight at once and no CTA runs a second unit after the first (latency).
+// Larger batches aim at ~IS_UNITS_PER_CTA units per CTA, so the dynamic
+// schedule's tail (at most one unit) stays short, with at least two layers
+// per unit so a unit's set-up (slot walk, cos/sin table) is shared by more
+// than one layer.
 __device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32_t grid_ctas,
                                           int32_t& lpu, int32_t& upb) {
   const long long grid = grid_ctas;
   upb = 1;
   if (total_blocks > 0 && (long long)total_blocks * L <= 2 * grid) {
-    upb = L;
+    const long long per = ((long long)total_blocks * L + grid - 1) / grid;  // 1 or 2 layers per unit
+    upb = int32_t((L + per - 1) / per);
   } else if (total_blocks > 0) {
     const long long want = (grid * IS_UNITS_PER_CTA + total_blocks - 1) / total_blocks;
     upb = int32_t(max(1LL, min(want, (long long)max(1, L / 2))));
@@ -129,24 +132,68 @@ struct PlanArgs {
   DevStatus* st;
 };
 
-template <int NT>
+// Shared-memory plan: batches of at most kPlanSmemRequests requests and
+// kPlanSmemIds fact ids keep the CSR, the start positions, the lengths /
+// segment offsets and the per-request sums in shared memory, so the
+// per-request phases chain shared-memory rather than L2 latencies; only seg,
+// req_tok0 and the descriptors (what the inject kernel reads) go to global
+// memory.  Larger batches run the same phases on the global work space.
+constexpr int kPlanSmemRequests = 1024;
+constexpr int kPlanSmemIds = 16384;
+
+__host__ __device__ constexpr size_t plan_smem_bytes(int R, int num_ids) {
+  return sizeof(long long) * size_t(R + 1) + sizeof(int32_t) * (size_t(R + 1) * 2 + size_t(R) * 4 + size_t(num_ids));
+}
+
+template <int NT, bool SMEM>
 __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ int s_bad;
   __shared__ int s_wsum_blk[NW];
   __shared__ long long s_wsum_tok[NW];
+  extern __shared__ __align__(16) unsigned char plan_dyn[];
 
   // The inject grid may be scheduled now; it waits for this grid's results
   // (griddepcontrol.wait) before reading any of them.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+  const int32_t* req_off = a.req_off;
+  const int32_t* start_pos = a.start_pos;
+  int32_t* seg = a.seg;
+  int32_t* req_nblk = a.req_nblk;
+  int32_t* req_blk0 = a.req_blk0;
+  long long* req_tok0 = a.req_tok0;
+  int32_t* req_len = a.req_len;
+  int32_t* req_valid = a.req_valid;
+  if constexpr (SMEM) {
+    long long* s_tok0 = reinterpret_cast<long long*>(plan_dyn);  // [R+1]
+    int32_t* s_off = reinterpret_cast<int32_t*>(s_tok0 + (a.R + 1));
+    int32_t* s_blk0 = s_off + (a.R + 1);     // [R+1]
+    int32_t* s_start = s_blk0 + (a.R + 1);   // [R]
+    int32_t* s_nblk = s_start + a.R;         // [R]
+    int32_t* s_len = s_nblk + a.R;           // [R]
+    int32_t* s_valid = s_len + a.R;          // [R]
+    int32_t* s_seg = s_valid + a.R;          // [num_ids]
+    for (int i = tid; i <= a.R; i += NT) s_off[i] = a.req_off[i];
+    for (int i = tid; i < a.R; i += NT) s_start[i] = a.start_pos[i];
+    __syncthreads();
+    req_off = s_off;
+    start_pos = s_start;
+    seg = s_seg;
+    req_nblk = s_nblk;
+    req_blk0 = s_blk0;
+    req_tok0 = s_tok0;
+    req_len = s_len;
+    req_valid = s_valid;
+  }
+
   // The CSR must start at 0, end at num_ids and never decrease; otherwise
   // the whole batch is rejected and nothing is written.
-  if (tid == 0) s_bad = a.R < 0 || a.req_off[0] != 0 || a.req_off[a.R] != a.num_ids;
+  if (tid == 0) s_bad = a.R < 0 || req_off[0] != 0 || req_off[a.R] != a.num_ids;
   __syncthreads();
   for (int r = tid; r < a.R; r += NT)
-    if (a.req_off[r + 1] < a.req_off[r]) s_bad = 1;
+    if (req_off[r + 1] < req_off[r]) s_bad = 1;
   __syncthreads();
   if (tid == 0 && s_bad) {
     record_error(a.st, kErrInvalidArg, -1);
@@ -162,17 +209,18 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   // Phase 0, all threads: the length of every listed fact (-1 for an id
   // outside the store), fetched in parallel into seg[], which phase 1 then
   // overwrites with segment offsets.
-  for (int32_t base = 0; base < a.num_ids; base += NT * 4) {
-    int32_t f[4];
+  constexpr int P0 = 8;  // loads in flight per thread
+  for (int32_t base = 0; base < a.num_ids; base += NT * P0) {
+    int32_t f[P0];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < P0; ++q) {
       const int32_t j = base + q * NT + tid;
       f[q] = j < a.num_ids ? a.fact_ids[j] : -1;
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < P0; ++q) {
       const int32_t j = base + q * NT + tid;
-      if (j < a.num_ids) a.seg[j] = (f[q] >= 0 && f[q] < a.num_facts) ? a.fact_len[f[q]] : -1;
+      if (j < a.num_ids) seg[j] = (f[q] >= 0 && f[q] < a.num_facts) ? a.fact_len[f[q]] : -1;
     }
   }
   __syncthreads();
@@ -180,7 +228,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   // Phase 1, one warp per request: segment offsets of its facts (exclusive
   // prefix of their lengths, in retrieval order), length, validity, blocks.
   for (int r = warp; r < a.R; r += NW) {
-    const int32_t j0 = a.req_off[r], j1 = a.req_off[r + 1];
+    const int32_t j0 = req_off[r], j1 = req_off[r + 1];
     int32_t err = kOk;
     long long S = 0;
     if (j0 < 0 || j1 < j0 || j1 > a.num_ids) {
@@ -188,7 +236,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     } else {
       for (int32_t base = j0; base < j1; base += 32) {
         const int32_t j = base + lane;
-        const int32_t lj = j < j1 ? a.seg[j] : 0;
+        const int32_t lj = j < j1 ? seg[j] : 0;
         const bool ok = lj >= 0;
         const int32_t len = ok ? lj : 0;
         int32_t x = len;  // inclusive warp scan
@@ -197,21 +245,21 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
           const int32_t y = __shfl_up_sync(0xffffffffu, x, d);
           if (lane >= d) x += y;
         }
-        if (j < j1) a.seg[j] = ok ? int32_t(S + x - len) : -1;
+        if (j < j1) seg[j] = ok ? int32_t(S + x - len) : -1;
         const unsigned badm = __ballot_sync(0xffffffffu, j < j1 && !ok);
         if (badm && err == kOk) err = kErrBadFactId;
         S += __shfl_sync(0xffffffffu, x, 31);
       }
     }
-    const int32_t start = a.start_pos[r];
+    const int32_t start = start_pos[r];
     if (err == kOk && start < 0) err = kErrInvalidArg;
     if (err == kOk && (long long)start + S > (long long)a.max_blocks * a.B) err = kErrPosition;
     if (lane == 0) {
       int32_t nblk = 0;
       if (err == kOk && S > 0) nblk = int32_t((start + S - 1) / a.B - start / a.B + 1);
-      a.req_nblk[r] = nblk;
-      a.req_len[r] = int32_t(S);
-      a.req_valid[r] = err == kOk;
+      req_nblk[r] = nblk;
+      req_len[r] = int32_t(S);
+      req_valid[r] = err == kOk;
       if (err != kOk) record_error(a.st, err, r);
     }
   }
@@ -223,7 +271,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   const int r0 = min(a.R, tid * per), r1 = min(a.R, r0 + per);
   int32_t my_blk = 0;
   long long my_tok = 0;
-  for (int r = r0; r < r1; ++r) { my_blk += a.req_nblk[r]; my_tok += a.req_len[r]; }
+  for (int r = r0; r < r1; ++r) { my_blk += req_nblk[r]; my_tok += req_len[r]; }
   int32_t xb = my_blk;
   long long xt = my_tok;
 #pragma unroll
@@ -234,24 +282,37 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   }
   if (lane == 31) { s_wsum_blk[warp] = xb; s_wsum_tok[warp] = xt; }
   __syncthreads();
-  int32_t wb = 0;
-  long long wt = 0;
-  for (int w = 0; w < warp; ++w) { wb += s_wsum_blk[w]; wt += s_wsum_tok[w]; }
+  // Exclusive prefix of the warp sums: a shuffle scan over lanes = warps.
+  int32_t wb = lane < NW ? s_wsum_blk[lane] : 0;
+  long long wt = lane < NW ? s_wsum_tok[lane] : 0;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t yb = __shfl_up_sync(0xffffffffu, wb, d);
+    const long long yt = __shfl_up_sync(0xffffffffu, wt, d);
+    if (lane >= d) { wb += yb; wt += yt; }
+  }
+  wb = warp > 0 ? __shfl_sync(0xffffffffu, wb, warp - 1) : 0;
+  wt = warp > 0 ? __shfl_sync(0xffffffffu, wt, warp - 1) : 0;
   int32_t eb = wb + xb - my_blk;
   long long et = wt + xt - my_tok;
   for (int r = r0; r < r1; ++r) {
-    a.req_blk0[r] = eb;
-    a.req_tok0[r] = et;
-    eb += a.req_nblk[r];
-    et += a.req_len[r];
+    req_blk0[r] = eb;
+    req_tok0[r] = et;
+    eb += req_nblk[r];
+    et += req_len[r];
   }
   if (tid == NT - 1) {
-    a.req_blk0[a.R] = eb;
-    a.req_tok0[a.R] = et;
+    req_blk0[a.R] = eb;
+    req_tok0[a.R] = et;
   }
   __syncthreads();
-  const int32_t total_blocks = a.req_blk0[a.R];
-  const long long total_tokens = a.req_tok0[a.R];
+  if constexpr (SMEM) {
+    // What the inject kernel reads: segment offsets and token prefixes.
+    for (int32_t j = tid; j < a.num_ids; j += NT) a.seg[j] = seg[j];
+    for (int r = tid; r <= a.R; r += NT) a.req_tok0[r] = req_tok0[r];
+  }
+  const int32_t total_blocks = req_blk0[a.R];
+  const long long total_tokens = req_tok0[a.R];
   const bool over_slots = a.slot_out != nullptr && total_tokens > a.slot_cap;
   const bool over_blocks = total_blocks > a.max_batch_blocks;
 
@@ -268,42 +329,64 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   }
   if (over_slots || over_blocks) return;
 
-  // Phase 3, one warp per request: block descriptors (lanes over facts), and
-  // -1 slots for the tokens of invalid requests.
+  // Phase 3, one warp per request: block descriptors (lanes over blocks, so
+  // a warp writes consecutive descriptors), and -1 slots for the tokens of
+  // invalid requests.
   for (int r = warp; r < a.R; r += NW) {
-    const int32_t j0 = a.req_off[r], j1 = a.req_off[r + 1];
-    const long long t0 = a.req_tok0[r];
-    if (!a.req_valid[r]) {
+    const int32_t j0 = req_off[r], j1 = req_off[r + 1];
+    const long long t0 = req_tok0[r];
+    if (!req_valid[r]) {
       if (a.slot_out)
-        for (int32_t i = lane; i < a.req_len[r]; i += 32) a.slot_out[t0 + i] = -1;
+        for (int32_t i = lane; i < req_len[r]; i += 32) a.slot_out[t0 + i] = -1;
       continue;
     }
-    const int32_t nblk = a.req_nblk[r];
+    const int32_t nblk = req_nblk[r];
     if (nblk == 0) continue;
-    const int32_t start = a.start_pos[r];
+    const int32_t start = start_pos[r];
     const int32_t fb = start / a.B;            // first logical block
-    const int32_t g0 = a.req_blk0[r];
-    // Fact j covers segment indices [seg[j], seg[j] + len_j).  Block bi >= 1
-    // starts at segment index (fb + bi) * B - start; block 0 starts at 0.
-    const int32_t S = a.req_len[r];
-    for (int32_t base = j0; base < j1; base += 32) {
-      const int32_t j = base + lane;
-      if (j >= j1) continue;
-      const int32_t s = a.seg[j];
-      const int32_t len = (j + 1 < j1 ? a.seg[j + 1] : S) - s;  // valid request: all seg >= 0
-      if (len == 0) continue;
-      const int32_t e = s + len;               // exclusive end
-      // blocks bi whose first segment index lies in [s, e)
-      int32_t bi_lo = (s + start + a.B - 1) / a.B - fb;
-      const int32_t bi_hi = (e + start + a.B - 1) / a.B - fb;  // exclusive
-      if (s == 0) bi_lo = 0;
-      for (int32_t bi = max(bi_lo, 0); bi < bi_hi && bi < nblk; ++bi) {
+    const int32_t g0 = req_blk0[r];
+    // Block bi >= 1 starts at segment index (fb + bi) * B - start, block 0
+    // at 0; in a valid request every fact has a length >= 1, so seg[] rises
+    // strictly over [j0, j1).
+    if constexpr (SMEM) {
+      // Lanes over blocks: the block's first fact is the last j with seg[j]
+      // <= its first index (binary search in shared memory); a warp writes
+      // consecutive descriptors.
+      for (int32_t bi = lane; bi < nblk; bi += 32) {
+        const int32_t i0 = bi == 0 ? 0 : (fb + bi) * a.B - start;
+        int32_t lo = j0, hi = j1 - 1;  // seg[j0] = 0 <= i0
+        while (lo < hi) {
+          const int32_t mid = (lo + hi + 1) >> 1;
+          if (seg[mid] <= i0) lo = mid; else hi = mid - 1;
+        }
         BlockDesc d;
         d.r = r;
         d.b = fb + bi;
-        d.j = j;
+        d.j = lo;
         d.pad = 0;
         a.desc[g0 + bi] = d;
+      }
+    } else {
+      // Lanes over facts (no dependent L2 reads): fact j [s, e) owns the
+      // blocks whose first segment index lies in [s, e).
+      const int32_t S = req_len[r];
+      for (int32_t base = j0; base < j1; base += 32) {
+        const int32_t j = base + lane;
+        if (j >= j1) continue;
+        const int32_t s = seg[j];
+        const int32_t e = j + 1 < j1 ? seg[j + 1] : S;  // exclusive end
+        if (e == s) continue;
+        int32_t bi_lo = (s + start + a.B - 1) / a.B - fb;
+        const int32_t bi_hi = (e + start + a.B - 1) / a.B - fb;  // exclusive
+        if (s == 0) bi_lo = 0;
+        for (int32_t bi = max(bi_lo, 0); bi < bi_hi && bi < nblk; ++bi) {
+          BlockDesc d;
+          d.r = r;
+          d.b = fb + bi;
+          d.j = j;
+          d.pad = 0;
+          a.desc[g0 + bi] = d;
+        }
       }
     }
   }
@@ -534,14 +617,17 @@ struct UnitShared {
 // j is the CSR index of the first fact with a token in the block, seg[] the
 // facts' segment offsets (global or shared memory), j1 the end of the
 // request's CSR range, len_r its segment length, tok0 its first slot-mapping
-// index.  The slot mapping is written when write_slots.  Vector order inside
+// index.  The slot mapping is written when write_slots.  jfid / joff, when
+// given (shared memory), hold each CSR entry's fact id and store offset, so
+// the slot walk reads no global memory.  Vector order inside
 // a layer: split_vec.  Every thread of the CTA calls this with the same
 // arguments; the caller puts a barrier between units.
 template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER, int HC, int BC, bool FAST>
 __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TIER>& sm,
                                          float4* s_cs4, int r, int b, int j_first,
                                          const int32_t* seg, int j1, int start, int len_r,
-                                         long long tok0, int l0, int l1, bool write_slots) {
+                                         long long tok0, int l0, int l1, bool write_slots,
+                                         const int32_t* jfid = nullptr, const long long* joff = nullptr) {
   constexpr int VPR = D / 8;  // 16-byte vectors per head row
   constexpr int LOG_VPR = (VPR == 4) ? 2 : (VPR == 8) ? 3 : (VPR == 16) ? 4 : 5;
   const int tid = threadIdx.x;
@@ -575,9 +661,9 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
       const int i = blk_pos + o - start;  // segment index
       int j = j_first;
       while (j + 1 < j1 && seg[j + 1] <= i) ++j;
-      const int f = a.fact_ids[j];
+      const int f = jfid ? jfid[j] : a.fact_ids[j];
       const int t = i - seg[j];
-      src = a.fact_off[f] + t;
+      src = (joff ? joff[j] : a.fact_off[f]) + t;
       if (HOST_TIER && a.shard_k) {
         const int sh = a.fact_shard[f];
         s_kb[o] = a.shard_k[sh] + src * D;
@@ -822,6 +908,8 @@ constexpr int kSmallRequests = 8;
 constexpr int kSmallIds = 256;
 
 struct SmallPlan {
+  long long off[kSmallIds];    // store token offset per CSR entry (valid ids)
+  int32_t fid[kSmallIds];      // fact id per CSR entry
   int32_t len[kSmallIds];      // fact length per CSR entry, -1 for an id outside the store
   int32_t seg[kSmallIds];      // segment offset of each entry inside its request
   int32_t pref[kSmallIds + 1]; // exclusive prefix of valid lengths over the whole batch
@@ -863,8 +951,11 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   if (tid < num_ids) {
     const int32_t f = a.fact_ids[tid];
     const bool ok = f >= 0 && f < a.fact_len_count;
-    p.len[tid] = ok ? a.fact_len[f] : -1;
-    len = ok ? p.len[tid] : 0;
+    const int32_t lf = ok ? a.fact_len[f] : -1;
+    p.off[tid] = ok ? a.fact_off[f] : -1;
+    p.fid[tid] = f;
+    p.len[tid] = lf;
+    len = ok ? lf : 0;
   }
   int32_t x = len;
 #pragma unroll
@@ -947,7 +1038,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     const int l0 = lg * lpu;
     run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC, FAST>(a, sm, s_cs4, r, b, lo, p.seg, j1, start,
                                                  p.pref[j1] - p.pref[j0], p.pref[j0], l0,
-                                                 min(a.L, l0 + lpu), lg == 0);
+                                                 min(a.L, l0 + lpu), lg == 0, p.fid, p.off);
   }
 }
 

@@ -150,6 +150,26 @@ def test_ragged_batches_parity(shape, path):
     assert_parity(oracle_run(wl, style, hm), gpu_run(wl, style, hm, path=path))
 
 
+@pytest.mark.parametrize("R,k", [(1024, 2), (1025, 2), (9, 2048), (9, 2049)],
+                         ids=["1024-requests", "1025-requests", "16384-ids", "16392-ids"])
+def test_plan_in_shared_and_global_memory(R, k):
+    """The plan kernel keeps batches of at most 1024 requests and 16384 fact
+    ids in shared memory and runs larger ones on its global work space:
+    both sides of both limits, against the oracle."""
+    model = synth.Model("m", 1, 1, 32, 1e4)
+    rng = np.random.default_rng(R * 7 + k)
+    F = 64
+    fl = rng.integers(1, 4, F).astype(np.int32)
+    ids = [rng.integers(0, F, k) for _ in range(R)]
+    ids[1] = np.zeros(0, np.int64)
+    sp = rng.integers(0, 40, R).astype(np.int32)
+    need = max(-(-(int(sp[r]) + int(fl[ids[r]].sum())) // 16) for r in range(R)) + 1
+    batch = synth.make_batch(rng, ids, sp, 16, R * need, need)
+    wl = synth.Workload("plan-limits", model, fl, batch, R)
+    assert len(wl.batch.fact_ids) == k * (R - 1)
+    assert_parity(oracle_run(wl), gpu_run(wl, path="two-kernel"))
+
+
 @pytest.mark.parametrize("path", list(PATHS))
 def test_many_requests_many_ids(path):
     """Past the single-kernel limits (9 requests; 300 ids): the two-kernel
