@@ -344,6 +344,48 @@ def copy_probe(dev, elems: int = 1 << 30, reps: int = 10):
     return 2 * elems * 2 / (best / 1e3) / 1e9, sustained
 
 
+L2_BYTES = 126 * (1 << 20)
+
+
+class L2Flush:
+    """Writes a buffer twice the size of L2 on the launching stream, so the
+    next step's reads start from HBM (for steps whose reads fit in L2)."""
+
+    def __init__(self, dev):
+        import torch
+        self.buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def timed_steps(step, steps, stream, flush=None) -> float:
+    """Milliseconds of `steps` calls of step() on `stream`, CUDA events: one
+    pair around all of them back to back, or, with `flush`, a flush before
+    each step and a pair around each step alone (the flush not counted)."""
+    import torch
+    if flush is None:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
+    pairs = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        pairs.append((a, b))
+    pairs[-1][1].synchronize()
+    return sum(a.elapsed_time(b) for a, b in pairs)
+
+
 def h2d_probe(dev, nbytes: int = 1 << 30, reps: int = 5) -> float:
     """Pinned host -> device copy bandwidth (GB/s), CUDA events."""
     import torch
@@ -509,6 +551,78 @@ def run_offload(args, rank, world, local_rank):
     return 0
 
 
+SWEEP_R = (1, 16, 100, 256)
+SWEEP_K = (5, 10, 20, 50)
+
+
+def run_sweep(args, rank, world, local_rank):
+    """Every (R, k) point of the Mistral / Qwen sweep with one store: the
+    sweep's fact lengths come first from its seed, so every point draws from
+    the same pool.  One JSON line per point (rank 0; each rank runs the
+    grid on its own GPU as a replica).  Points whose reads fit in a few L2s
+    are timed step by step with an L2 flush between steps."""
+    import torch
+
+    from gpu_common import batch_tensors, make_cache, make_store
+    from kv_cache_injection_gather_b200 import binding as B
+    S = _synth()
+    if args.workload not in ("qwen-sweep", "mistral-sweep"):
+        raise SystemExit("--sweep is defined for qwen-sweep and mistral-sweep")
+    model, nf = (S.QWEN25_7B, 50_000) if args.workload == "qwen-sweep" else (S.MISTRAL_7B, 20_000)
+    dev = torch.device("cuda", local_rank)
+    base = S.sweep(model, 1, 5, rank, num_facts=nf)
+    store = make_store(base, on_device_gen=True, device=local_rank)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = hbm_peak()
+    flusher = L2Flush(dev)
+    for R in SWEEP_R:
+        for k in SWEEP_K:
+            wl = S.sweep(model, R, k, rank, num_facts=nf)
+            if not np.array_equal(wl.fact_lens, base.fact_lens):
+                raise RuntimeError("sweep points must share the fact pool")
+            kc, vc, desc = make_cache(wl, device=local_rank, fill=False)  # kc, vc live for the point
+            ro, ids, sp, bt = batch_tensors(wl.batch, local_rank)
+            n_tok = wl.tokens()
+            slots = torch.empty(max(n_tok, 1), dtype=torch.int64, device=dev)
+
+            def step():
+                store.inject(ro, ids, sp, bt, desc, slots[:n_tok], stream.cuda_stream)
+
+            for _ in range(args.warmup):
+                step()
+            rc, _ = store.last_error()
+            if rc != 0:
+                raise RuntimeError(f"sweep R={R} k={k}: {B.status_string(rc)}")
+            read_bytes = n_tok * model.bytes_per_token
+            flush = flusher if read_bytes < 4 * L2_BYTES else None
+            est_s = 2 * read_bytes / (peak * 1e9) + 15e-6
+            steps = int(min(2000, max(20, 0.3 / est_s)))
+            torch.cuda.synchronize(dev)
+            ms = timed_steps(step, steps, stream, flush)
+            store.set_timing(True)
+            store.kernel_time()
+            for _ in range(steps):
+                if flush is not None:
+                    flush()
+                step()
+            kern_ms, kern_n = store.kernel_time()
+            store.set_timing(False)
+            kern = kern_ms / max(kern_n, 1)
+            if rank == 0:
+                print(json.dumps({
+                    "metric": METRIC, "workload": WORKLOADS[args.workload][0].split(",")[0],
+                    "model_shapes": model.name, "requests": R, "k": k, "tokens_per_batch": n_tok,
+                    "steps": steps, "l2": "flushed before every step" if flush else "reads > 4x L2",
+                    "us_per_batch": ms / steps * 1e3, "tokens_per_s": n_tok / (ms / steps / 1e3),
+                    "kernel_us": kern * 1e3,
+                    "kernel_frac_of_peak": 2 * read_bytes / (kern / 1e3) / 1e9 / peak,
+                    "peak_gbs": peak, "peak_source": f"{peak_kind} hbm_gbs"}), flush=True)
+            del kc, vc, desc, slots
+            torch.cuda.empty_cache()
+    store.close()
+    return 0
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -522,6 +636,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     if args.workload == "offload":
         return run_offload(args, rank, world, local_rank)
+    if args.sweep:
+        return run_sweep(args, rank, world, local_rank)
     extra_cfg = {}
     heads = None
     owner = None
@@ -585,19 +701,21 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
+    # Steps whose reads fit in a few L2s would re-read cached rows: flush L2
+    # before each of them and time each step alone.
+    read_bytes = n_tok * m.bytes_per_token
+    flush = L2Flush(dev) if read_bytes < 4 * L2_BYTES else None
+    if flush is not None:
+        extra_cfg["l2"] = (f"flushed before every step (a {2 * L2_BYTES >> 20} MiB write, not timed): "
+                           f"{read_bytes / 1e6:.1f} MB read per step, L2 126 MB")
+
     clocks = ClockSampler(gpu_id(dev, local_rank))
     # ---- device-resident timed region (the value)
     barrier()
     clocks.start()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step()
-    t1.record(stream)
+    ms = timed_steps(step, args.steps, stream, flush)
     barrier()
     clk = clocks.stop()
-    ms = t0.elapsed_time(t1)
     rc, _ = store.last_error()
     if rc != 0:
         raise RuntimeError(f"inject failed: {B.status_string(rc)}")
@@ -608,6 +726,8 @@ def run_ours(args, rank, world, local_rank):
     store.kernel_time()  # reset
     barrier()
     for _ in range(args.steps):
+        if flush is not None:
+            flush()
         step()
     barrier()
     kern_ms, kern_n = store.kernel_time()
@@ -623,16 +743,14 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(max(1, args.warmup // 2)):
         store.inject_host(h_ro, h_ids, h_sp, h_bt, desc, h_slots, stream.cuda_stream)
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+
+    def host_step():
         rc = store.inject_host(h_ro, h_ids, h_sp, h_bt, desc, h_slots, stream.cuda_stream)
         if rc != 0:
             raise RuntimeError(f"inject_host failed: {B.status_string(rc)}")
-    e1.record(stream)
+
+    e2e_ms = timed_steps(host_step, args.steps, stream, flush)
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
 
     # ---- max over ranks
     ms, e2e_ms, kern_avg_ms = max_over_ranks([ms, e2e_ms, kern_ms / max(kern_n, 1)], world)
@@ -712,6 +830,9 @@ def main():
                          "batch of 100 x N requests (both weak scaling, no collective), or fact "
                          "shards (each rank holds 1/N of the facts and injects 100 requests, "
                          "reading the rest from peers over NVLink)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="qwen-sweep / mistral-sweep: every point of R in {1, 16, 100, 256} x k in "
+                         "{5, 10, 20, 50} with one store, one JSON line per point")
     ap.add_argument("--head-major", action="store_true",
                     help="cache layout [L][num_blocks][H][B][D] instead of [L][num_blocks][B][H][D]")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama-batch",

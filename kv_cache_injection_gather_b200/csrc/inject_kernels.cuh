@@ -34,6 +34,17 @@
 #ifndef IS_UNITS_PER_CTA
 #define IS_UNITS_PER_CTA 256
 #endif
+// Smallest (layer, head) row count of a work unit of a large batch, and the
+// larger count used when it still leaves IS_UNITS_PER_CTA_MIN units per CTA.
+#ifndef IS_UNIT_MIN_ROWS
+#define IS_UNIT_MIN_ROWS 16
+#endif
+#ifndef IS_UNIT_ROWS_LARGE
+#define IS_UNIT_ROWS_LARGE 32
+#endif
+#ifndef IS_UNITS_PER_CTA_MIN
+#define IS_UNITS_PER_CTA_MIN 32
+#endif
 // 1: the copy loop keeps two half-chunks in flight (software pipeline).
 #ifndef IS_PIPELINE
 #define IS_PIPELINE 1
@@ -87,10 +98,15 @@ __device__ __forceinline__ void record_error(DevStatus* st, int32_t code, long l
 // per unit that fit one wave (one layer when they already do): everything is
 // in flight at once and no CTA runs a second unit after the first (latency).
 // Larger batches aim at ~IS_UNITS_PER_CTA units per CTA, so the dynamic
-// schedule's tail (at most one unit) stays short, with at least two layers
-// per unit so a unit's set-up (slot walk, cos/sin table) is shared by more
-// than one layer.
-__device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32_t grid_ctas,
+// schedule's tail (at most one unit) stays short, with at least
+// IS_UNIT_MIN_ROWS (layer, head) rows per unit (and at least two layers) so
+// a unit's set-up (slot walk, cos/sin table, barriers) is shared by enough
+// copies, and IS_UNIT_ROWS_LARGE rows when the batch still has
+// IS_UNITS_PER_CTA_MIN units per CTA with them.  Measured on B200 over the
+// Mistral/Qwen sweep grid: with H = 4, two-layer units ran at 0.87 of the
+// copy peak, 16-row units at 0.93-0.96, 32-row units up to 0.97 on large
+// batches but slower where they leave few units per CTA.
+__device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32_t H, int32_t grid_ctas,
                                           int32_t& lpu, int32_t& upb) {
   const long long grid = grid_ctas;
   upb = 1;
@@ -98,8 +114,14 @@ __device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32
     const long long per = ((long long)total_blocks * L + grid - 1) / grid;  // 1 or 2 layers per unit
     upb = int32_t((L + per - 1) / per);
   } else if (total_blocks > 0) {
+    const int32_t h = max(H, 1);
+    const int32_t lmin = min(L, max(2, (IS_UNIT_MIN_ROWS + h - 1) / h));
+    const int32_t lbig = min(L, max(2, (IS_UNIT_ROWS_LARGE + h - 1) / h));
+    const long long cap_big = max(1, L / lbig);
+    const long long cap = (long long)total_blocks * cap_big >= IS_UNITS_PER_CTA_MIN * grid
+                              ? cap_big : (long long)max(1, L / lmin);
     const long long want = (grid * IS_UNITS_PER_CTA + total_blocks - 1) / total_blocks;
-    upb = int32_t(max(1LL, min(want, (long long)max(1, L / 2))));
+    upb = int32_t(max(1LL, min(want, cap)));
   }
   lpu = (L + upb - 1) / upb;
   upb = (L + lpu - 1) / lpu;
@@ -114,6 +136,7 @@ struct PlanArgs {
   int32_t max_blocks;
   int32_t B;
   int32_t L;
+  int32_t H;
   const int32_t* fact_len;   // store: [num_facts]
   int32_t num_facts;
   int64_t* slot_out;         // optional
@@ -318,7 +341,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
 
   if (tid == 0) {
     int32_t lpu, upb;
-    unit_size(total_blocks, a.L, a.grid_ctas, lpu, upb);
+    unit_size(total_blocks, a.L, a.H, a.grid_ctas, lpu, upb);
     a.hdr->layers_per_unit = lpu;
     a.hdr->units_per_block = upb;
     a.hdr->total_blocks = total_blocks;
@@ -992,7 +1015,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     // which path a batch takes
     const bool over = (a.slot_out != nullptr && total_tokens > slot_cap) || acc > max_batch_blocks;
     int32_t lpu, upb;
-    unit_size(acc, a.L, grid_ctas, lpu, upb);
+    unit_size(acc, a.L, a.H, grid_ctas, lpu, upb);
     p.lpu = lpu;
     p.total_blocks = acc;
     p.total_units = over ? 0 : acc * upb;

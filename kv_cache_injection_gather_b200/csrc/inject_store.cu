@@ -896,6 +896,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.max_blocks = max_blocks_per_req;
   pa.B = c.block_size;
   pa.L = cf.num_layers;
+  pa.H = cf.num_kv_heads;
   // With a sharded view attached, ids are global: the view's fact table.
   const bool view = s->shard_n > 0;
   const int32_t nfacts = view ? s->shard_facts : s->num_facts;
@@ -1266,6 +1267,7 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   pa.max_blocks = max_blocks_per_req;
   pa.B = k.block_size;
   pa.L = c.num_layers;
+  pa.H = c.num_kv_heads;
   pa.fact_len = fact_lens;
   pa.num_facts = num_facts;
   pa.slot_out = slot_out;
