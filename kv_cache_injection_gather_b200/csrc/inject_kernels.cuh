@@ -625,9 +625,12 @@ __device__ __forceinline__ void split_vec(int rem, int order, const Divisor<POW2
   }
 }
 
+constexpr int kMaxHalfDim = 128;  // D / 2 for the largest head_dim (256)
+
 // Shared-memory state of a CTA of the inject kernels, reused unit after unit.
 template <bool HOST_TIER>
 struct UnitShared {
+  double inv_freq[kMaxHalfDim];  // the store's RoPE frequencies, loaded once per CTA
   long long src[kMaxBlockSize];  // store token of each in-block slot (-1: none)
   // per-slot sources (host tier, sharded view): K/V row bases (token offset
   // applied) and plane stride
@@ -708,16 +711,17 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
     }
     s_src[o] = src;
   }
-  if (!phys_ok) {
-    if (tid == 0 && write_slots) record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
-    return;  // uniform; the caller's barrier follows
-  }
-  // cos/sin of every (slot, frequency): fp64 angle and sincos, kept fp32.
+  // cos/sin of every (slot, frequency): fp64 angle and sincos, kept fp32
+  // (computed before the block-table entry is checked, so its load overlaps).
   for (int e = tid; e < B * (D / 2); e += NT) {
     const int o = e / (D / 2), i = e % (D / 2);
     double sn, cn;
-    sincos(double(blk_pos + o) * a.inv_freq[i], &sn, &cn);
+    sincos(double(blk_pos + o) * sm.inv_freq[i], &sn, &cn);
     reinterpret_cast<float2*>(s_cs4)[cs_index<D, STYLE>(o, i)] = make_float2(float(cn), float(sn));
+  }
+  if (!phys_ok) {
+    if (tid == 0 && write_slots) record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
+    return;  // uniform; the caller's barrier follows
   }
   __syncthreads();
 
@@ -890,6 +894,7 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   __shared__ int s_unit;
 
   const int tid = threadIdx.x;
+  for (int i = tid; i < D / 2; i += NT) sm.inv_freq[i] = a.inv_freq[i];  // store data, not the plan's
   // When launched as a programmatic dependent of the plan kernel, wait here
   // for its results; without such a launch this returns at once.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -957,10 +962,14 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool reporter = blockIdx.x == 0;
 
-  // CSR: starts at 0, ends at num_ids, never decreases.
+  // Everything the plan reads from the caller is loaded at once: the CSR,
+  // the starts, the ids (then their lengths and offsets) and the frequencies.
+  const int32_t fid = tid < num_ids ? a.fact_ids[tid] : -1;
   if (tid <= R) p.roff[tid] = a.req_off[tid];
   if (tid < R) p.start[tid] = a.start_pos[tid];
+  for (int i = tid; i < D / 2; i += NT) sm.inv_freq[i] = a.inv_freq[i];
   if (tid == 0) p.bad = 0;
+  // CSR: starts at 0, ends at num_ids, never decreases.
   __syncthreads();
   if ((tid < R && p.roff[tid + 1] < p.roff[tid]) || (tid == 0 && (p.roff[0] != 0 || p.roff[R] != num_ids)))
     p.bad = 1;
@@ -972,7 +981,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   // Lengths, and their exclusive prefix over the batch (invalid ids count 0).
   int32_t len = 0;
   if (tid < num_ids) {
-    const int32_t f = a.fact_ids[tid];
+    const int32_t f = fid;
     const bool ok = f >= 0 && f < a.fact_len_count;
     const int32_t lf = ok ? a.fact_len[f] : -1;
     p.off[tid] = ok ? a.fact_off[f] : -1;
