@@ -211,7 +211,7 @@ void free_store(is_store* s) {
 
 bool head_dim_supported(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
 
-template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0, bool FAST = false>
+template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0, int FAST = 0>
 void* inject_fn() {
   return reinterpret_cast<void*>(&isk::inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread,
                                                      kInjectMinBlocks, POW2, HOST_TIER, HC, BC, FAST>);
@@ -219,7 +219,7 @@ void* inject_fn() {
 
 
 
-template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0, bool FAST = false>
+template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0, int FAST = 0>
 void* small_fn() {
   return reinterpret_cast<void*>(&isk::small_inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread,
                                                            kInjectMinBlocks, POW2, HOST_TIER, HC, BC, FAST>);
@@ -239,24 +239,32 @@ void* pick_small_t(int D, int style) {
 // Compile-time shapes for the common models (D = 128, block size 16, 4 or 8
 // KV heads: Llama-3.1-8B, Mistral-7B, Qwen2.5-7B): the per-vector index
 // arithmetic folds to constants.  Returns nullptr for other shapes.
-template <bool SMALL, bool HOST_TIER, int HC, bool FAST>
+template <bool SMALL, bool HOST_TIER, int HC, int FAST>
 void* fixed_fn(int style) {
-  return SMALL ? (style ? small_fn<128, 1, true, HOST_TIER, HC, 16, FAST>()
+  return SMALL ? (style ? small_fn<128, 1, true, HOST_TIER, HC, 16, (FAST == 2 ? 1 : FAST)>()
                         : small_fn<128, 0, true, HOST_TIER, HC, 16, FAST>())
-               : (style ? inject_fn<128, 1, true, HOST_TIER, HC, 16, FAST>()
+               : (style ? inject_fn<128, 1, true, HOST_TIER, HC, 16, (FAST == 2 ? 1 : FAST)>()
                         : inject_fn<128, 0, true, HOST_TIER, HC, 16, FAST>());
 }
 
-// order: the launch's vector order (1: slot-fastest, the FAST copy loop).
+// loop: the copy loop of the launch -- 0 generic, 1 per-thread, 2 per-thread
+// with both rotate-half halves in one thread (device tier, rotate-half only;
+// other cases fall back to 1).
 template <bool SMALL, bool HOST_TIER>
-void* pick_fixed(int D, int style, int H, int B, int order) {
+void* pick_fixed(int D, int style, int H, int B, int loop) {
 #ifndef IS_NO_FIXED_SHAPES
   if (D != 128 || B != 16) return nullptr;
-  const bool fast = order == 1;
-  if (H == 8) return fast ? fixed_fn<SMALL, HOST_TIER, 8, true>(style) : fixed_fn<SMALL, HOST_TIER, 8, false>(style);
-  if (H == 4) return fast ? fixed_fn<SMALL, HOST_TIER, 4, true>(style) : fixed_fn<SMALL, HOST_TIER, 4, false>(style);
+  if (loop == 2 && (HOST_TIER || style != 0)) loop = 1;
+  if (H == 8)
+    return loop == 2 ? fixed_fn<SMALL, HOST_TIER, 8, (HOST_TIER ? 1 : 2)>(style)
+         : loop == 1 ? fixed_fn<SMALL, HOST_TIER, 8, 1>(style)
+                     : fixed_fn<SMALL, HOST_TIER, 8, 0>(style);
+  if (H == 4)
+    return loop == 2 ? fixed_fn<SMALL, HOST_TIER, 4, (HOST_TIER ? 1 : 2)>(style)
+         : loop == 1 ? fixed_fn<SMALL, HOST_TIER, 4, 1>(style)
+                     : fixed_fn<SMALL, HOST_TIER, 4, 0>(style);
 #else
-  (void)D; (void)style; (void)H; (void)B; (void)order;
+  (void)D; (void)style; (void)H; (void)B; (void)loop;
 #endif
   return nullptr;
 }
@@ -277,8 +285,8 @@ bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 // The inject kernel for a head dim, RoPE style and (H, B): the shift variant
 // when both are powers of two; the host-tier variant for stores in pinned
 // host memory.
-void* pick_inject(int D, int style, int H, int B, bool host_tier = false, int order = 0) {
-  if (void* f = host_tier ? pick_fixed<false, true>(D, style, H, B, order) : pick_fixed<false, false>(D, style, H, B, order))
+void* pick_inject(int D, int style, int H, int B, bool host_tier = false, int loop = 0) {
+  if (void* f = host_tier ? pick_fixed<false, true>(D, style, H, B, loop) : pick_fixed<false, false>(D, style, H, B, loop))
     return f;
   const bool p2 = is_pow2(H) && is_pow2(B);
   if (host_tier) return p2 ? pick_inject_t<true, true>(D, style) : pick_inject_t<false, true>(D, style);
@@ -286,8 +294,8 @@ void* pick_inject(int D, int style, int H, int B, bool host_tier = false, int or
 }
 
 // The single-kernel variant for small batches, same selection.
-void* pick_small(int D, int style, int H, int B, bool host_tier, int order) {
-  if (void* f = host_tier ? pick_fixed<true, true>(D, style, H, B, order) : pick_fixed<true, false>(D, style, H, B, order))
+void* pick_small(int D, int style, int H, int B, bool host_tier, int loop) {
+  if (void* f = host_tier ? pick_fixed<true, true>(D, style, H, B, loop) : pick_fixed<true, false>(D, style, H, B, loop))
     return f;
   const bool p2 = is_pow2(H) && is_pow2(B);
   if (host_tier) return p2 ? pick_small_t<true, true>(D, style) : pick_small_t<false, true>(D, style);
@@ -335,6 +343,21 @@ int vec_order_for(int64_t token_stride, int64_t head_stride) { return token_stri
 // the generic loop on the benchmark batch and lifts the small case from
 // 0.952 to 0.991 of the copy peak); other shapes take the order whose
 // fastest row index has the larger cache stride.
+// Copy loop of a batch launch (see pick_fixed): the fixed shapes take the
+// per-thread loop; on a head-major cache (head stride above the token stride)
+// the paired rotate-half loop, whose CTA writes two heads' rows at once
+// (B200, Llama-3.1-8B-shaped batch on the head-major cache: 0.967 -> 0.987 of
+// the copy peak; on the token-major cache it was level on the benchmark
+// batch and 0.7% slower on the small case, so that layout keeps loop 1).
+int launch_loop(int D, int B, int H, int64_t token_stride, int64_t head_stride) {
+#ifndef IS_NO_FIXED_SHAPES
+  if (D == 128 && B == 16 && (H == 4 || H == 8)) return head_stride > token_stride ? 2 : 1;
+#else
+  (void)D; (void)B; (void)H; (void)token_stride; (void)head_stride;
+#endif
+  return 0;
+}
+
 int launch_vec_order(int D, int B, int H, int64_t token_stride, int64_t head_stride) {
 #ifndef IS_NO_FIXED_SHAPES
   if (D == 128 && B == 16 && (H == 4 || H == 8)) return 1;
@@ -464,11 +487,11 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                        int(isk::plan_smem_bytes(isk::kPlanSmemRequests, isk::kPlanSmemIds)));
   for (int h : {4, 8})
-    for (int order : {0, 1})
-      for (void* f : {pick_fixed<false, false>(c.head_dim, c.rope_style, h, 16, order),
-                      pick_fixed<false, true>(c.head_dim, c.rope_style, h, 16, order),
-                      pick_fixed<true, false>(c.head_dim, c.rope_style, h, 16, order),
-                      pick_fixed<true, true>(c.head_dim, c.rope_style, h, 16, order)})
+    for (int loop : {0, 1, 2})
+      for (void* f : {pick_fixed<false, false>(c.head_dim, c.rope_style, h, 16, loop),
+                      pick_fixed<false, true>(c.head_dim, c.rope_style, h, 16, loop),
+                      pick_fixed<true, false>(c.head_dim, c.rope_style, h, 16, loop),
+                      pick_fixed<true, true>(c.head_dim, c.rope_style, h, 16, loop)})
         if (f) cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
   void* fn = pick_inject_t<true>(c.head_dim, c.rope_style);
   int per_sm = 0;
@@ -963,9 +986,9 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.fact_len_count = nfacts;
   // Per-slot sources: the host tier, or the arenas of a sharded view.
   const bool per_slot = s->host_arena || view;
-  void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, ia.vec_order)
-                   : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot,
-                                 ia.vec_order);
+  const int loop = launch_loop(cf.head_dim, c.block_size, cf.num_kv_heads, c.token_stride, c.head_stride);
+  void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop)
+                   : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop);
   int32_t small_R = R, small_ids = num_ids, small_grid = s->inject_grid, small_blocks = s->max_blocks;
   int64_t small_cap = slot_cap;
   void* small_args[] = {&ia, &small_R, &small_ids, &small_cap, &small_grid, &small_blocks};
@@ -1314,7 +1337,8 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   ia.desc = pa.desc;
   ia.hdr = hdr;
   ia.st = status;
-  void* fn = pick_inject(c.head_dim, c.rope_style, c.num_kv_heads, k.block_size, false, ia.vec_order);
+  void* fn = pick_inject(c.head_dim, c.rope_style, c.num_kv_heads, k.block_size, false,
+                         ia.vec_order);  // loop 1 (per-thread) on slot-fastest orders, else 0
   void* args[] = {&ia};
   if (cudaLaunchKernel(fn, dim3(unsigned(grid)), dim3(kInjectThreads), args,
                        cs_smem_bytes(c.head_dim, k.block_size), st) != cudaSuccess)
