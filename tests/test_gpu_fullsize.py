@@ -1,9 +1,10 @@
 """Full-size parity on the benchmark's workload, in the benchmark's launch
 configuration: Llama-3.1-8B shapes (32 layers, 8 KV heads, D=128, llama3
 RoPE scaling), 10k facts of 16-64 tokens (about 52 GB of store), 100
-requests x k=50 distinct facts after a 64-token prefix, 25 600-block cache.
+requests x k=50 distinct facts after a 64-token prefix, 25 600-block cache
+(53.7 GB of K and V), token-major and head-major.
 
-The oracle cannot hold the 107 GB cache, so:
+The oracle cannot hold the cache, so:
   * slot mapping: every token, against the oracle's segment composition;
   * V: every row of every token, compared on the device with the store row
     the oracle's composition names (bit-exact);
@@ -36,7 +37,8 @@ def _lengths_store(wl):
     return st
 
 
-def test_llama_batch_full_size():
+@pytest.fixture(scope="module")
+def llama_store():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     free, _ = torch.cuda.mem_get_info()
@@ -46,7 +48,15 @@ def test_llama_batch_full_size():
     if free < need + (8 << 30):
         pytest.skip(f"needs {need / 1e9:.0f} GB free on the device")
     store = make_store(wl, on_device_gen=True)
-    k, v, desc = make_cache(wl)
+    yield wl, store
+    store.close()
+
+
+@pytest.mark.parametrize("head_major", [False, True], ids=["token-major", "head-major"])
+def test_llama_batch_full_size(llama_store, head_major):
+    wl, store = llama_store
+    m, b = wl.model, wl.batch
+    k, v, desc = make_cache(wl, head_major=head_major)
     ro, ids, sp, bt = batch_tensors(b)
     n_tok = wl.tokens()
     slots = torch.empty(n_tok, dtype=torch.int64, device="cuda")
@@ -62,14 +72,22 @@ def test_llama_batch_full_size():
         assert store.fact_info(f)[0] == int(np.concatenate([[0], np.cumsum(wl.fact_lens)])[f])
 
     L, H, D, NB, Bs = m.num_layers, m.num_kv_heads, m.head_dim, b.num_blocks, b.block_size
+    shape5 = (L, NB, H, Bs, D) if head_major else (L, NB, Bs, H, D)
+    k5, v5 = k.view(shape5), v.view(shape5)
+
+    def slot_rows(t5, blk, o):  # rows of the given slots, all layers and heads: [L][n][H][D]
+        return t5[:, blk, :, o].permute(1, 0, 2, 3) if head_major else t5[:, blk, o]
+
+    def layer_by_slot(t4):  # one layer as [NB][Bs][H][D] (a view)
+        return t4.permute(0, 2, 1, 3) if head_major else t4
+
     ka, va = store.arena()
-    kc = k.view(L, NB * Bs, H, D)
-    vc = v.view(L, NB * Bs, H, D)
     slot_d = torch.from_numpy(seg["slot"]).cuda()
     src_d = torch.from_numpy(seg["src"]).cuda()
     for a in range(0, n_tok, 8192):
         s_, t_ = slot_d[a:a + 8192], src_d[a:a + 8192]
-        assert torch.equal(vc[:, s_], va[:, :, t_].permute(0, 2, 1, 3)), f"V rows at {a}"
+        got_v = slot_rows(v5, s_ // Bs, s_ % Bs)
+        assert torch.equal(got_v, va[:, :, t_].permute(0, 2, 1, 3)), f"V rows at {a}"
 
     # K: one whole request plus random rows
     f = oracle.rope_inv_freq(D, m.rope_theta, m.scaling())
@@ -81,8 +99,9 @@ def test_llama_batch_full_size():
     toks = np.concatenate([np.repeat(np.arange(r0, r1), L * H), rng.integers(0, n_tok, 20000)])
     ls = np.concatenate([np.tile(np.repeat(np.arange(L), H), r1 - r0), rng.integers(0, L, 20000)])
     hs = np.concatenate([np.tile(np.tile(np.arange(H), L), r1 - r0), rng.integers(0, H, 20000)])
-    got = to_bits(kc[torch.from_numpy(ls).cuda(), slot_d[torch.from_numpy(toks).cuda()],
-                     torch.from_numpy(hs).cuda()])
+    sl = slot_d[torch.from_numpy(toks).cuda()]
+    l_d, h_d = torch.from_numpy(ls).cuda(), torch.from_numpy(hs).cuda()
+    got = to_bits(k5[l_d, sl // Bs, h_d, sl % Bs] if head_major else k5[l_d, sl // Bs, sl % Bs, h_d])
     for fid in np.unique(tok_fact[toks]):
         sel = tok_fact[toks] == fid
         x = synth.fact_rows(wl.seed, int(fid), False, L, H, int(wl.fact_lens[fid]), D,
@@ -94,15 +113,16 @@ def test_llama_batch_full_size():
     # untouched slots keep the seeded pre-fill
     touched = torch.zeros(NB * Bs, dtype=torch.bool, device="cuda")
     touched[slot_d] = True
-    untouched = ~touched
+    untouched = (~touched).view(NB, Bs)
     per_layer = NB * Bs * H * D
     buf = torch.empty(per_layer, dtype=torch.int16, device="cuda")
     cs = torch.cuda.current_stream().cuda_stream
-    for tens, tag in ((kc, 0), (vc, 1)):
+    for t5, tag in ((k5, 0), (v5, 1)):
         for l in range(L):
             synth.fill_device(buf.data_ptr(), per_layer, CACHE_FILL_SEED, synth.TAG_CACHE | tag,
                               l * per_layer, cs)
-            want = buf.view(NB * Bs, H, D)[untouched]
-            have = tens[l].view(torch.int16)[untouched]
+            want = layer_by_slot(buf.view(shape5[1:]))[untouched]
+            have = layer_by_slot(t5[l].view(torch.int16))[untouched]
             assert torch.equal(have, want), f"untouched slots changed (tensor {tag}, layer {l})"
-    store.close()
+    del k, v, k5, v5
+    torch.cuda.empty_cache()

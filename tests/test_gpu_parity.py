@@ -132,6 +132,7 @@ SHAPES = [
     ("qwen-like", 2, 4, 128, 1e6, False, 16, 0, False),
     ("interleaved", 2, 4, 128, 1e4, False, 16, 1, False),
     ("head-major", 2, 8, 128, 5e5, True, 16, 0, True),
+    ("qwen-head-major", 3, 4, 128, 1e6, False, 16, 0, True),
     ("h3-generic", 2, 3, 128, 1e4, False, 16, 0, False),
     ("d64-b8", 2, 2, 64, 1e4, False, 8, 0, False),
     ("d256-b32", 1, 2, 256, 1e4, False, 32, 1, False),
