@@ -258,8 +258,10 @@ def workload_config(wl, name="llama-batch", extra=None):
            "store_gb": round(float(wl.fact_lens.sum()) * m.bytes_per_token / 1e9, 2),
            "tokens_per_batch": wl.tokens(), "block_size": b.block_size,
            "num_blocks": b.num_blocks, "start_pos": 64,
-           "l2": f"inputs larger than L2 ({wl.tokens() * m.bytes_per_token / 1e9:.1f} GB read + "
-                 f"the same written per step, L2 126 MB)"}
+           "l2": (f"inputs larger than L2 ({wl.tokens() * m.bytes_per_token / 1e9:.1f} GB read + "
+                  f"the same written per step, L2 126 MB)"
+                  if wl.tokens() * m.bytes_per_token >= 4 * L2_BYTES else
+                  f"{wl.tokens() * m.bytes_per_token / 1e6:.1f} MB read per step, L2 126 MB")}
     if extra:
         cfg.update(extra)
     return cfg

@@ -1,0 +1,79 @@
+"""The benchmark's command-line contract, checked on CPU: the reference arm
+(the CPU oracle) prints one JSON line with the keys the driver reads, only
+rank 0 prints under torchrun, too few warm-up steps are refused, and the
+GPU arm fails loudly without a CUDA device (no CPU fallback)."""
+from __future__ import annotations
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+BASE = [sys.executable, os.path.join(ROOT, "bench.py")]
+REF = ["--impl", "reference", "--steps", "1", "--warmup", "3", "--workload", "llama-single"]
+
+
+def _run(args, **kw):
+    return subprocess.run(args, cwd=ROOT, capture_output=True, text=True, timeout=300, **kw)
+
+
+def _json_lines(out: str):
+    return [json.loads(line) for line in out.splitlines() if line.startswith("{")]
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def test_reference_arm_prints_the_contract_line():
+    r = _run(BASE + REF)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1
+    d = lines[0]
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert "workload" in d["config"] and d["data"] == "synthetic"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    e = d["e2e"]
+    assert e["value"] == d["value"] and e["unit"] == d["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+@pytest.mark.timeout(300)
+def test_reference_arm_under_torchrun_prints_once():
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1")
+    r = _run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+              "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+              os.path.join(ROOT, "bench.py"), "--gpus", "2"] + REF, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1 and lines[0]["impl"] == "reference"
+
+
+def test_too_few_warmup_steps_are_refused():
+    r = _run(BASE + ["--impl", "reference", "--steps", "1", "--warmup", "2"])
+    assert r.returncode != 0 and "warmup" in (r.stderr + r.stdout)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_gpu_arm_fails_loudly_without_a_gpu():
+    r = _run(BASE + ["--steps", "1", "--warmup", "3", "--workload", "llama-single",
+                     "--no-cpu-baseline"])
+    assert r.returncode != 0
+    assert "CUDA device" in (r.stderr + r.stdout)
+    assert not _json_lines(r.stdout)
