@@ -228,6 +228,9 @@ WORKLOADS = {
                                                             slots_per_request=1024)),
     "llama-single": ("llama3.1-8b-shapes 10k-fact store, 1 request x k=5, block 16, 64 blocks",
                      lambda seed: _synth().llama_single(seed)),
+    "llama-single-small": ("llama3.1-8b-shapes 500-fact store, 1 request x k=5, block 16, 64 blocks "
+                           "(profiling case of the single request, ~2.7 GB on the device)",
+                           lambda seed: _synth().llama_single(seed, num_facts=500)),
     "offload": ("qwen2.5-7b-shapes store of 16..48-token facts in pinned host memory, HBM hot "
                 "set = top 20% by Zipf rank, 100 requests x k=50 drawn Zipf(1.1), block 16",
                 lambda seed, n=100_000: _synth().offload(seed, num_facts=n, extra_batches=7)),

@@ -649,6 +649,20 @@ __device__ __forceinline__ uint4 rotate_vec(const uint4 own, int c, const float4
   return rotate_regs<D, STYLE>(own, c, t);
 }
 
+// cos and sin of an fp64 RoPE angle: reduced to [-pi, pi] by the nearest
+// multiple of 2*pi (one fused multiply-add in fp64; for positions below 2^31
+// the reduction is off by < 1e-7 rad, the fp64 angle itself by < 3e-7 rad),
+// then the hardware single-precision sin/cos of the reduced angle (absolute
+// error below 2^-21.4 on [-pi, pi]; the values are kept in fp32 anyway).  The
+// hardware form is used only on the reduced angle: on the raw angle (up to
+// ~2e9 rad) it would be far off.
+__device__ __forceinline__ void rope_cos_sin(double ang, float& c, float& s) {
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+  const double k = rint(ang * kInvTwoPi);
+  __sincosf(float(fma(-k, kTwoPi, ang)), &s, &c);
+}
+
 constexpr int kMaxBlockSize = 128;
 
 // x / d and x % d for a divisor fixed per launch: shifts when d is a power
@@ -773,19 +787,29 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
     }
     s_src[o] = src;
   }
-  // cos/sin of every (slot, frequency): fp64 angle and sincos, kept fp32
-  // (computed before the block-table entry is checked, so its load overlaps).
-  for (int e = tid; e < B * (D / 2); e += NT) {
-    const int o = e / (D / 2), i = e % (D / 2);
-    double sn, cn;
-    sincos(double(blk_pos + o) * sm.inv_freq[i], &sn, &cn);
-    reinterpret_cast<float2*>(s_cs4)[cs_index<D, STYLE>(o, i)] = make_float2(float(cn), float(sn));
-  }
-  if (!phys_ok) {
+  // cos/sin of every (slot, frequency) of the block: fp64 angle, fp32 values.
+  auto fill_cs = [&]() {
+    for (int e = tid; e < B * (D / 2); e += NT) {
+      const int o = e / (D / 2), i = e % (D / 2);
+      float cn, sn;
+      rope_cos_sin(double(blk_pos + o) * sm.inv_freq[i], cn, sn);
+      reinterpret_cast<float2*>(s_cs4)[cs_index<D, STYLE>(o, i)] = make_float2(cn, sn);
+    }
+  };
+  // A block-table entry outside the cache: nothing is stored (uniform; the
+  // caller's barrier follows).
+  auto bad_block = [&]() {
     if (tid == 0 && write_slots) record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
-    return;  // uniform; the caller's barrier follows
+  };
+  if constexpr (FAST == 0) {
+    fill_cs();  // before the block-table entry is checked, so its load overlaps
+    if (!phys_ok) return bad_block();
+    __syncthreads();
+  } else {
+    // The per-thread loops issue their first loads (which need only the
+    // slots' sources), then fill the table while those loads are in flight.
+    __syncthreads();
   }
-  __syncthreads();
 
   // FAST: compile-time H and B with one head's block row of vectors (B * D/8)
   // equal to the CTA, slot-fastest rows (token-major cache; the launch picks
@@ -811,8 +835,7 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
     const int o = (tid % (NT / 2)) / VH, c = tid % VH;
     const long long src = s_src[o];
     const bool act = src >= 0;
-    CsPairs cp;
-    load_cs_pairs<D>(s_cs4 + o * (D / 4), c, cp);
+    CsPairs cp;  // loaded once the table is filled
     const long long pl = a.plane;
     const uint16_t* kp = a.k_store + (act ? src : 0) * D + c * 8 + (long long)(l0 * HC + rp) * pl;
     const uint16_t* vp = a.v_store + (act ? src : 0) * D + c * 8 + (long long)(l0 * HC + rp) * pl;
@@ -854,6 +877,10 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
 #if IS_PIPELINE
     uint4 k0[HR], k1[HR], v0[HR], v1[HR], k2[HR], k3[HR], v2[HR], v3[HR];
     if (nr > 0) load_r(k0, k1, v0, v1, 0);
+    fill_cs();
+    __syncthreads();
+    if (!phys_ok) return bad_block();
+    load_cs_pairs<D>(s_cs4 + o * (D / 4), c, cp);
     for (int i0 = 0; i0 < nr; i0 += 2 * HR) {
       if (i0 + HR < nr) load_r(k2, k3, v2, v3, i0 + HR);
       store_r(k0, k1, v0, v1, i0);
@@ -862,6 +889,10 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
       store_r(k2, k3, v2, v3, i0 + HR);
     }
 #else
+    fill_cs();
+    __syncthreads();
+    if (!phys_ok) return bad_block();
+    load_cs_pairs<D>(s_cs4 + o * (D / 4), c, cp);
     for (int i0 = 0; i0 < nr; i0 += HR) {
       uint4 k0[HR], k1[HR], v0[HR], v1[HR];
       load_r(k0, k1, v0, v1, i0);
@@ -874,8 +905,7 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
       const int o = tid / VPR, c = tid % VPR;
       const long long src = s_src[o];
       const bool act = src >= 0;
-      float4 cs[4];
-      load_cs<D, STYLE>(s_cs4 + o * (D / 4), c, cs);
+      float4 cs[4];  // loaded once the table is filled
       const uint16_t* krow;
       const uint16_t* vrow;
       long long pl;
@@ -922,6 +952,10 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
 #if IS_PIPELINE
       uint4 ka[HW], va[HW], kb[HW], vb[HW];
       if (nw > 0) load_w(ka, va, 0);
+      fill_cs();
+      __syncthreads();
+      if (!phys_ok) return bad_block();
+      load_cs<D, STYLE>(s_cs4 + o * (D / 4), c, cs);
       for (int w0 = 0; w0 < nw; w0 += 2 * HW) {
         if (w0 + HW < nw) load_w(kb, vb, w0 + HW);
         store_w(ka, va, w0);
@@ -930,6 +964,10 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
         store_w(kb, vb, w0 + HW);
       }
 #else
+      fill_cs();
+      __syncthreads();
+      if (!phys_ok) return bad_block();
+      load_cs<D, STYLE>(s_cs4 + o * (D / 4), c, cs);
       for (int w0 = 0; w0 < nw; w0 += HW) {
         uint4 kv[HW], vv[HW];
         load_w(kv, vv, w0);
