@@ -344,16 +344,17 @@ int vec_order_for(int64_t token_stride, int64_t head_stride) { return token_stri
 // 0.952 to 0.991 of the copy peak); other shapes take the order whose
 // fastest row index has the larger cache stride.
 // Copy loop of a batch launch (see pick_fixed): the fixed shapes take the
-// per-thread loop; on a head-major cache (head stride above the token stride)
-// the paired rotate-half loop, whose CTA writes two heads' rows at once
-// (B200, Llama-3.1-8B-shaped batch on the head-major cache: 0.967 -> 0.987 of
-// the copy peak; on the token-major cache it was level on the benchmark
-// batch and 0.7% slower on the small case, so that layout keeps loop 1).
-int launch_loop(int D, int B, int H, int64_t token_stride, int64_t head_stride) {
+// paired rotate-half loop (2) on either cache layout; pick_fixed falls back to
+// the per-thread loop (1) for the interleaved pairing and for per-slot
+// sources.  B200: on the head-major cache the paired loop's CTA writes two
+// heads' rows at once (Llama-3.1-8B-shaped batch 0.967 -> 0.990 of the copy
+// peak); on the token-major cache it is 0.15% faster on the benchmark batch
+// and the Qwen2.5-7B-shaped batch and 0.15% slower on the small case.
+int launch_loop(int D, int B, int H) {
 #ifndef IS_NO_FIXED_SHAPES
-  if (D == 128 && B == 16 && (H == 4 || H == 8)) return head_stride > token_stride ? 2 : 1;
+  if (D == 128 && B == 16 && (H == 4 || H == 8)) return 2;
 #else
-  (void)D; (void)B; (void)H; (void)token_stride; (void)head_stride;
+  (void)D; (void)B; (void)H;
 #endif
   return 0;
 }
@@ -986,7 +987,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.fact_len_count = nfacts;
   // Per-slot sources: the host tier, or the arenas of a sharded view.
   const bool per_slot = s->host_arena || view;
-  const int loop = launch_loop(cf.head_dim, c.block_size, cf.num_kv_heads, c.token_stride, c.head_stride);
+  const int loop = launch_loop(cf.head_dim, c.block_size, cf.num_kv_heads);
   void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop)
                    : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop);
   int32_t small_R = R, small_ids = num_ids, small_grid = s->inject_grid, small_blocks = s->max_blocks;
