@@ -1,5 +1,5 @@
 """The benchmark's command-line contract, checked on CPU: the reference arm
-(the CPU oracle) prints one JSON line with the keys the driver reads, only
+(the CPU oracle) prints one JSON line with the keys of its output contract, only
 rank 0 prints under torchrun, too few warm-up steps are refused, and the
 GPU arm fails loudly without a CUDA device (no CPU fallback)."""
 from __future__ import annotations
