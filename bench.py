@@ -199,12 +199,27 @@ def time_oracle(args, threads: int) -> float:
     return dt
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(wl, device, budget_s=15.0):
-    """The oracle as it stands, on the host cores, on a bounded sample."""
+    """The oracle as it stands, on the host cores, on a bounded sample; also
+    its single-thread rate on the first request."""
     import oracle
     threads = oracle.max_threads()
     args, tok = oracle_sample(wl, [0], device)
     dt = time_oracle(args, threads)
+    dt1 = time_oracle(args, 1)
+    tok1 = tok
     n_req = int(max(1, min(wl.batch.num_requests, budget_s / max(dt, 1e-3))))
     if n_req > 1:
         del args
@@ -213,7 +228,10 @@ def cpu_baseline(wl, device, budget_s=15.0):
     return {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"first {n_req} of {wl.batch.num_requests} requests ({tok} tokens, all "
                       f"{wl.model.num_layers} layers x {wl.model.num_kv_heads} KV heads), "
-                      f"{dt:.2f} s"}
+                      f"{dt:.2f} s",
+            "single_thread_value": tok1 / dt1,
+            "single_thread_sample": f"request 0 ({tok1} tokens), {dt1:.2f} s",
+            "nproc": os.cpu_count(), "cpu_model": cpu_model()}
 
 
 # ------------------------------------------------------------------ main
