@@ -65,3 +65,17 @@ def test_host_validation_without_gpu():
                                0, None) == B.IS_ERR_INVALID_ARG
     assert lib.is_last_error(None, None, None) == B.IS_ERR_INVALID_ARG
     lib.is_store_destroy(None)  # ignored
+
+
+def test_cache_desc_rejects_what_the_library_cannot_address():
+    """Host-side checks of the torch wrapper: caches must be CUDA bf16 5-D
+    tensors with a unit innermost stride, K and V alike."""
+    import torch
+    from kv_cache_injection_gather_b200 import cache_desc
+    cpu = torch.zeros(1, 2, 16, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        cache_desc(cpu, cpu)  # not on a CUDA device
+    with pytest.raises(ValueError):
+        cache_desc(cpu.float(), cpu.float())
+    with pytest.raises(ValueError):
+        cache_desc(cpu[0], cpu[0])  # 4-D
