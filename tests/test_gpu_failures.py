@@ -81,3 +81,32 @@ def test_host_entry_point_reports_device_errors():
                            pin(b.block_tables), desc)
     assert rc == B.IS_OK
     store.close()
+
+
+@pytest.mark.parametrize("host_tier", [False, True], ids=["device-tier", "host-tier"])
+def test_failed_allocation_returns_oom_and_leaves_the_device_usable(host_tier):
+    """An HBM arena no device can hold (2^31 - 1 tokens per plane of
+    Llama-3.1-8B shapes, ~140 TB): the store's arena on the device tier, the
+    hot arena on the host tier (whose pinned store arena is small and is
+    freed again).  cudaMalloc refuses at once, create returns IS_ERR_OOM with
+    nothing leaked, and a normal store created afterwards injects correctly."""
+    _need_gpu()
+    from gpu_common import rope_of
+    from kv_cache_injection_gather_b200 import FactStore
+    m = synth.LLAMA31_8B
+    huge = (1 << 31) - 1
+    free0, _ = torch.cuda.mem_get_info()
+    with pytest.raises(B.InjectError) as e:
+        FactStore(m.num_layers, m.num_kv_heads, m.head_dim, rope_of(m), 64 if host_tier else huge, 16,
+                  host_tier=host_tier, hot_capacity_tokens=huge if host_tier else 0)
+    assert e.value.status == B.IS_ERR_OOM
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 >= free0 - (64 << 20)  # nothing of the failed store stays allocated
+    wl = synth.tiny(0)
+    store = make_store(wl)
+    k, v, desc = make_cache(wl)
+    ro, ids, sp, bt = batch_tensors(wl.batch)
+    store.inject(ro, ids, sp, bt, desc)
+    assert store.last_error()[0] == 0
+    store.close()
