@@ -1,8 +1,10 @@
 """The pins must catch plausible mistakes planted in the oracle.
 
 Each case compiles a copy of oracle/inject_oracle.c with one edit (a flipped
-sign, a wrong pair index, a dropped factor, an off-by-one position, a wrong
-slot, truncation instead of rounding, V taken from K, a misplaced offset),
+sign, a wrong pair index, a dropped factor, positions off by one, without the
+start or restarting per fact, a wrong slot, truncation or ties away from zero
+instead of round-to-even, V taken from K, K left unrotated, a misplaced
+offset, swapped cache strides, a bad id skipped, the wrong llama3 band),
 points ORACLE_LIB at it and runs the pin suite in a fresh process, which must
 fail.  CPU only; the real oracle is untouched.
 """
@@ -27,6 +29,25 @@ MUTANTS = {
     "truncating_bf16": ("double n = nearbyint(a / spacing);", "double n = floor(a / spacing);"),
     "v_from_k": ("c->v[dst + d] = s->v[src + d];", "c->v[dst + d] = s->k[src + d];"),
     "store_offset": ("s->off[id] = off;", "s->off[id] = off + 1;"),
+    # positions that ignore the request's start, or restart at every fact
+    "start_ignored": ("int64_t pos = (int64_t)start[r] + i;", "int64_t pos = i;"),
+    "position_restarts_per_fact": ("int64_t pos = (int64_t)start[r] + i;",
+                                   "int64_t pos = (int64_t)start[r] + t;"),
+    # a bad fact id skipped instead of invalidating its request
+    "bad_id_ignored": ("if (f < 0 || f >= s->num_facts) { st = ORC_ERR_BAD_FACT_ID; continue; }",
+                       "if (f < 0 || f >= s->num_facts) { continue; }"),
+    # the Llama-3.1 rule scaling the high frequencies it must keep
+    "llama3_high_band_scaled": ("if (lam < high_wl) return f;", "if (lam < high_wl) return f / factor;"),
+    # ties rounded away from zero instead of to even
+    "bf16_ties_away": ("double n = nearbyint(a / spacing);", "double n = round(a / spacing);"),
+    # the head and token strides of the cache swapped
+    "cache_strides_swapped": ("o * c->token_stride +\n                            h * c->head_stride;",
+                              "o * c->head_stride +\n                            h * c->token_stride;"),
+    # the block-table bound off by one (reads one entry past the row)
+    "table_bound_off_by_one": ("if (pos < 0 || pos / B >= max_blocks) return -1;",
+                               "if (pos < 0 || pos / B > max_blocks) return -1;"),
+    # K left unrotated
+    "k_not_rotated": ("c->k[dst + d] = orc_f64_to_bf16(y[d]);", "c->k[dst + d] = orc_f64_to_bf16(x[d]);"),
 }
 
 

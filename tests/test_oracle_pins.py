@@ -417,6 +417,23 @@ def test_segment_positions_brute_force():
     assert [tuple(map(int, w)) for w in want] == [tuple(map(int, g)) for g in got]
 
 
+def test_slot_formula_and_table_edges():
+    """slot = table[pos / B] * B + pos mod B inside the table; -1 for a
+    negative position, a position at or past the table's end, or an entry
+    outside the cache.  The row is a view into a longer array whose next
+    entry is a valid block, so reading one entry past the row would show."""
+    B, nb = 16, 64
+    full = np.array([5, 9, 2, 7], np.int32)
+    row = full[:3]
+    for pos in range(0, 3 * B):
+        assert oracle.slot(row, B, nb, pos) == int(row[pos // B]) * B + pos % B
+    assert oracle.slot(row, B, nb, 3 * B) == -1
+    assert oracle.slot(row, B, nb, 3 * B + 5) == -1
+    assert oracle.slot(row, B, nb, -1) == -1
+    assert oracle.slot(np.array([5, 64], np.int32), B, nb, B) == -1   # block id == num_blocks
+    assert oracle.slot(np.array([5, -1], np.int32), B, nb, B + 3) == -1
+
+
 def test_golden_tiny_regression():
     """The oracle's result on the tiny workload, frozen by
     tests/golden/make_golden.py (which calls only the oracle and the input
