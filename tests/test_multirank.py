@@ -144,7 +144,7 @@ class _HostShardStore:
         self.detached += 1
 
 
-def _fact_shard_worker(rank, world, port, out_dir):
+def _fact_shard_worker(rank, world, port, out_dir, contiguous=False):
     import sys
     sys.path.insert(0, ROOT)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -154,7 +154,10 @@ def _fact_shard_worker(rank, world, port, out_dir):
         from kv_cache_injection_gather_b200 import shard
         wl = _tiny_multi(seed=3)
         m = wl.model
-        owner = shard.round_robin_owner(len(wl.fact_lens), world)
+        n = len(wl.fact_lens)
+        owner = (np.concatenate([np.full(b - a, p, np.int32) for p, (a, b) in
+                                 enumerate(shard.contiguous_range(n, world, q) for q in range(world))])
+                 if contiguous else shard.round_robin_owner(n, world))
         mine = shard.owned_facts(owner, rank)
         st = oracle.Store(m.num_layers, m.num_kv_heads, m.head_dim,
                           int(wl.fact_lens[mine].sum()) + 7 * rank, len(mine))
@@ -176,7 +179,7 @@ def _fact_shard_worker(rank, world, port, out_dir):
         dist.all_gather_object(arenas, (st.k, st.v))
         grp.close()
         out = {"attached": fake.attached, "opened": opened, "closed": closed,
-               "detached": fake.detached, "arenas": arenas}
+               "detached": fake.detached, "arenas": arenas, "owner": owner}
         np.save(os.path.join(out_dir, f"fs{rank}.npy"), np.array([out], dtype=object),
                 allow_pickle=True)
     finally:
@@ -184,25 +187,27 @@ def _fact_shard_worker(rank, world, port, out_dir):
 
 
 @pytest.mark.timeout(300)
-def test_fact_shard_view_routes_every_global_id_with_gloo():
-    """Fact shards, host side: over world-size-2 gloo ranks holding alternate
-    facts, every rank builds the same global table and arena list (its own
-    arena, the peer's through the IPC mapping), and each global id's entry
-    points at that fact's rows in its owner's arena."""
+@pytest.mark.parametrize("world,contiguous", [(2, False), (3, True)], ids=["2-round-robin", "3-contiguous"])
+def test_fact_shard_view_routes_every_global_id_with_gloo(world, contiguous):
+    """Fact shards, host side: over gloo ranks holding alternate facts (or
+    contiguous id ranges), every rank builds the same global table and arena
+    list (its own arena, the peers' through the IPC mapping), and each global
+    id's entry points at that fact's rows in its owner's arena."""
     import synth
-    world = 2
     with tempfile.TemporaryDirectory() as d:
-        mp.start_processes(_fact_shard_worker, args=(world, _free_port(), d), nprocs=world,
-                           join=True, start_method="spawn")
+        mp.start_processes(_fact_shard_worker, args=(world, _free_port(), d, contiguous),
+                           nprocs=world, join=True, start_method="spawn")
         outs = [np.load(os.path.join(d, f"fs{r}.npy"), allow_pickle=True)[0] for r in range(world)]
     wl = _tiny_multi(seed=3)
     m = wl.model
     for rank, o in enumerate(outs):
         arenas, shard_of, off, ln = o["attached"]
         assert [a[:2] for a in arenas] == [(1000 + p, 2000 + p) for p in range(world)]
-        assert sorted(o["opened"]) == sorted(o["closed"]) == [1000 + 1 - rank, 2000 + 1 - rank]
+        peers = [p for p in range(world) if p != rank]
+        assert sorted(o["opened"]) == sorted(o["closed"]) == sorted([1000 + p for p in peers] +
+                                                                     [2000 + p for p in peers])
         assert o["detached"] == 1
-        assert np.array_equal(shard_of, np.arange(len(wl.fact_lens)) % world)
+        assert np.array_equal(shard_of, o["owner"])
         assert np.array_equal(ln, wl.fact_lens)
         for g in range(len(wl.fact_lens)):
             kp, vp, plane = arenas[shard_of[g]]
