@@ -10,6 +10,11 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # The CUDA library is built in-tree (nvcc, sm_100a); this is a no-op when
+    # it is newer than its sources.  The binding itself never builds: without
+    # the library it refuses to load.
+    from kv_cache_injection_gather_b200 import build
+    build.build()
 
 
 @pytest.fixture(scope="session")
