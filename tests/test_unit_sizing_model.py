@@ -4,8 +4,9 @@ its default knobs) checked for the properties the kernels and their
 documentation rely on, over far more shapes than the GPU tests run:
 
   * the layer ranges of a block's units partition [0, L), none empty;
-  * a batch whose one-layer units fit in two waves gets at most one unit per
-    CTA when its blocks fit the grid (latency), else one unit per block;
+  * a batch whose one-layer units fit in two waves gets about one wave of
+    units (latency): at most the grid plus one unit per block, since layers
+    are grouped in equal ranges;
   * a large batch gets units of at least 16 (layer, head) rows and two
     layers whenever the model has them;
   * the unit count fits the kernels' 32-bit counters.
@@ -49,7 +50,7 @@ def test_unit_sizing_invariants():
         assert ranges[0][0] == 0 and ranges[-1][1] == L
         assert all(ranges[i][1] == ranges[i + 1][0] for i in range(upb - 1))
         if tb * L <= 2 * grid:
-            assert tb * upb <= max(grid, tb), "one-wave batch: one unit per CTA (or per block)"
+            assert tb * upb <= grid + tb, "one-wave batch: about one wave of units"
         else:
             assert lpu >= min(L, 2)
             assert lpu * H >= min(MIN_ROWS, L * H) or lpu == L
