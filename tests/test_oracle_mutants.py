@@ -46,6 +46,10 @@ MUTANTS = {
     # the block-table bound off by one (reads one entry past the row)
     "table_bound_off_by_one": ("if (pos < 0 || pos / B >= max_blocks) return -1;",
                                "if (pos < 0 || pos / B > max_blocks) return -1;"),
+    # a blend weight that is monotone and exact at both band edges but not
+    # linear in orig / wavelength
+    "llama3_blend_squared": ("double smooth = (orig / lam - low) / (high - low);",
+                             "double smooth = (orig / lam - low) / (high - low);\n  smooth = smooth * smooth;"),
     # K left unrotated
     "k_not_rotated": ("c->k[dst + d] = orc_f64_to_bf16(y[d]);", "c->k[dst + d] = orc_f64_to_bf16(x[d]);"),
 }

@@ -118,6 +118,21 @@ def test_llama3_scaling_band_edges_and_identity():
     assert np.allclose(same, base, rtol=1e-15, atol=0)
 
 
+def test_llama3_blend_interior_values():
+    """Inside the band the rule mixes f/factor and f linearly in orig/lambda;
+    two interior points whose mixing weight is a simple fraction fix the
+    ratio scaled/unscaled exactly (a weight that is monotone and right at
+    both edges but not linear, e.g. its square, misses both):
+      factor 8, low 1, high 4, orig 8192, lambda 4096: weight 1/3, ratio
+        (2/3)(1/8) + 1/3 = 5/12;
+      factor 4, low 2, high 8, orig 16384, lambda 16384/5: weight 1/2,
+        ratio (1/2)(1/4) + 1/2 = 5/8."""
+    for lam, args, ratio in ((4096.0, (8.0, 1.0, 4.0, 8192.0), 5.0 / 12.0),
+                             (16384.0 / 5.0, (4.0, 2.0, 8.0, 16384.0), 5.0 / 8.0)):
+        f = 2 * math.pi / lam
+        assert math.isclose(oracle.llama3_scale(f, *args) / f, ratio, rel_tol=1e-13)
+
+
 def test_llama3_no_frequency_on_a_band_edge():
     """For D=128, theta=5e5 no wavelength equals 2048 or 8192 exactly, so the
     strict inequalities of the rule need no tie-break."""
