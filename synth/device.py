@@ -1,8 +1,12 @@
-"""Helpers shared by the GPU tests, the smoke check and the benchmark:
-building a FactStore and a paged cache from a seeded synthetic workload.
+"""Device-side inputs of a seeded synthetic workload: a FactStore holding
+its facts, a paged cache pre-filled with seeded values, the batch's index
+arrays as device tensors.  Used by the GPU tests, the smoke check and the
+benchmark.
 
-Input generation only (synth), plus marshalling into the library; no part
-of the inject arithmetic lives here.
+Input construction only (the generator of this package, then marshalling
+into the library's store); no part of the inject arithmetic lives here.
+The library is imported when a store is built, never at import time, so
+the host-side generator stays importable without it.
 """
 from __future__ import annotations
 
@@ -10,18 +14,18 @@ import numpy as np
 import torch
 
 import synth
-from kv_cache_injection_gather_b200 import FactStore, RopeConfig, cache_desc
 
 CACHE_FILL_SEED = 7
 
 
-def rope_of(model: synth.Model, style: int = 0) -> RopeConfig:
+def rope_of(model: synth.Model, style: int = 0):
+    from kv_cache_injection_gather_b200 import RopeConfig
     return RopeConfig(theta=model.rope_theta, style=style, llama3=model.scaling())
 
 
 def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = None,
                device: int = 0, extra_tokens: int = 0, small_limit: int | None = None,
-               heads: tuple[int, int] | None = None, facts=None, **limits) -> FactStore:
+               heads: tuple[int, int] | None = None, facts=None, **limits):
     """Put every fact of the workload, in id order (ids equal indices).
 
     Small stores are generated on the host (numpy) and copied; large ones are
@@ -30,6 +34,7 @@ def make_store(wl: synth.Workload, style: int = 0, on_device_gen: bool | None = 
     workload's model then names the full head count).  facts = increasing
     global ids keeps only those facts, local id i holding facts[i] (a
     fact-sharded store)."""
+    from kv_cache_injection_gather_b200 import FactStore
     full = wl.model
     m = full if heads is None else synth.Model(full.name, full.num_layers, heads[1] - heads[0],
                                                full.head_dim, full.rope_theta, full.llama3)
@@ -85,6 +90,7 @@ def make_cache(wl: synth.Workload, device: int = 0, fill: bool = True, head_majo
     """K and V caches (bf16, device); filled with seeded values so untouched
     slots can be checked, or left uninitialised.  num_kv_heads overrides the
     model's (a head-sharded cache)."""
+    from kv_cache_injection_gather_b200 import cache_desc
     shape = list(cache_shape(wl, head_major))
     if num_kv_heads is not None:
         shape[2 if head_major else 3] = num_kv_heads

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import synth
-from gpu_common import batch_tensors, make_cache, make_store
+from synth.device import batch_tensors, make_cache, make_store
 from kv_cache_injection_gather_b200 import binding as B
 
 pytestmark = pytest.mark.gpu
@@ -91,7 +91,7 @@ def test_failed_allocation_returns_oom_and_leaves_the_device_usable(host_tier):
     freed again).  cudaMalloc refuses at once, create returns IS_ERR_OOM with
     nothing leaked, and a normal store created afterwards injects correctly."""
     _need_gpu()
-    from gpu_common import rope_of
+    from synth.device import rope_of
     from kv_cache_injection_gather_b200 import FactStore
     m = synth.LLAMA31_8B
     huge = (1 << 31) - 1

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from gpu_common import make_store
+from synth.device import make_store
 from kv_cache_injection_gather_b200 import binding as B
 from test_gpu_parity import _ragged, assert_parity, gpu_run, oracle_run
 
@@ -84,7 +84,7 @@ def test_set_hot_errors_keep_previous_set():
 
 
 def _host_inject(store, wl):
-    from gpu_common import make_cache
+    from synth.device import make_cache
     from test_gpu_parity import to_bits
     b = wl.batch
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731

@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import synth
-from gpu_common import make_store
+from synth.device import make_store
 from kv_cache_injection_gather_b200 import binding as B
 from test_gpu_parity import assert_parity, gpu_run, oracle_run
 

@@ -22,7 +22,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import synth
-from gpu_common import make_store
+from synth.device import make_store
 from kv_cache_injection_gather_b200 import binding as B
 from kv_cache_injection_gather_b200 import shard
 from test_gpu_parity import PATHS, _need_gpu, _ragged, assert_parity, gpu_run, oracle_run
@@ -121,7 +121,7 @@ def test_attach_shards_validates_on_the_host():
     finally:
         for s in stores:
             s.close()
-    from gpu_common import rope_of
+    from synth.device import rope_of
     from kv_cache_injection_gather_b200 import FactStore
     m = wl.model
     host = FactStore(m.num_layers, m.num_kv_heads, m.head_dim, rope_of(m), 64, 4, host_tier=True,
