@@ -41,12 +41,8 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
-sys.path.insert(0, os.path.join(ROOT, "tests"))
 
 METRIC = "injected KV tokens/s and achieved HBM GB/s (vs ~8 TB/s); per-batch inject µs"
-# NVLink 5 peer copy measured on this kind of node, per direction per GPU
-# (900 GB/s nominal): the bound of reads from a peer's arenas.
-NVLINK_PEER_GBS = 770.0
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["kv_cache_injection_gather_b200/csrc/inject_kernels.cuh",
                   "kv_cache_injection_gather_b200/csrc/inject_store.cu"]
@@ -426,6 +422,38 @@ def h2d_probe(dev, nbytes: int = 1 << 30, reps: int = 5) -> float:
     return reps * nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9
 
 
+def peer_probe(dev, world: int, nbytes: int = 1 << 30, reps: int = 5) -> float:
+    """Per-GPU receive bandwidth from the peers (GB/s), measured in this run:
+    an all-to-all of nbytes per rank, in which every GPU takes (N-1)/N of its
+    bytes from the other GPUs at once -- the pattern of a fact-sharded batch,
+    whose rows come from every peer's arenas.  Timed with CUDA events on the
+    current stream (wall clock on CPU ranks), max over ranks."""
+    import torch
+    import torch.distributed as dist
+    cuda = torch.device(dev).type == "cuda"
+    n = (nbytes // (4 * world)) * world
+    src = torch.ones(n, dtype=torch.float32, device=dev)
+    dst = torch.empty_like(src)
+    dist.all_to_all_single(dst, src)  # warm-up (connections)
+    dist.barrier()
+    if cuda:
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        dist.all_to_all_single(dst, src)
+    if cuda:
+        e1.record()
+        torch.cuda.synchronize(dev)
+        sec = e0.elapsed_time(e1) / 1e3
+    else:
+        sec = time.perf_counter() - t0
+    (sec,) = max_over_ranks([sec], world)
+    return reps * (n * 4) * (world - 1) / world / sec / 1e9
+
+
 def max_over_ranks(values, world):
     """Element-wise max of per-rank numbers (timings) over all ranks."""
     import torch
@@ -447,7 +475,7 @@ def run_offload(args, rank, world, local_rank):
     import torch
 
     import synth
-    from gpu_common import make_cache, make_store
+    from synth.device import make_cache, make_store
     from kv_cache_injection_gather_b200 import binding as B
 
     torch.cuda.set_device(local_rank)
@@ -586,7 +614,7 @@ def run_sweep(args, rank, world, local_rank):
     are timed step by step with an L2 flush between steps."""
     import torch
 
-    from gpu_common import batch_tensors, make_cache, make_store
+    from synth.device import batch_tensors, make_cache, make_store
     from kv_cache_injection_gather_b200 import binding as B
     S = _synth()
     if args.workload not in ("qwen-sweep", "mistral-sweep"):
@@ -650,7 +678,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    from gpu_common import batch_tensors, make_cache, make_store
+    from synth.device import batch_tensors, make_cache, make_store
     from kv_cache_injection_gather_b200 import binding as B
 
     if not torch.cuda.is_available():
@@ -705,6 +733,8 @@ def run_ours(args, rank, world, local_rank):
                                       num_kv_heads=None if heads is None else heads[1] - heads[0])
     extra_cfg["cache_layout"] = "[L][num_blocks][H][B][D]" if args.head_major else "[L][num_blocks][B][H][D]"
     copy_ref, copy_sus = copy_probe(dev)
+    # every rank takes part in the same collectives, in the same order
+    peer_gbs = peer_probe(dev, world) if (owner is not None and world > 1) else None
     ro, ids, sp, bt = batch_tensors(b, local_rank)
     n_tok = wl.tokens()
     slots = torch.empty(n_tok, dtype=torch.int64, device=dev)
@@ -796,14 +826,15 @@ def run_ours(args, rank, world, local_rank):
                 "kernel": "inject_kernel (plan_kernel excluded)"}
     if owner is not None and world > 1:
         # Peer reads: rows of facts other ranks own cross NVLink once; the
-        # bound is those bytes at the measured peer-copy bandwidth.
+        # bound is those bytes at the peer bandwidth measured in this run.
         ids_all = b.fact_ids
         remote_tok = int(wl.fact_lens[ids_all[owner[ids_all] != rank]].sum())
         link_bytes = remote_tok * m.bytes_per_token
         link = link_bytes / (kern_avg_ms / 1e3) / 1e9
-        roofline = {"bound": "nvlink", "achieved": link, "peak": NVLINK_PEER_GBS,
-                    "unit": "GB/s", "frac": link / NVLINK_PEER_GBS,
-                    "peak_source": "measured peer copy per direction (pool reference)",
+        roofline = {"bound": "nvlink", "achieved": link, "peak": peer_gbs,
+                    "unit": "GB/s", "frac": link / peer_gbs,
+                    "peak_source": f"in-run peer probe: NCCL all-to-all of 1 GiB per rank, "
+                                   f"per-GPU receive bandwidth over {world} GPUs (max over ranks)",
                     "link_bytes": link_bytes, "hbm_achieved_gbs": achieved,
                     "hbm_frac": achieved / peak, "traffic": None, "algorithmic_bytes": algo_bytes,
                     "kernel": "inject_kernel (plan_kernel excluded)"}

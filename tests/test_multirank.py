@@ -3,7 +3,8 @@ standing in for each rank's GPU.  Head shards and request shards each
 reproduce the single-rank result with no data exchange; the fact-shard
 view's set-up (table and handle swap, peer mapping, collective close)
 routes every global fact id to its rows; the benchmark's max-over-ranks
-timing reduction works across processes."""
+timing reduction and its in-run peer-bandwidth probe work across
+processes."""
 from __future__ import annotations
 
 import os
@@ -80,7 +81,10 @@ def _worker(rank, world, port, out_dir):
         dist.all_gather_object(rparts, (kr, vr, sr))
         # max over ranks of the step time, as the benchmark reports it
         got = bench.max_over_ranks([10.0 + rank, 3.0 * (1 - rank)], world)
+        # the in-run peer probe of the fact-shard roofline (all-to-all)
+        peer = bench.peer_probe("cpu", world, nbytes=1 << 22, reps=2)
         if rank == 0:
+            np.save(os.path.join(out_dir, "peer.npy"), np.array([peer]))
             np.save(os.path.join(out_dir, "heads.npy"), np.array(parts, dtype=object), allow_pickle=True)
             np.save(os.path.join(out_dir, "reqs.npy"), np.array(rparts, dtype=object), allow_pickle=True)
             np.save(os.path.join(out_dir, "max.npy"), np.array(got))
@@ -97,6 +101,7 @@ def test_partitions_reproduce_single_rank_with_gloo():
         heads = np.load(os.path.join(d, "heads.npy"), allow_pickle=True)
         reqs = np.load(os.path.join(d, "reqs.npy"), allow_pickle=True)
         mx = np.load(os.path.join(d, "max.npy"))
+        peer = float(np.load(os.path.join(d, "peer.npy"))[0])
     wl = _tiny_multi()
     kf, vf, sf = _oracle_inject(wl)
     # head shards concatenate to the full cache
@@ -112,6 +117,7 @@ def test_partitions_reproduce_single_rank_with_gloo():
         v_u.reshape(flat_v.shape)[:, sr] = flat_v[:, sr]
     assert np.array_equal(k_u, kf) and np.array_equal(v_u, vf)
     assert list(mx) == [11.0, 3.0]
+    assert 0.0 < peer < float("inf")
 
 
 class _HostShardStore:
