@@ -72,8 +72,8 @@ struct DevStatus {
 // Written by plan_kernel, read by inject_kernel.
 struct PlanHeader {
   int32_t total_blocks;      // touched cache blocks over all valid requests
-  int32_t layers_per_unit;   // layers one work unit covers
-  int32_t units_per_block;   // ceil(L / layers_per_unit)
+  int32_t rows_per_unit;     // (layer, head) rows one work unit covers
+  int32_t units_per_block;   // ceil(L * H / rows_per_unit)
   int32_t total_units;       // total_blocks * units_per_block (0: write nothing)
   unsigned int next_unit;    // dynamic work counter, reset by plan_kernel
   int32_t pad;
@@ -94,22 +94,33 @@ __device__ __forceinline__ void record_error(DevStatus* st, int32_t code, long l
 
 // ---------------------------------------------------------------- plan kernel
 
-// Work-unit size (layers per unit lpu, units per block upb).  A batch whose
-// one-layer units fit in about two waves of the grid takes the fewest layers
-// per unit that fit one wave (one layer when they already do): everything is
-// in flight at once and no CTA runs a second unit after the first (latency).
-// Larger batches aim at ~IS_UNITS_PER_CTA units per CTA, so the dynamic
-// schedule's tail (at most one unit) stays short, with at least
-// IS_UNIT_MIN_ROWS (layer, head) rows per unit (and at least two layers) so
-// a unit's set-up (slot walk, cos/sin table, barriers) is shared by enough
-// copies, and IS_UNIT_ROWS_LARGE rows when the batch still has
-// IS_UNITS_PER_CTA_MIN units per CTA with them.  Measured on B200 over the
-// Mistral/Qwen sweep grid: with H = 4, two-layer units ran at 0.87 of the
-// copy peak, 16-row units at 0.93-0.96, 32-row units up to 0.97 on large
-// batches but slower where they leave few units per CTA.
+// Work-unit size: rows per unit rpu and units per block upb, where a row is
+// one (layer, head) pair of a cache block, numbered w = layer * H + head, and
+// unit g of a block covers rows [g * rpu, min(L * H, (g + 1) * rpu)).  A batch
+// whose one-layer units fit in about two waves of the grid is split into
+// about one wave of units (latency: everything is in flight at once and no
+// CTA runs a second unit after the first): with row_units (the per-thread
+// copy loops, which take any row range) into equal row ranges, otherwise
+// into equal layer ranges.  Larger batches aim at ~IS_UNITS_PER_CTA units
+// per CTA, so the dynamic schedule's tail (at most one unit) stays short,
+// in whole layers with at least IS_UNIT_MIN_ROWS rows (and at least two
+// layers) per unit so a unit's set-up (slot walk, cos/sin table, barriers)
+// is shared by enough copies, and IS_UNIT_ROWS_LARGE rows when the batch
+// still has IS_UNITS_PER_CTA_MIN units per CTA with them.  Measured on B200
+// over the Mistral/Qwen sweep grid: with H = 4, two-layer units ran at 0.87
+// of the copy peak, 16-row units at 0.93-0.96, 32-row units up to 0.97 on
+// large batches but slower where they leave few units per CTA.
 __device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32_t H, int32_t grid_ctas,
-                                          int32_t& lpu, int32_t& upb) {
+                                          bool row_units, int32_t& rpu, int32_t& upb) {
   const long long grid = grid_ctas;
+  const int32_t LH = L * H;
+  if (total_blocks > 0 && row_units && (long long)total_blocks * L <= 2 * grid) {
+    const long long per = ((long long)total_blocks * LH + grid - 1) / grid;  // rows per unit
+    upb = int32_t((LH + per - 1) / per);
+    rpu = (LH + upb - 1) / upb;
+    upb = (LH + rpu - 1) / rpu;
+    return;
+  }
   upb = 1;
   if (total_blocks > 0 && (long long)total_blocks * L <= 2 * grid) {
     const long long per = ((long long)total_blocks * L + grid - 1) / grid;  // 1 or 2 layers per unit
@@ -124,8 +135,9 @@ __device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32
     const long long want = (grid * IS_UNITS_PER_CTA + total_blocks - 1) / total_blocks;
     upb = int32_t(max(1LL, min(want, cap)));
   }
-  lpu = (L + upb - 1) / upb;
+  const int32_t lpu = (L + upb - 1) / upb;
   upb = (L + lpu - 1) / lpu;
+  rpu = lpu * H;
 }
 
 struct PlanArgs {
@@ -134,15 +146,24 @@ struct PlanArgs {
   const int32_t* fact_ids;   // [num_ids]
   int32_t num_ids;
   const int32_t* start_pos;  // [R]
+  const int32_t* block_tables;  // [R][max_blocks]
   int32_t max_blocks;
+  int32_t num_blocks;        // cache blocks (table entries outside: BAD_BLOCK)
   int32_t B;
   int32_t L;
   int32_t H;
   const int32_t* fact_len;   // store: [num_facts]
   int32_t num_facts;
+  // A fact table the library did not build (the allocation-free entry
+  // point): when chk_off is set, an id whose entry does not lie inside the
+  // arenas -- offset < 0, length < 1 or offset + length > chk_plane tokens
+  // -- counts as an id outside the store.
+  const int64_t* chk_off;
+  int64_t chk_plane;
   int64_t* slot_out;         // optional
   int64_t slot_cap;
   int32_t grid_ctas;         // size of the inject grid (for unit sizing)
+  int32_t row_units;         // the inject kernel's copy loop takes any row range
   int32_t max_batch_blocks;  // capacity of desc
   // work space
   int32_t* seg;              // [num_ids]   segment offset of each CSR entry (-1: bad id)
@@ -150,7 +171,7 @@ struct PlanArgs {
   int32_t* req_blk0;         // [R+1]       exclusive prefix of req_nblk
   long long* req_tok0;       // [R+1]       exclusive prefix of segment lengths
   int32_t* req_len;          // [R]         segment length (valid facts)
-  int32_t* req_valid;        // [R]
+  int32_t* req_err;          // [R]         0, or the request's IS_ERR code
   BlockDesc* desc;           // [max_batch_blocks]
   PlanHeader* hdr;
   DevStatus* st;
@@ -174,8 +195,13 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ int s_bad;
-  __shared__ int s_wsum_blk[NW];
+  __shared__ int s_len_over;  // a request's facts total more than 2^31 - 1 tokens
+  __shared__ long long s_wsum_blk[NW];
   __shared__ long long s_wsum_tok[NW];
+  __shared__ long long s_total_blk;
+  // First error in request order: (request << 32) | logical block, the
+  // block part used for a block-table entry outside the cache.
+  __shared__ unsigned long long s_err_key;
   extern __shared__ __align__(16) unsigned char plan_dyn[];
 
   // The inject grid may be scheduled now; it waits for this grid's results
@@ -189,7 +215,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   int32_t* req_blk0 = a.req_blk0;
   long long* req_tok0 = a.req_tok0;
   int32_t* req_len = a.req_len;
-  int32_t* req_valid = a.req_valid;
+  int32_t* req_err = a.req_err;
   if constexpr (SMEM) {
     long long* s_tok0 = reinterpret_cast<long long*>(plan_dyn);  // [R+1]
     int32_t* s_off = reinterpret_cast<int32_t*>(s_tok0 + (a.R + 1));
@@ -209,12 +235,16 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     req_blk0 = s_blk0;
     req_tok0 = s_tok0;
     req_len = s_len;
-    req_valid = s_valid;
+    req_err = s_valid;
   }
 
   // The CSR must start at 0, end at num_ids and never decrease; otherwise
   // the whole batch is rejected and nothing is written.
-  if (tid == 0) s_bad = a.R < 0 || req_off[0] != 0 || req_off[a.R] != a.num_ids;
+  if (tid == 0) {
+    s_bad = a.R < 0 || req_off[0] != 0 || req_off[a.R] != a.num_ids;
+    s_len_over = 0;
+    s_err_key = ~0ull;
+  }
   __syncthreads();
   for (int r = tid; r < a.R; r += NT)
     if (req_off[r + 1] < req_off[r]) s_bad = 1;
@@ -224,7 +254,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     a.hdr->total_blocks = 0;
     a.hdr->total_units = 0;
     a.hdr->units_per_block = 1;
-    a.hdr->layers_per_unit = a.L;
+    a.hdr->rows_per_unit = a.L * a.H;
     a.hdr->next_unit = 0;
     a.hdr->total_tokens = 0;
   }
@@ -241,10 +271,25 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
       const int32_t j = base + q * NT + tid;
       f[q] = j < a.num_ids ? a.fact_ids[j] : -1;
     }
+    if (a.chk_off == nullptr) {
 #pragma unroll
-    for (int q = 0; q < P0; ++q) {
-      const int32_t j = base + q * NT + tid;
-      if (j < a.num_ids) seg[j] = (f[q] >= 0 && f[q] < a.num_facts) ? a.fact_len[f[q]] : -1;
+      for (int q = 0; q < P0; ++q) {
+        const int32_t j = base + q * NT + tid;
+        if (j < a.num_ids) seg[j] = (f[q] >= 0 && f[q] < a.num_facts) ? a.fact_len[f[q]] : -1;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < P0; ++q) {
+        const int32_t j = base + q * NT + tid;
+        if (j >= a.num_ids) continue;
+        int32_t lf = -1;
+        if (f[q] >= 0 && f[q] < a.num_facts) {
+          const int32_t n = a.fact_len[f[q]];
+          const int64_t o = a.chk_off[f[q]];
+          if (n >= 1 && o >= 0 && o <= a.chk_plane - n) lf = n;
+        }
+        seg[j] = lf;
+      }
     }
   }
   __syncthreads();
@@ -262,13 +307,15 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
         const int32_t j = base + lane;
         const int32_t lj = j < j1 ? seg[j] : 0;
         const bool ok = lj >= 0;
-        const int32_t len = ok ? lj : 0;
-        int32_t x = len;  // inclusive warp scan
+        const long long len = ok ? lj : 0;
+        long long x = len;  // inclusive warp scan, 64-bit: lengths may be large
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-          const int32_t y = __shfl_up_sync(0xffffffffu, x, d);
+          const long long y = __shfl_up_sync(0xffffffffu, x, d);
           if (lane >= d) x += y;
         }
+        // (offsets of a request longer than 2^31 - 1 tokens wrap here, but
+        // such a request fails the batch below and its offsets are not read)
         if (j < j1) seg[j] = ok ? int32_t(S + x - len) : -1;
         const unsigned badm = __ballot_sync(0xffffffffu, j < j1 && !ok);
         if (badm && err == kOk) err = kErrBadFactId;
@@ -282,9 +329,10 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
       int32_t nblk = 0;
       if (err == kOk && S > 0) nblk = int32_t((start + S - 1) / a.B - start / a.B + 1);
       req_nblk[r] = nblk;
-      req_len[r] = int32_t(S);
-      req_valid[r] = err == kOk;
-      if (err != kOk) record_error(a.st, err, r);
+      if (S > 0x7fffffffLL) s_len_over = 1;
+      req_len[r] = int32_t(min(S, 0x7fffffffLL));
+      req_err[r] = err;
+      if (err != kOk) atomicMin(&s_err_key, (unsigned long long)r << 32);
     }
   }
   __syncthreads();
@@ -293,41 +341,44 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   // owns a contiguous run of requests.
   const int per = (a.R + NT - 1) / NT;
   const int r0 = min(a.R, tid * per), r1 = min(a.R, r0 + per);
-  int32_t my_blk = 0;
+  long long my_blk = 0;
   long long my_tok = 0;
   for (int r = r0; r < r1; ++r) { my_blk += req_nblk[r]; my_tok += req_len[r]; }
-  int32_t xb = my_blk;
+  long long xb = my_blk;
   long long xt = my_tok;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
-    const int32_t yb = __shfl_up_sync(0xffffffffu, xb, d);
+    const long long yb = __shfl_up_sync(0xffffffffu, xb, d);
     const long long yt = __shfl_up_sync(0xffffffffu, xt, d);
     if (lane >= d) { xb += yb; xt += yt; }
   }
   if (lane == 31) { s_wsum_blk[warp] = xb; s_wsum_tok[warp] = xt; }
   __syncthreads();
   // Exclusive prefix of the warp sums: a shuffle scan over lanes = warps.
-  int32_t wb = lane < NW ? s_wsum_blk[lane] : 0;
+  long long wb = lane < NW ? s_wsum_blk[lane] : 0;
   long long wt = lane < NW ? s_wsum_tok[lane] : 0;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
-    const int32_t yb = __shfl_up_sync(0xffffffffu, wb, d);
+    const long long yb = __shfl_up_sync(0xffffffffu, wb, d);
     const long long yt = __shfl_up_sync(0xffffffffu, wt, d);
     if (lane >= d) { wb += yb; wt += yt; }
   }
   wb = warp > 0 ? __shfl_sync(0xffffffffu, wb, warp - 1) : 0;
   wt = warp > 0 ? __shfl_sync(0xffffffffu, wt, warp - 1) : 0;
-  int32_t eb = wb + xb - my_blk;
+  // Block prefixes are stored in 32 bits: a batch whose total would not
+  // fit is over every block capacity and fails below before they are read.
+  long long eb = wb + xb - my_blk;
   long long et = wt + xt - my_tok;
   for (int r = r0; r < r1; ++r) {
-    req_blk0[r] = eb;
+    req_blk0[r] = int32_t(min(eb, 0x7fffffffLL));
     req_tok0[r] = et;
     eb += req_nblk[r];
     et += req_len[r];
   }
   if (tid == NT - 1) {
-    req_blk0[a.R] = eb;
+    req_blk0[a.R] = int32_t(min(eb, 0x7fffffffLL));
     req_tok0[a.R] = et;
+    s_total_blk = eb;
   }
   __syncthreads();
   if constexpr (SMEM) {
@@ -337,29 +388,34 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   }
   const int32_t total_blocks = req_blk0[a.R];
   const long long total_tokens = req_tok0[a.R];
-  const bool over_slots = a.slot_out != nullptr && total_tokens > a.slot_cap;
-  const bool over_blocks = total_blocks > a.max_batch_blocks;
+  const bool over_slots = (a.slot_out != nullptr && total_tokens > a.slot_cap) || s_len_over;
+  const bool over_blocks = s_total_blk > a.max_batch_blocks;
 
   if (tid == 0) {
-    int32_t lpu, upb;
-    unit_size(total_blocks, a.L, a.H, a.grid_ctas, lpu, upb);
-    a.hdr->layers_per_unit = lpu;
+    int32_t rpu, upb;
+    unit_size(total_blocks, a.L, a.H, a.grid_ctas, a.row_units != 0, rpu, upb);
+    a.hdr->rows_per_unit = rpu;
     a.hdr->units_per_block = upb;
     a.hdr->total_blocks = total_blocks;
     a.hdr->total_tokens = total_tokens;
     a.hdr->next_unit = 0;
     a.hdr->total_units = (over_slots || over_blocks) ? 0 : total_blocks * upb;
+    // A batch over capacity writes nothing and reports only that.
     if (over_slots || over_blocks) record_error(a.st, kErrCapacity, total_tokens);
   }
   if (over_slots || over_blocks) return;
 
   // Phase 3, one warp per request: block descriptors (lanes over blocks, so
-  // a warp writes consecutive descriptors), and -1 slots for the tokens of
-  // invalid requests.
+  // a warp writes consecutive descriptors), the check of every touched
+  // block-table entry, and -1 slots for the tokens of invalid requests.
+  auto check_entry = [&](int r, int32_t b) {
+    const int32_t phys = a.block_tables[(long long)r * a.max_blocks + b];
+    if (phys < 0 || phys >= a.num_blocks) atomicMin(&s_err_key, ((unsigned long long)r << 32) | unsigned(b));
+  };
   for (int r = warp; r < a.R; r += NW) {
     const int32_t j0 = req_off[r], j1 = req_off[r + 1];
     const long long t0 = req_tok0[r];
-    if (!req_valid[r]) {
+    if (req_err[r] != kOk) {
       if (a.slot_out)
         for (int32_t i = lane; i < req_len[r]; i += 32) a.slot_out[t0 + i] = -1;
       continue;
@@ -389,6 +445,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
         d.j = lo;
         d.pad = 0;
         a.desc[g0 + bi] = d;
+        check_entry(r, fb + bi);
       }
     } else {
       // Lanes over facts (no dependent L2 reads): fact j [s, e) owns the
@@ -410,9 +467,20 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
           d.j = j;
           d.pad = 0;
           a.desc[g0 + bi] = d;
+          check_entry(r, fb + bi);
         }
       }
     }
+  }
+  // The batch's first error in request order: a request's own error, or,
+  // in a valid request, its first block-table entry outside the cache (the
+  // inject kernel skips such blocks).
+  __syncthreads();
+  if (tid == 0 && s_err_key != ~0ull) {
+    const int r = int(s_err_key >> 32);
+    const int32_t b = int32_t(s_err_key & 0xffffffffull);
+    if (req_err[r] != kOk) record_error(a.st, req_err[r], r);
+    else record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
   }
 }
 
@@ -449,6 +517,13 @@ struct InjectArgs {
   const uint16_t* v_hot;
   int64_t hot_plane;         // hot_cap * D
   const int64_t* hot_off;    // [num_facts], -1 when the fact is not in HBM
+  // least-recently-used hot set, promotion fused into the batch: facts with
+  // pend[f] >= 0 are read from host memory as cold ones and their rows are
+  // also written to hot tokens [pend[f], pend[f] + len) of these (the hot)
+  // arenas; pend == nullptr: no promotion in this batch
+  const int64_t* pend;
+  uint16_t* k_prom;
+  uint16_t* v_prom;
   // fact-sharded view (per-slot source variant; shard_k == nullptr: none):
   // fact f's rows sit in arena fact_shard[f] ([L][H][plane][D], this GPU's
   // or a peer's memory) at token fact_off[f]
@@ -713,9 +788,15 @@ struct UnitShared {
   const uint16_t* kb[HOST_TIER ? kMaxBlockSize : 1];
   const uint16_t* vb[HOST_TIER ? kMaxBlockSize : 1];
   long long pl[HOST_TIER ? kMaxBlockSize : 1];
+  // host tier, fused promotion: hot-arena row bases that also receive the
+  // slot's stored K and V rows (nullptr: none); plane stride a.hot_plane
+  uint16_t* pk[HOST_TIER ? kMaxBlockSize : 1];
+  uint16_t* pv[HOST_TIER ? kMaxBlockSize : 1];
 };
 
-// One work unit: cache block b (logical, of request r) x layers [l0, l1).
+// One work unit: cache block b (logical, of request r) x (layer, head) rows
+// [w0, w1), row w = layer * H + head (the copy loop FAST == 0 takes whole
+// layers only: w0 and w1 multiples of H).
 // j is the CSR index of the first fact with a token in the block, seg[] the
 // facts' segment offsets (global or shared memory), j1 the end of the
 // request's CSR range, len_r its segment length, tok0 its first slot-mapping
@@ -728,7 +809,7 @@ template <int D, int STYLE, int NT, int VPT, bool POW2, bool HOST_TIER, int HC, 
 __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TIER>& sm,
                                          float4* s_cs4, int r, int b, int j_first,
                                          const int32_t* seg, int j1, int start, int len_r,
-                                         long long tok0, int l0, int l1, bool write_slots,
+                                         long long tok0, int w0, int w1, bool write_slots,
                                          const int32_t* jfid = nullptr, const long long* joff = nullptr) {
   constexpr int VPR = D / 8;  // 16-byte vectors per head row
   constexpr int LOG_VPR = (VPR == 4) ? 2 : (VPR == 8) ? 3 : (VPR == 16) ? 4 : 5;
@@ -747,6 +828,8 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
   const uint16_t** s_kb = sm.kb;
   const uint16_t** s_vb = sm.vb;
   long long* s_pl = sm.pl;
+  uint16_t** s_pk = sm.pk;
+  uint16_t** s_pv = sm.pv;
 
   const int blk_pos = b * B;                         // position of in-block slot 0
   const int o_lo = max(start - blk_pos, 0);
@@ -759,6 +842,7 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
   if (tid < B) {
     const int o = tid;
     long long src = -1;
+    if (HOST_TIER) s_pk[o] = s_pv[o] = nullptr;
     if (o >= o_lo && o < o_hi) {
       const int i = blk_pos + o - start;  // segment index
       int j = j_first;
@@ -781,6 +865,11 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
           s_kb[o] = a.k_store + src * D;
           s_vb[o] = a.v_store + src * D;
           s_pl[o] = a.plane;
+          const long long pd = a.pend ? a.pend[f] : -1;
+          if (pd >= 0) {
+            s_pk[o] = a.k_prom + (pd + t) * D;
+            s_pv[o] = a.v_prom + (pd + t) * D;
+          }
         }
       }
       if (write_slots && a.slot_out) a.slot_out[tok0 + i] = phys_ok ? (long long)phys * B + o : -1;
@@ -797,10 +886,8 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
     }
   };
   // A block-table entry outside the cache: nothing is stored (uniform; the
-  // caller's barrier follows).
-  auto bad_block = [&]() {
-    if (tid == 0 && write_slots) record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
-  };
+  // caller's barrier follows).  The plan reports it.
+  auto bad_block = [&]() {};
   if constexpr (FAST == 0) {
     fill_cs();  // before the block-table entry is checked, so its load overlaps
     if (!phys_ok) return bad_block();
@@ -837,11 +924,11 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
     const bool act = src >= 0;
     CsPairs cp;  // loaded once the table is filled
     const long long pl = a.plane;
-    const uint16_t* kp = a.k_store + (act ? src : 0) * D + c * 8 + (long long)(l0 * HC + rp) * pl;
-    const uint16_t* vp = a.v_store + (act ? src : 0) * D + c * 8 + (long long)(l0 * HC + rp) * pl;
+    const uint16_t* kp = a.k_store + (act ? src : 0) * D + c * 8 + (long long)(w0 + rp) * pl;
+    const uint16_t* vp = a.v_store + (act ? src : 0) * D + c * 8 + (long long)(w0 + rp) * pl;
     uint16_t* kd = a.k_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
     uint16_t* vd = a.v_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
-    const int nr = ((l1 - l0) * HC - rp + 1) / 2;  // rows w = 2i + rp, i < nr
+    const int nr = (w1 - w0 - rp + 1) / 2;  // rows w0 + 2i + rp, i < nr
     constexpr int HR = IS_PIPELINE ? VPT / 4 : VPT / 2;  // rows per stage, 4 vectors each
     auto load_r = [&](uint4 (&ka)[HR], uint4 (&kb)[HR], uint4 (&va)[HR], uint4 (&vb)[HR], int i0) {
 #pragma unroll
@@ -864,8 +951,8 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
         const int i = i0 + q;
         rotate_half_pair(ka[q], kb[q], cp);
         if (act && i < nr) {
-          const int w = 2 * i + rp;
-          const int l = l0 + w / HC, h = w % HC;
+          const int w = w0 + 2 * i + rp;
+          const int l = w / HC, h = w % HC;
           const long long off = (long long)l * a.ls + (long long)h * a.hs;
           st_stream(kd + off, ka[q]);
           st_stream(kd + off + HALF, kb[q]);
@@ -909,25 +996,32 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
       const uint16_t* krow;
       const uint16_t* vrow;
       long long pl;
+      uint16_t* pkp = nullptr;  // fused promotion: this slot's hot rows
+      uint16_t* pvp = nullptr;
       if constexpr (HOST_TIER) {
         krow = act ? s_kb[o] : a.k_store;
         vrow = act ? s_vb[o] : a.v_store;
         pl = act ? s_pl[o] : 0;
+        if (act && s_pk[o] != nullptr) {
+          pkp = s_pk[o] + c * 8 + (long long)w0 * a.hot_plane;
+          pvp = s_pv[o] + c * 8 + (long long)w0 * a.hot_plane;
+        }
       } else {
         krow = a.k_store + (act ? src : 0) * D;
         vrow = a.v_store + (act ? src : 0) * D;
         pl = a.plane;
       }
-      const uint16_t* kp = krow + c * 8 + (long long)l0 * HC * pl;
-      const uint16_t* vp = vrow + c * 8 + (long long)l0 * HC * pl;
+      const uint16_t* kp = krow + c * 8 + (long long)w0 * pl;
+      const uint16_t* vp = vrow + c * 8 + (long long)w0 * pl;
       uint16_t* kd = a.k_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
       uint16_t* vd = a.v_cache + (long long)phys * a.bs + (long long)o * a.ts + c * 8;
-      const int nw = (l1 - l0) * HC;  // (layer, head) rows of this thread, in plane order
+      const int nw = w1 - w0;  // (layer, head) rows of this thread, in plane order
       constexpr int HW = IS_PIPELINE ? VPT / 2 : VPT;
-      auto load_w = [&](uint4 (&kv)[HW], uint4 (&vv)[HW], int w0) {
+      // (stage rows s0 + q of the unit; w0 is the unit's first row)
+      auto load_w = [&](uint4 (&kv)[HW], uint4 (&vv)[HW], int s0) {
 #pragma unroll
         for (int q = 0; q < HW; ++q) {
-          const int w = w0 + q;
+          const int w = s0 + q;
           kv[q] = make_uint4(0, 0, 0, 0);
           vv[q] = kv[q];
           if (act && w < nw) {
@@ -936,16 +1030,20 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
           }
         }
       };
-      auto store_w = [&](const uint4 (&kv)[HW], const uint4 (&vv)[HW], int w0) {
+      auto store_w = [&](const uint4 (&kv)[HW], const uint4 (&vv)[HW], int s0) {
 #pragma unroll
         for (int q = 0; q < HW; ++q) {
-          const int w = w0 + q;
+          const int w = s0 + q;
           const uint4 kr = rotate_regs<D, STYLE>(kv[q], c, cs);
           if (act && w < nw) {
-            const int l = l0 + w / HC, h = w % HC;
+            const int l = (w0 + w) / HC, h = (w0 + w) % HC;
             const long long off = (long long)l * a.ls + (long long)h * a.hs;
             st_stream(kd + off, kr);
             st_stream(vd + off, vv[q]);
+            if (HOST_TIER && pkp != nullptr) {  // the stored rows, unrotated
+              st_stream(pkp + (long long)w * a.hot_plane, kv[q]);
+              st_stream(pvp + (long long)w * a.hot_plane, vv[q]);
+            }
           }
         }
       };
@@ -956,26 +1054,27 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
       __syncthreads();
       if (!phys_ok) return bad_block();
       load_cs<D, STYLE>(s_cs4 + o * (D / 4), c, cs);
-      for (int w0 = 0; w0 < nw; w0 += 2 * HW) {
-        if (w0 + HW < nw) load_w(kb, vb, w0 + HW);
-        store_w(ka, va, w0);
-        if (w0 + HW >= nw) break;
-        if (w0 + 2 * HW < nw) load_w(ka, va, w0 + 2 * HW);
-        store_w(kb, vb, w0 + HW);
+      for (int s0 = 0; s0 < nw; s0 += 2 * HW) {
+        if (s0 + HW < nw) load_w(kb, vb, s0 + HW);
+        store_w(ka, va, s0);
+        if (s0 + HW >= nw) break;
+        if (s0 + 2 * HW < nw) load_w(ka, va, s0 + 2 * HW);
+        store_w(kb, vb, s0 + HW);
       }
 #else
       fill_cs();
       __syncthreads();
       if (!phys_ok) return bad_block();
       load_cs<D, STYLE>(s_cs4 + o * (D / 4), c, cs);
-      for (int w0 = 0; w0 < nw; w0 += HW) {
+      for (int s0 = 0; s0 < nw; s0 += HW) {
         uint4 kv[HW], vv[HW];
-        load_w(kv, vv, w0);
-        store_w(kv, vv, w0);
+        load_w(kv, vv, s0);
+        store_w(kv, vv, s0);
       }
 #endif
     }
   } else {
+    const int l0 = w0 / H, l1 = w1 / H;  // whole layers
     const int total = (l1 - l0) * vecs_layer;
     const uint16_t* kst = a.k_store;
     const uint16_t* vst = a.v_store;
@@ -1023,6 +1122,11 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
                                 (long long)(hv >> LOG_VPR) * a.hs + c * 8;
           st_stream(a.k_cache + dst, kr);
           st_stream(a.v_cache + dst, vv[q]);
+          if (HOST_TIER && s_pk[o] != nullptr) {  // fused promotion: the stored rows
+            const long long hso = (long long)(l * H + (hv >> LOG_VPR)) * a.hot_plane + c * 8;
+            st_stream(s_pk[o] + hso, kv[q]);
+            st_stream(s_pv[o] + hso, vv[q]);
+          }
         }
       }
     };
@@ -1051,7 +1155,7 @@ __device__ __forceinline__ void run_unit(const InjectArgs& a, UnitShared<HOST_TI
 }
 
 // Persistent gather-rotate-scatter kernel.  Work unit u covers global block
-// gb = u % total_blocks and layers [lg * lpu, min(L, (lg + 1) * lpu)),
+// gb = u % total_blocks and rows [lg * rpu, min(L * H, (lg + 1) * rpu)),
 // lg = u / total_blocks, so CTAs running side by side read neighbouring
 // tokens of the same layers.  Units are taken from an atomic counter; the
 // next unit is fetched while the current one is copied.  POW2: H and B are
@@ -1074,7 +1178,7 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int total_units = a.hdr->total_units;
   const int total_blocks = a.hdr->total_blocks;
-  const int lpu = a.hdr->layers_per_unit;
+  const int rpu = a.hdr->rows_per_unit;
 
   int next = 0;
   if (tid == 0) next = int(atomicAdd(&a.hdr->next_unit, 1u));
@@ -1092,10 +1196,10 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
     const BlockDesc d = a.desc[gb];
     const int r = d.r;
     const long long tok0 = a.req_tok0[r];
-    const int l0 = lg * lpu;
+    const int w0 = lg * rpu;
     run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC, FAST>(a, sm, s_cs4, r, d.b, d.j, a.seg, a.req_off[r + 1],
                                                  a.start_pos[r], int(a.req_tok0[r + 1] - tok0), tok0,
-                                                 l0, min(a.L, l0 + lpu), lg == 0);
+                                                 w0, min(a.L * a.H, w0 + rpu), lg == 0);
   }
 }
 
@@ -1103,9 +1207,10 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
 // one kernel.  Every CTA of the persistent grid composes the batch itself in
 // shared memory -- the same definitions as plan_kernel (CSR check, lengths,
 // segment offsets, validity, token and block prefixes, work-unit size) --
-// and takes units u = blockIdx.x, blockIdx.x + gridDim.x, ...  CTA 0 alone
-// records batch- and request-level errors and the -1 slots of invalid
-// requests.  No work space, no second launch.
+// and takes units u = blockIdx.x, blockIdx.x + gridDim.x, ...  The last CTA
+// (the one a small batch leaves without units) alone records the batch's
+// errors and writes the -1 slots of invalid requests.  No work space, no
+// second launch.
 constexpr int kSmallRequests = 8;
 constexpr int kSmallIds = 256;
 
@@ -1120,7 +1225,7 @@ struct SmallPlan {
   int32_t err[kSmallRequests];
   int32_t nblk[kSmallRequests];
   int32_t blk0[kSmallRequests + 1];
-  int32_t bad, total_units, total_blocks, lpu;
+  int32_t bad, total_units, total_blocks, rpu;
 };
 
 template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0,
@@ -1133,16 +1238,31 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   __shared__ UnitShared<HOST_TIER> sm;
   __shared__ SmallPlan p;
   __shared__ int32_t s_wsum[NT / 32];
+  __shared__ unsigned long long s_err_key;
+  __shared__ unsigned int s_bad_ids;  // bit r: request r lists an id outside the store
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool reporter = blockIdx.x == 0;
+  const bool reporter = blockIdx.x == gridDim.x - 1;
 
   // Everything the plan reads from the caller is loaded at once: the CSR,
-  // the starts, the ids (then their lengths and offsets) and the frequencies.
+  // the starts, the ids and right behind them their lengths and store
+  // offsets (which need nothing but the id), and the frequencies.
   const int32_t fid = tid < num_ids ? a.fact_ids[tid] : -1;
   if (tid <= R) p.roff[tid] = a.req_off[tid];
   if (tid < R) p.start[tid] = a.start_pos[tid];
   for (int i = tid; i < D / 2; i += NT) sm.inv_freq[i] = a.inv_freq[i];
-  if (tid == 0) p.bad = 0;
+  const bool id_ok = fid >= 0 && fid < a.fact_len_count;  // false past num_ids
+  int32_t len = 0;  // length of this thread's id (0 for an id outside the store)
+  if (tid < num_ids) {
+    const int32_t lf = id_ok ? a.fact_len[fid] : -1;
+    p.off[tid] = id_ok ? a.fact_off[fid] : -1;
+    p.fid[tid] = fid;
+    p.len[tid] = lf;
+    len = id_ok ? lf : 0;
+  }
+  if (tid == 0) {
+    p.bad = 0;
+    s_bad_ids = 0u;
+  }
   // CSR: starts at 0, ends at num_ids, never decreases.
   __syncthreads();
   if ((tid < R && p.roff[tid + 1] < p.roff[tid]) || (tid == 0 && (p.roff[0] != 0 || p.roff[R] != num_ids)))
@@ -1152,17 +1272,19 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     if (reporter && tid == 0) record_error(a.st, kErrInvalidArg, -1);
     return;
   }
-  // Lengths, and their exclusive prefix over the batch (invalid ids count 0).
-  int32_t len = 0;
-  if (tid < num_ids) {
-    const int32_t f = fid;
-    const bool ok = f >= 0 && f < a.fact_len_count;
-    const int32_t lf = ok ? a.fact_len[f] : -1;
-    p.off[tid] = ok ? a.fact_off[f] : -1;
-    p.fid[tid] = f;
-    p.len[tid] = lf;
-    len = ok ? lf : 0;
+  // Warm L2 with the block-table lines of each request's first blocks (up to
+  // 128 entries), read later by every unit's slot set-up.
+  if (tid < R * 4) {
+    const int r = tid >> 2, st0 = p.start[r];
+    const int b = (st0 >= 0 ? st0 / a.B : a.max_blocks) + 32 * (tid & 3);
+    if (b < a.max_blocks)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a.block_tables + (long long)r * a.max_blocks + b));
   }
+  // This id's request; requests holding an id outside the store.
+  int myr = 0;
+  while (myr + 1 < R && p.roff[myr + 1] <= tid) ++myr;
+  if (tid < num_ids && !id_ok) atomicOr(&s_bad_ids, 1u << myr);
+  // Exclusive prefix of the lengths over the batch.
   int32_t x = len;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -1180,9 +1302,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   if (tid < R) {
     const int r = tid, j0 = p.roff[r], j1 = p.roff[r + 1];
     const long long S = p.pref[j1] - p.pref[j0];
-    int32_t err = kOk;
-    for (int j = j0; j < j1; ++j)
-      if (p.len[j] < 0) { err = kErrBadFactId; break; }
+    int32_t err = (s_bad_ids >> r) & 1u ? kErrBadFactId : kOk;
     if (err == kOk && p.start[r] < 0) err = kErrInvalidArg;
     if (err == kOk && (long long)p.start[r] + S > (long long)a.max_blocks * a.B) err = kErrPosition;
     p.err[r] = err;
@@ -1197,23 +1317,17 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     // the same limits as the two-kernel path, so results never depend on
     // which path a batch takes
     const bool over = (a.slot_out != nullptr && total_tokens > slot_cap) || acc > max_batch_blocks;
-    int32_t lpu, upb;
-    unit_size(acc, a.L, a.H, grid_ctas, lpu, upb);
-    p.lpu = lpu;
+    int32_t rpu, upb;
+    unit_size(acc, a.L, a.H, grid_ctas, FAST != 0, rpu, upb);
+    p.rpu = rpu;
     p.total_blocks = acc;
     p.total_units = over ? 0 : acc * upb;
-    if (reporter) {
-      for (int r = 0; r < R; ++r)
-        if (p.err[r] != kOk) record_error(a.st, p.err[r], r);
-      if (over) record_error(a.st, kErrCapacity, total_tokens);
-    }
+    // A batch over capacity writes nothing and reports only that.
+    if (reporter && over) record_error(a.st, kErrCapacity, total_tokens);
+    s_err_key = ~0ull;
   }
   // Segment offsets inside each request.
-  if (tid < num_ids) {
-    int r = 0;
-    while (r + 1 < R && p.roff[r + 1] <= tid) ++r;
-    p.seg[tid] = p.pref[tid] - p.pref[p.roff[r]];
-  }
+  if (tid < num_ids) p.seg[tid] = p.pref[tid] - p.pref[p.roff[myr]];
   __syncthreads();
   // -1 slots for the tokens of invalid requests (nothing at all on capacity).
   const bool over_cap =
@@ -1225,8 +1339,28 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
       for (int32_t i = tid; i < S; i += NT) a.slot_out[p.pref[p.roff[r]] + i] = -1;
     }
   }
+  // The batch's first error in request order: a request's own error, or, in
+  // a valid request, its first block-table entry outside the cache (units
+  // skip such blocks).
+  if (reporter && !over_cap) {
+    if (tid < R && p.err[tid] != kOk) atomicMin(&s_err_key, (unsigned long long)tid << 32);
+    for (int gb = tid; gb < p.total_blocks; gb += NT) {
+      int r = 0;
+      while (r + 1 < R && p.blk0[r + 1] <= gb) ++r;
+      const int b = p.start[r] / a.B + (gb - p.blk0[r]);
+      const int32_t phys = a.block_tables[(long long)r * a.max_blocks + b];
+      if (phys < 0 || phys >= a.num_blocks) atomicMin(&s_err_key, ((unsigned long long)r << 32) | unsigned(b));
+    }
+    __syncthreads();
+    if (tid == 0 && s_err_key != ~0ull) {
+      const int r = int(s_err_key >> 32);
+      const int b = int(s_err_key & 0xffffffffull);
+      if (p.err[r] != kOk) record_error(a.st, p.err[r], r);
+      else record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
+    }
+  }
 
-  const int total_units = p.total_units, total_blocks = p.total_blocks, lpu = p.lpu;
+  const int total_units = p.total_units, total_blocks = p.total_blocks, rpu = p.rpu;
   for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
     __syncthreads();  // the previous unit's tables are no longer read
     const int gb = u % total_blocks, lg = u / total_blocks;
@@ -1241,10 +1375,10 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
       const int mid = (lo + hi + 1) >> 1;
       if (p.seg[mid] <= i_first) lo = mid; else hi = mid - 1;
     }
-    const int l0 = lg * lpu;
+    const int w0 = lg * rpu;
     run_unit<D, STYLE, NT, VPT, POW2, HOST_TIER, HC, BC, FAST>(a, sm, s_cs4, r, b, lo, p.seg, j1, start,
-                                                 p.pref[j1] - p.pref[j0], p.pref[j0], l0,
-                                                 min(a.L, l0 + lpu), lg == 0, p.fid, p.off);
+                                                 p.pref[j1] - p.pref[j0], p.pref[j0], w0,
+                                                 min(a.L * a.H, w0 + rpu), lg == 0, p.fid, p.off);
   }
 }
 
@@ -1279,11 +1413,13 @@ __global__ void promote_kernel(const Promotion* __restrict__ list, int32_t n, in
   }
 }
 
-// Hot-table changes: entry pairs (fact, token offset in the hot planes or -1).
-__global__ void hot_table_kernel(int64_t* __restrict__ hot_off, const int64_t* __restrict__ pairs,
-                                 int32_t n) {
+// Hot-table changes: entry pairs (fact, token offset in the hot planes or -1)
+// applied to table t0 (n0 pairs) and table t1 (n1 pairs after them).
+__global__ void hot_table_kernel(int64_t* __restrict__ t0, int64_t* __restrict__ t1,
+                                 const int64_t* __restrict__ pairs, int32_t n0, int32_t n1) {
   const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) hot_off[pairs[2 * i]] = pairs[2 * i + 1];
+  if (i < n0) t0[pairs[2 * i]] = pairs[2 * i + 1];
+  else if (i < n0 + n1) t1[pairs[2 * i]] = pairs[2 * i + 1];
 }
 
 // RoPE frequencies, fp64: inv_freq_i = theta^(-2i/D), optionally with the

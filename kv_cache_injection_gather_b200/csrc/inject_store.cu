@@ -78,6 +78,11 @@ struct is_store {
   int64_t* d_pairs = nullptr;
   size_t promo_cap = 0;
   cudaEvent_t touch_done = nullptr;
+  // promotion fused into the next batch (is_inject_batch_host): per-fact hot
+  // token of a pending promotion (-1: none), and the pending lists' sizes
+  int64_t* d_pend = nullptr;
+  size_t pend_ne = 0, pend_np = 0;
+  bool batch_pend = false;   // the batch being launched reads d_pend
   // fact table
   int64_t* d_off = nullptr;
   int32_t* d_len = nullptr;
@@ -85,6 +90,7 @@ struct is_store {
   std::vector<int32_t> h_len;
   int64_t used_tokens = 0;
   int32_t num_facts = 0;
+  int32_t max_len = 0;        // longest fact put so far
   double* d_inv_freq = nullptr;
   // per-batch work space
   int32_t max_req = 0, max_ids = 0, max_blocks = 0;
@@ -93,7 +99,7 @@ struct is_store {
   int32_t* ws_blk0 = nullptr;
   long long* ws_tok0 = nullptr;
   int32_t* ws_len = nullptr;
-  int32_t* ws_valid = nullptr;
+  int32_t* ws_err = nullptr;
   isk::BlockDesc* ws_desc = nullptr;
   isk::PlanHeader* ws_hdr = nullptr;
   isk::DevStatus* d_status = nullptr;
@@ -118,6 +124,7 @@ struct is_store {
   int32_t* d_shard_of = nullptr;     // [shard_facts]
   int64_t* d_shard_off = nullptr;
   int32_t* d_shard_len = nullptr;
+  int32_t shard_max_len = 0;
   // kernel configuration
   int inject_grid = 0;
   int32_t small_limit = isk::kSmallRequests;  // batches up to this many requests: one kernel
@@ -166,6 +173,7 @@ void free_view(is_store* s) {
   s->d_shard_plane = s->d_shard_off = nullptr;
   s->d_shard_of = s->d_shard_len = nullptr;
   s->shard_n = s->shard_facts = 0;
+  s->shard_max_len = 0;
 }
 
 void free_store(is_store* s) {
@@ -179,7 +187,7 @@ void free_store(is_store* s) {
   cudaFree(s->ws_blk0);
   cudaFree(s->ws_tok0);
   cudaFree(s->ws_len);
-  cudaFree(s->ws_valid);
+  cudaFree(s->ws_err);
   cudaFree(s->ws_desc);
   cudaFree(s->ws_hdr);
   cudaFree(s->d_status);
@@ -194,6 +202,7 @@ void free_store(is_store* s) {
   cudaFreeHost(s->h_pairs);
   cudaFree(s->d_promo);
   cudaFree(s->d_pairs);
+  cudaFree(s->d_pend);
   if (s->touch_done) cudaEventDestroy(s->touch_done);
   if (s->host_arena) {
     cudaFreeHost(s->k);
@@ -440,7 +449,9 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
     ok = ok && (s->hot_cap == 0 ||
                 (dalloc(&s->k_hot, hot_elems) == cudaSuccess && dalloc(&s->v_hot, hot_elems) == cudaSuccess));
     ok = ok && dalloc(&s->d_hot, size_t(c.max_facts)) == cudaSuccess &&
-         cudaMemset(s->d_hot, 0xFF, sizeof(int64_t) * size_t(c.max_facts)) == cudaSuccess;
+         cudaMemset(s->d_hot, 0xFF, sizeof(int64_t) * size_t(c.max_facts)) == cudaSuccess &&
+         dalloc(&s->d_pend, size_t(c.max_facts)) == cudaSuccess &&
+         cudaMemset(s->d_pend, 0xFF, sizeof(int64_t) * size_t(c.max_facts)) == cudaSuccess;
     if (ok) s->h_hot.assign(size_t(c.max_facts), -1);
   } else {
     ok = dalloc(&s->k, arena_elems) == cudaSuccess && dalloc(&s->v, arena_elems) == cudaSuccess;
@@ -455,7 +466,7 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
             dalloc(&s->ws_blk0, size_t(s->max_req) + 1) == cudaSuccess &&
             dalloc(&s->ws_tok0, size_t(s->max_req) + 1) == cudaSuccess &&
             dalloc(&s->ws_len, size_t(s->max_req)) == cudaSuccess &&
-            dalloc(&s->ws_valid, size_t(s->max_req)) == cudaSuccess &&
+            dalloc(&s->ws_err, size_t(s->max_req)) == cudaSuccess &&
             dalloc(&s->ws_desc, size_t(s->max_blocks)) == cudaSuccess &&
             dalloc(&s->ws_hdr, 1) == cudaSuccess && dalloc(&s->d_status, 1) == cudaSuccess;
   if (!ok) {
@@ -542,6 +553,7 @@ int is_store_put_fact_window(is_store_t* s, const void* k_pre, const void* v, in
   }
   s->h_off[size_t(id)] = off;
   s->h_len[size_t(id)] = len;
+  s->max_len = std::max(s->max_len, len);
   s->num_facts = id + 1;
   s->used_tokens = off + len;
   if (fact_id_out) *fact_id_out = id;
@@ -647,6 +659,7 @@ int is_store_attach_shards(is_store_t* s, int32_t n, const void* const* k_arenas
   s->d_shard_len = nv.len;
   s->shard_n = n;
   s->shard_facts = nf;
+  s->shard_max_len = *std::max_element(fact_len, fact_len + nf);
   return IS_OK;
 }
 
@@ -759,7 +772,9 @@ int is_store_set_hot_policy(is_store_t* s, int policy, int32_t slot_tokens) {
   DeviceGuard guard(s->device);
   if (cudaDeviceSynchronize() != cudaSuccess) return IS_ERR_CUDA;  // no batch may read the old set
   // every fact cold
-  if (cudaMemset(s->d_hot, 0xFF, sizeof(int64_t) * size_t(s->cfg.max_facts)) != cudaSuccess) return IS_ERR_CUDA;
+  if (cudaMemset(s->d_hot, 0xFF, sizeof(int64_t) * size_t(s->cfg.max_facts)) != cudaSuccess ||
+      cudaMemset(s->d_pend, 0xFF, sizeof(int64_t) * size_t(s->cfg.max_facts)) != cudaSuccess)
+    return IS_ERR_CUDA;
   std::fill(s->h_hot.begin(), s->h_hot.end(), int64_t(-1));
   s->hot_used = 0;
   s->hot_facts = 0;
@@ -780,19 +795,23 @@ int is_store_set_hot_policy(is_store_t* s, int policy, int32_t slot_tokens) {
 }
 
 // LRU promotion of the listed facts: hits move to the front; misses that fit
-// a slot take the least recently used slot not used by this call.  The data
-// moves on `stream` (promote_kernel reads the mapped host arenas), then the
-// hot table is patched; later work on the stream sees the new set.
-int is_store_touch(is_store_t* s, const int32_t* fact_ids, int32_t n, void* stream, int32_t* promoted_out) {
-  if (!s || n < 0 || (n > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
-  if (!s->host_arena || s->hot_policy != IS_HOT_LRU) return IS_ERR_NOT_SUPPORTED;
-  DeviceGuard guard(s->device);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+// a slot take the least recently used slot not used by this call.
+//   fused == false: the data moves on `stream` now (promote_kernel reads the
+//     mapped host arenas), then the hot table is patched; later work on the
+//     stream sees the new set.
+//   fused == true (a batch of these ids follows on `stream`): evicted facts
+//     leave the hot table now and the promoted ones are marked pending, so
+//     the batch reads them from host memory and, as it goes, also writes
+//     their rows into their HBM slots -- each row crosses the host link once
+//     and no copy runs ahead of the batch; lru_finish then enters them in
+//     the hot table.
+static int lru_touch(is_store* s, const int32_t* fact_ids, int32_t n, cudaStream_t st, bool fused,
+                     int32_t* promoted_out) {
   // The staging of the previous touch must have been consumed.
   if (cudaEventSynchronize(s->touch_done) != cudaSuccess) return IS_ERR_CUDA;
   const uint64_t tick = ++s->tick;
   std::vector<isk::Promotion> promo;
-  std::vector<int64_t> pairs;
+  std::vector<int64_t> evict, prom;  // evicted facts; (fact, hot token) promoted
   for (int32_t i = 0; i < n; ++i) {
     const int32_t f = fact_ids[i];
     if (f < 0 || f >= s->num_facts) continue;  // the batch itself reports it
@@ -813,8 +832,7 @@ int is_store_touch(is_store_t* s, const int32_t* fact_ids, int32_t n, void* stre
     const int32_t old = s->slot_owner[size_t(slot)];
     if (old >= 0) {
       s->h_hot[size_t(old)] = -1;
-      pairs.push_back(old);
-      pairs.push_back(-1);
+      evict.push_back(old);
     } else {
       ++s->hot_facts;
     }
@@ -823,17 +841,30 @@ int is_store_touch(is_store_t* s, const int32_t* fact_ids, int32_t n, void* stre
     s->slot_tick[size_t(slot)] = tick;
     s->h_hot[size_t(f)] = dst;
     s->lru.splice(s->lru.begin(), s->lru, s->lru_at[size_t(slot)]);
-    pairs.push_back(f);
-    pairs.push_back(dst);
+    prom.push_back(f);
+    prom.push_back(dst);
     promo.push_back(isk::Promotion{s->h_off[size_t(f)], dst, s->h_len[size_t(f)], 0});
     s->lru_promoted_tokens += s->h_len[size_t(f)];
   }
   s->lru_promoted += int64_t(promo.size());
   s->hot_used = int64_t(s->hot_facts) * s->slot_tokens;
   if (promoted_out) *promoted_out = int32_t(promo.size());
+  s->pend_ne = s->pend_np = 0;
   if (promo.empty()) return IS_OK;
-  const size_t np = promo.size(), nq = pairs.size() / 2;
-  if (np > s->promo_cap || nq > s->promo_cap) {
+  // Pair lists (fact, value) for the table kernel: evictions (fact, -1),
+  // then the promotions as (fact, hot token); fused adds the promotions
+  // again (for the hot table after the batch) and as (fact, -1) (to clear
+  // their pending mark).
+  const size_t ne = evict.size(), np = promo.size();
+  std::vector<int64_t> pairs;
+  for (int64_t f : evict) { pairs.push_back(f); pairs.push_back(-1); }
+  pairs.insert(pairs.end(), prom.begin(), prom.end());
+  if (fused) {
+    pairs.insert(pairs.end(), prom.begin(), prom.end());
+    for (size_t i = 0; i < np; ++i) { pairs.push_back(prom[2 * i]); pairs.push_back(-1); }
+  }
+  const size_t nq = pairs.size() / 2;
+  if (np > s->promo_cap || nq > 2 * s->promo_cap) {
     const size_t cap = std::max(np, nq) * 2;
     cudaFreeHost(s->h_promo);
     cudaFreeHost(s->h_pairs);
@@ -845,27 +876,64 @@ int is_store_touch(is_store_t* s, const int32_t* fact_ids, int32_t n, void* stre
     s->d_pairs = nullptr;
     s->promo_cap = 0;
     if (cudaHostAlloc(reinterpret_cast<void**>(&s->h_promo), cap * sizeof(isk::Promotion), 0) != cudaSuccess ||
-        cudaHostAlloc(reinterpret_cast<void**>(&s->h_pairs), cap * 2 * sizeof(int64_t), 0) != cudaSuccess ||
-        dalloc(&s->d_promo, cap) != cudaSuccess || dalloc(&s->d_pairs, cap * 2) != cudaSuccess)
+        cudaHostAlloc(reinterpret_cast<void**>(&s->h_pairs), cap * 4 * sizeof(int64_t), 0) != cudaSuccess ||
+        dalloc(&s->d_promo, cap) != cudaSuccess || dalloc(&s->d_pairs, cap * 4) != cudaSuccess)
       return IS_ERR_OOM;
     s->promo_cap = cap;
   }
   std::memcpy(s->h_promo, promo.data(), np * sizeof(isk::Promotion));
   std::memcpy(s->h_pairs, pairs.data(), pairs.size() * sizeof(int64_t));
-  const is_store_config_t& c = s->cfg;
   if (cudaMemcpyAsync(s->d_promo, s->h_promo, np * sizeof(isk::Promotion), cudaMemcpyHostToDevice, st) !=
           cudaSuccess ||
       cudaMemcpyAsync(s->d_pairs, s->h_pairs, pairs.size() * sizeof(int64_t), cudaMemcpyHostToDevice, st) !=
           cudaSuccess)
     return IS_ERR_CUDA;
+  if (fused) {
+    isk::hot_table_kernel<<<unsigned((ne + np + 255) / 256), 256, 0, st>>>(s->d_hot, s->d_pend, s->d_pairs,
+                                                                          int32_t(ne), int32_t(np));
+    s->pend_ne = ne;
+    s->pend_np = np;
+    return cudaGetLastError() == cudaSuccess ? IS_OK : IS_ERR_CUDA;
+  }
+  const is_store_config_t& c = s->cfg;
   const int vpr = c.head_dim / 8;
   dim3 grid(unsigned(std::max(1, s->sm_count / 2)), unsigned(std::min<size_t>(np, 65535)));
   isk::promote_kernel<<<grid, 256, 0, st>>>(s->d_promo, int32_t(np), c.num_layers * c.num_kv_heads, vpr,
                                              s->k_view, s->v_view, int64_t(c.capacity_tokens) * c.head_dim,
                                              s->k_hot, s->v_hot, s->hot_cap * c.head_dim);
-  isk::hot_table_kernel<<<unsigned((nq + 255) / 256), 256, 0, st>>>(s->d_hot, s->d_pairs, int32_t(nq));
+  isk::hot_table_kernel<<<unsigned((nq + 255) / 256), 256, 0, st>>>(s->d_hot, s->d_hot, s->d_pairs,
+                                                                    int32_t(nq), 0);
   if (cudaEventRecord(s->touch_done, st) != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
   return IS_OK;
+}
+
+// After the batch of a fused touch: the pending promotions enter the hot
+// table.  A batch that did not run clean (an error skipped requests or
+// blocks, so some rows may not have been written to the slots) first copies
+// the promoted facts whole, as an unfused touch does.
+static int lru_finish(is_store* s, cudaStream_t st, bool batch_ok) {
+  if (s->pend_np == 0) return IS_OK;
+  const size_t ne = s->pend_ne, np = s->pend_np;
+  s->pend_ne = s->pend_np = 0;
+  const is_store_config_t& c = s->cfg;
+  if (!batch_ok) {
+    dim3 grid(unsigned(std::max(1, s->sm_count / 2)), unsigned(std::min<size_t>(np, 65535)));
+    isk::promote_kernel<<<grid, 256, 0, st>>>(s->d_promo, int32_t(np), c.num_layers * c.num_kv_heads,
+                                               c.head_dim / 8, s->k_view, s->v_view,
+                                               int64_t(c.capacity_tokens) * c.head_dim, s->k_hot, s->v_hot,
+                                               s->hot_cap * c.head_dim);
+  }
+  isk::hot_table_kernel<<<unsigned((2 * np + 255) / 256), 256, 0, st>>>(
+      s->d_hot, s->d_pend, s->d_pairs + 2 * (ne + np), int32_t(np), int32_t(np));
+  if (cudaEventRecord(s->touch_done, st) != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
+  return IS_OK;
+}
+
+int is_store_touch(is_store_t* s, const int32_t* fact_ids, int32_t n, void* stream, int32_t* promoted_out) {
+  if (!s || n < 0 || (n > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
+  if (!s->host_arena || s->hot_policy != IS_HOT_LRU) return IS_ERR_NOT_SUPPORTED;
+  DeviceGuard guard(s->device);
+  return lru_touch(s, fact_ids, n, static_cast<cudaStream_t>(stream), false, promoted_out);
 }
 
 int is_store_lru_stats(const is_store_t* s, int64_t* hits, int64_t* misses, int64_t* promoted,
@@ -917,10 +985,14 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.fact_ids = fact_ids;
   pa.num_ids = num_ids;
   pa.start_pos = start_pos;
+  pa.block_tables = block_tables;
   pa.max_blocks = max_blocks_per_req;
+  pa.num_blocks = c.num_blocks;
   pa.B = c.block_size;
   pa.L = cf.num_layers;
   pa.H = cf.num_kv_heads;
+  pa.chk_off = nullptr;  // the library's own fact table
+  pa.chk_plane = 0;
   // With a sharded view attached, ids are global: the view's fact table.
   const bool view = s->shard_n > 0;
   const int32_t nfacts = view ? s->shard_facts : s->num_facts;
@@ -929,17 +1001,25 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.slot_out = slot_out;
   pa.slot_cap = slot_cap;
   pa.grid_ctas = s->inject_grid;
+  // The per-thread copy loops of the common shapes take any (layer, head)
+  // row range as a unit; the generic loop takes whole layers.
+  const int loop = launch_loop(cf.head_dim, c.block_size, cf.num_kv_heads);
+  pa.row_units = loop != 0;
   pa.max_batch_blocks = s->max_blocks;
   pa.seg = s->ws_seg;
   pa.req_nblk = s->ws_nblk;
   pa.req_blk0 = s->ws_blk0;
   pa.req_tok0 = s->ws_tok0;
   pa.req_len = s->ws_len;
-  pa.req_valid = s->ws_valid;
+  pa.req_err = s->ws_err;
   pa.desc = s->ws_desc;
   pa.hdr = s->ws_hdr;
   pa.st = s->d_status;
-  const bool small = R <= s->small_limit && num_ids <= isk::kSmallIds;
+  // The single-kernel path sums a batch's lengths in 32 bits: only batches
+  // whose ids cannot total more than 2^31 - 1 tokens take it.
+  const int64_t longest = view ? s->shard_max_len : s->max_len;
+  const bool small = R <= s->small_limit && num_ids <= isk::kSmallIds &&
+                     int64_t(num_ids) * longest <= int64_t(0x7fffffff);
   if (!small) {
     if (R <= isk::kPlanSmemRequests && num_ids <= isk::kPlanSmemIds)
       isk::plan_kernel<kPlanThreads, true><<<1, kPlanThreads, isk::plan_smem_bytes(R, num_ids), st>>>(pa);
@@ -954,6 +1034,9 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.v_hot = s->v_hot;
   ia.hot_plane = s->hot_cap * cf.head_dim;
   ia.hot_off = s->d_hot;
+  ia.pend = s->batch_pend ? s->d_pend : nullptr;
+  ia.k_prom = s->k_hot;
+  ia.v_prom = s->v_hot;
   ia.plane = int64_t(cf.capacity_tokens) * cf.head_dim;
   ia.fact_off = view ? s->d_shard_off : s->d_off;
   ia.fact_len = view ? s->d_shard_len : s->d_len;
@@ -987,7 +1070,6 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.fact_len_count = nfacts;
   // Per-slot sources: the host tier, or the arenas of a sharded view.
   const bool per_slot = s->host_arena || view;
-  const int loop = launch_loop(cf.head_dim, c.block_size, cf.num_kv_heads);
   void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop)
                    : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop);
   int32_t small_R = R, small_ids = num_ids, small_grid = s->inject_grid, small_blocks = s->max_blocks;
@@ -1047,8 +1129,9 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
   const int64_t n_slots = slot_out ? slot_cap : 0;
   int rc = grow_stage(s, n_off + n_ids + n_sp + n_bt + 4, n_slots);
   if (rc != IS_OK) return rc;
-  if (s->hot_policy == IS_HOT_LRU) {  // promote this batch's cold facts first
-    rc = is_store_touch(s, fact_ids, num_ids, stream, nullptr);
+  const bool lru = s->hot_policy == IS_HOT_LRU;
+  if (lru) {  // this batch's cold facts: promotions fused into the batch
+    rc = lru_touch(s, fact_ids, num_ids, st, true, nullptr);
     if (rc != IS_OK) return rc;
   }
   // Pack the four index arrays into one pinned buffer: one host-to-device copy.
@@ -1061,11 +1144,18 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
   int32_t* d_ids = d_off + n_off;
   int32_t* d_sp = d_ids + n_ids;
   int32_t* d_bt = d_sp + n_sp;
-  if (cudaMemcpyAsync(d_off, h, (n_off + n_ids + n_sp + n_bt) * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  if (cudaMemcpyAsync(d_off, h, (n_off + n_ids + n_sp + n_bt) * 4, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    lru_finish(s, st, false);
     return IS_ERR_CUDA;
+  }
+  s->batch_pend = s->pend_np > 0;
   rc = is_inject_batch(s, R, d_off, d_ids, num_ids, d_sp, d_bt, max_blocks_per_req, cache,
                        slot_out ? s->stage_slots : nullptr, slot_cap, stream);
-  if (rc != IS_OK) return rc;
+  s->batch_pend = false;
+  if (rc != IS_OK) {
+    lru_finish(s, st, false);  // nothing ran: copy the promoted facts instead
+    return rc;
+  }
   if (slot_out && slot_cap > 0 &&
       cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost, st) !=
           cudaSuccess)
@@ -1076,6 +1166,8 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
       cudaStreamSynchronize(st) != cudaSuccess)
     return IS_ERR_CUDA;
   const int code = s->host_status->code;
+  if (s->pend_np > 0 && (lru_finish(s, st, code == 0) != IS_OK || cudaStreamSynchronize(st) != cudaSuccess))
+    return IS_ERR_CUDA;
   if (code != 0 && cudaMemset(s->d_status, 0, sizeof(isk::DevStatus)) != cudaSuccess) return IS_ERR_CUDA;
   return code;
 }
@@ -1162,8 +1254,8 @@ constexpr size_t kNaNblk = align256(kNaSeg + sizeof(int32_t) * IS_NOALLOC_MAX_FA
 constexpr size_t kNaBlk0 = align256(kNaNblk + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
 constexpr size_t kNaTok0 = align256(kNaBlk0 + sizeof(int32_t) * (IS_NOALLOC_MAX_REQUESTS + 1));
 constexpr size_t kNaLen = align256(kNaTok0 + sizeof(long long) * (IS_NOALLOC_MAX_REQUESTS + 1));
-constexpr size_t kNaValid = align256(kNaLen + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
-constexpr size_t kNaDesc = align256(kNaValid + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
+constexpr size_t kNaErr = align256(kNaLen + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
+constexpr size_t kNaDesc = align256(kNaErr + sizeof(int32_t) * IS_NOALLOC_MAX_REQUESTS);
 constexpr size_t kNaBytes = align256(kNaDesc + sizeof(isk::BlockDesc) * IS_NOALLOC_MAX_BLOCKS);
 
 constexpr int kNaMaxDevices = 64;
@@ -1288,22 +1380,29 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   pa.fact_ids = fact_ids;
   pa.num_ids = num_ids;
   pa.start_pos = start_pos;
+  pa.block_tables = block_tables;
   pa.max_blocks = max_blocks_per_req;
+  pa.num_blocks = k.num_blocks;
   pa.B = k.block_size;
   pa.L = c.num_layers;
   pa.H = c.num_kv_heads;
   pa.fact_len = fact_lens;
   pa.num_facts = num_facts;
+  // The caller's fact table: ids whose entry leaves the arenas are refused.
+  pa.chk_off = fact_offsets;
+  pa.chk_plane = plane_tokens;
   pa.slot_out = slot_out;
   pa.slot_cap = slot_cap;
   pa.grid_ctas = grid;
+  const int loop = launch_loop(c.head_dim, k.block_size, c.num_kv_heads);
+  pa.row_units = loop != 0;
   pa.max_batch_blocks = IS_NOALLOC_MAX_BLOCKS;
   pa.seg = reinterpret_cast<int32_t*>(ws + kNaSeg);
   pa.req_nblk = reinterpret_cast<int32_t*>(ws + kNaNblk);
   pa.req_blk0 = reinterpret_cast<int32_t*>(ws + kNaBlk0);
   pa.req_tok0 = reinterpret_cast<long long*>(ws + kNaTok0);
   pa.req_len = reinterpret_cast<int32_t*>(ws + kNaLen);
-  pa.req_valid = reinterpret_cast<int32_t*>(ws + kNaValid);
+  pa.req_err = reinterpret_cast<int32_t*>(ws + kNaErr);
   pa.desc = reinterpret_cast<isk::BlockDesc*>(ws + kNaDesc);
   pa.hdr = hdr;
   pa.st = status;
@@ -1331,15 +1430,15 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   ia.hs = k.head_stride;
   ia.num_blocks = k.num_blocks;
   ia.B = k.block_size;
-  ia.vec_order = vec_order_for(k.token_stride, k.head_stride);
+  ia.vec_order = launch_vec_order(c.head_dim, k.block_size, c.num_kv_heads, k.token_stride, k.head_stride);
   ia.slot_out = slot_out;
   ia.seg = pa.seg;
   ia.req_tok0 = pa.req_tok0;
   ia.desc = pa.desc;
   ia.hdr = hdr;
   ia.st = status;
-  void* fn = pick_inject(c.head_dim, c.rope_style, c.num_kv_heads, k.block_size, false,
-                         ia.vec_order);  // loop 1 (per-thread) on slot-fastest orders, else 0
+  // The kernel variant is_inject_batch launches for the same shape and layout.
+  void* fn = pick_inject(c.head_dim, c.rope_style, c.num_kv_heads, k.block_size, false, loop);
   void* args[] = {&ia};
   if (cudaLaunchKernel(fn, dim3(unsigned(grid)), dim3(kInjectThreads), args,
                        cs_smem_bytes(c.head_dim, k.block_size), st) != cudaSuccess)

@@ -146,3 +146,34 @@ def test_lru_eviction_keeps_results_exact():
         assert_parity(oracle_run(wl), _host_inject(store, wl))
     assert store.lru_stats()["promoted"] > 5
     store.close()
+
+
+def test_lru_promotion_survives_a_batch_with_errors():
+    """The host entry point fuses each batch's promotions into the batch (the
+    kernel writes the promoted facts' rows into their HBM slots as it reads
+    them from host memory).  A batch with a bad block-table entry skips some
+    rows, so the library copies its promoted facts whole instead; the next
+    batches, reading those facts from HBM through either entry point, must
+    still equal the oracle."""
+    _need_gpu()
+    model = synth.Model("llama-like", 2, 8, 128, 5e5, llama3=True)
+    wl = _ragged(model, seed=47, R=5, max_k=8, lens=(1, 30), num_facts=30)
+    b = wl.batch
+    store = make_store(wl, host_tier=True, hot_capacity_tokens=32 * 40)
+    store.set_hot_policy(True, 32)
+    bad_bt = b.block_tables.copy()
+    r = int(np.argmax(np.diff(b.req_offsets) > 0))        # a request with facts
+    bad_bt[r, int(b.start_pos[r]) // b.block_size] = b.num_blocks + 5
+    bad = synth.Workload(wl.name, model, wl.fact_lens,
+                         synth.Batch(b.req_offsets, b.fact_ids, b.start_pos, bad_bt, b.block_size,
+                                     b.num_blocks), wl.seed)
+    o_bad = oracle_run(bad)
+    assert o_bad[0] == oracle.ERR_BAD_BLOCK
+    assert_parity(o_bad, _host_inject(store, bad))
+    promoted = store.lru_stats()["promoted"]
+    assert promoted >= 1
+    want = oracle_run(wl)
+    assert_parity(want, _host_inject(store, wl))           # hot now: read from HBM
+    assert store.lru_stats()["promoted"] == promoted       # nothing left to promote
+    assert_parity(want, gpu_run(wl, store=store))          # device entry point, same hot set
+    store.close()

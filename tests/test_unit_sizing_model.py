@@ -1,14 +1,17 @@
 """The work-unit sizing rule of the inject kernels (unit_size in
 kv_cache_injection_gather_b200/csrc/inject_kernels.cuh, transcribed here with
 its default knobs) checked for the properties the kernels and their
-documentation rely on, over far more shapes than the GPU tests run:
+documentation rely on, over far more shapes than the GPU tests run.  A unit
+covers (layer, head) rows [g * rpu, min(L * H, (g + 1) * rpu)) of one cache
+block, row = layer * H + head:
 
-  * the layer ranges of a block's units partition [0, L), none empty;
+  * the row ranges of a block's units partition [0, L * H), none empty;
+  * without row units (the generic copy loop) every range is whole layers;
   * a batch whose one-layer units fit in two waves gets about one wave of
-    units (latency): at most the grid plus one unit per block, since layers
-    are grouped in equal ranges;
-  * a large batch gets units of at least 16 (layer, head) rows and two
-    layers whenever the model has them;
+    units (latency): at most the grid plus one unit per block, since rows
+    (or layers) are grouped in equal ranges;
+  * a large batch gets units of whole layers, at least 16 rows and two
+    layers whenever the model has them, with or without row units;
   * the unit count fits the kernels' 32-bit counters.
 """
 from __future__ import annotations
@@ -18,7 +21,13 @@ import itertools
 UNITS_PER_CTA, MIN_ROWS, ROWS_LARGE, UNITS_PER_CTA_MIN = 256, 16, 32, 32
 
 
-def unit_size(total_blocks: int, L: int, H: int, grid: int) -> tuple[int, int]:
+def unit_size(total_blocks: int, L: int, H: int, grid: int, row_units: bool = False):
+    LH = L * H
+    if total_blocks > 0 and row_units and total_blocks * L <= 2 * grid:
+        per = (total_blocks * LH + grid - 1) // grid
+        upb = (LH + per - 1) // per
+        rpu = (LH + upb - 1) // upb
+        return rpu, (LH + rpu - 1) // rpu
     upb = 1
     if total_blocks > 0 and total_blocks * L <= 2 * grid:
         per = (total_blocks * L + grid - 1) // grid
@@ -33,34 +42,41 @@ def unit_size(total_blocks: int, L: int, H: int, grid: int) -> tuple[int, int]:
         upb = max(1, min(want, cap))
     lpu = (L + upb - 1) // upb
     upb = (L + lpu - 1) // lpu
-    return lpu, upb
+    return lpu * H, upb
 
 
 def test_unit_sizing_invariants():
     grids = (296, 444, 148)
     layers = (1, 2, 3, 5, 12, 16, 28, 32, 40, 61, 80)
     heads = (1, 2, 3, 4, 8, 16)
-    blocks = (1, 2, 5, 9, 10, 37, 100, 147, 148, 296, 297, 592, 1000, 4625, 12_600, 65_536,
+    blocks = (1, 2, 5, 9, 10, 13, 37, 100, 147, 148, 296, 297, 592, 1000, 4625, 12_600, 65_536,
               1 << 20)
-    for grid, L, H, tb in itertools.product(grids, layers, heads, blocks):
-        lpu, upb = unit_size(tb, L, H, grid)
-        assert 1 <= lpu <= L and 1 <= upb <= L
-        ranges = [(g * lpu, min(L, (g + 1) * lpu)) for g in range(upb)]
-        assert all(a < b for a, b in ranges), (grid, L, H, tb, lpu, upb)
-        assert ranges[0][0] == 0 and ranges[-1][1] == L
+    for grid, L, H, tb, rows in itertools.product(grids, layers, heads, blocks, (False, True)):
+        LH = L * H
+        rpu, upb = unit_size(tb, L, H, grid, rows)
+        assert 1 <= rpu <= LH and 1 <= upb <= LH
+        ranges = [(g * rpu, min(LH, (g + 1) * rpu)) for g in range(upb)]
+        assert all(a < b for a, b in ranges), (grid, L, H, tb, rpu, upb)
+        assert ranges[0][0] == 0 and ranges[-1][1] == LH
         assert all(ranges[i][1] == ranges[i + 1][0] for i in range(upb - 1))
+        if not rows:
+            assert all(a % H == 0 and (b % H == 0) for a, b in ranges), "whole layers"
         if tb * L <= 2 * grid:
             assert tb * upb <= grid + tb, "one-wave batch: about one wave of units"
         else:
-            assert lpu >= min(L, 2)
-            assert lpu * H >= min(MIN_ROWS, L * H) or lpu == L
+            assert rpu % H == 0, "large batches: whole layers"
+            assert rpu // H >= min(L, 2)
+            assert rpu >= min(MIN_ROWS, LH) or rpu == LH
+            assert unit_size(tb, L, H, grid, not rows) == (rpu, upb)
         assert tb * upb < 2 ** 31
 
 
 def test_unit_sizing_at_the_benchmark_shapes():
     # Llama-3.1-8B batch: ~12.6k touched blocks, 32 layers, 8 heads -> units of 6 layers
-    assert unit_size(12_633, 32, 8, 296) == (6, 6)
+    assert unit_size(12_633, 32, 8, 296, True) == (48, 6)
     # Qwen2.5-7B, R=100 k=20: ~4.6k blocks, 4 heads -> 10-layer units (32-row rule)
-    assert unit_size(4_625, 28, 4, 296) == (10, 3)
-    # one Llama request of 10 blocks: one wave, two layers per unit
-    assert unit_size(10, 32, 8, 296) == (2, 16)
+    assert unit_size(4_625, 28, 4, 296, True) == (40, 3)
+    # one Llama request of 10 blocks: one wave; whole layers give 160 units of
+    # two layers, row units 290 units of 9 rows
+    assert unit_size(10, 32, 8, 296) == (16, 16)
+    assert unit_size(10, 32, 8, 296, True) == (9, 29)
