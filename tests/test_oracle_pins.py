@@ -82,6 +82,33 @@ def test_bf16_matches_torch_on_fp32_inputs():
     assert np.array_equal(ours, theirs)
 
 
+def test_bf16_special_values_and_overflow():
+    """Outside the finite range: signed zeros keep their sign, infinities map
+    to themselves, a NaN stays a NaN (quiet), and the overflow threshold of
+    round-to-nearest-even is the midpoint between the largest finite bf16
+    (2^128 - 2^120) and 2^128 -- the tie rounds up to the infinity, whose
+    mantissa is the even one.  torch's fp32 -> bf16 (an independent
+    implementation) agrees on fp32 inputs next to the threshold, at the
+    subnormal end and on the specials."""
+    b = oracle.f64_to_bf16(np.array([0.0, -0.0, np.inf, -np.inf, np.nan, -np.nan]))
+    assert list(b[:4]) == [0x0000, 0x8000, 0x7F80, 0xFF80]
+    for x in b[4:]:
+        assert (x & 0x7F80) == 0x7F80 and (x & 0x007F) != 0 and (x & 0x0040), hex(x)
+    top = 2.0 ** 128 - 2.0 ** 120
+    mid = 2.0 ** 128 - 2.0 ** 119
+    xs = np.array([top, np.nextafter(mid, 0.0), mid, np.nextafter(mid, np.inf), 2.0 ** 128, 1e300,
+                   -np.nextafter(mid, 0.0), -mid])
+    assert list(oracle.f64_to_bf16(xs)) == [0x7F7F, 0x7F7F, 0x7F80, 0x7F80, 0x7F80, 0x7F80,
+                                             0xFF7F, 0xFF80]
+    import torch
+    f32 = np.array([3.38e38, 3.3953e38, 3.3961e38, 3.3962e38, 3.4e38, np.finfo(np.float32).max,
+                    -3.3962e38, 1e-45, -1e-45, 9.2e-41, 1.17e-38, 2.0 ** -133, 3 * 2.0 ** -134,
+                    0.0, -0.0, np.inf, -np.inf], np.float32)
+    ours = oracle.f64_to_bf16(f32.astype(np.float64))
+    theirs = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, theirs), (ours, theirs)
+
+
 # --------------------------------------------------------------- RoPE frequencies
 
 @pytest.mark.parametrize("D,theta", [(64, 1.0e4), (128, 5.0e5), (128, 1.0e6), (4, 100.0)])
@@ -204,6 +231,40 @@ def test_rope_is_a_power_of_the_unit_step(style):
         want = np.linalg.matrix_power(R1, p) @ x
         got = oracle.rope_rows(x[None], [p], f, style)[0]
         assert np.allclose(got, want, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("style", [oracle.ROTATE_HALF, oracle.INTERLEAVED])
+def test_rope_non_finite_inputs_follow_ieee_pairwise(style):
+    """A NaN or an infinity in a key changes only its own rotation pair, and
+    within it follows IEEE arithmetic of x cos - y sin, y cos + x sin: a NaN
+    makes both members NaN; an infinity with a finite partner gives
+    infinities signed by cos and sin, except that at position 0 the partner
+    becomes inf * sin 0 = NaN."""
+    D = 16
+    f = oracle.rope_inv_freq(D, 1e4)
+    pair = (lambda i: (i, i + D // 2)) if style == oracle.ROTATE_HALF else (lambda i: (2 * i, 2 * i + 1))
+    rng = np.random.default_rng(9)
+    base = rng.standard_normal(D)
+    for pos in (0, 3, 1000):
+        clean = oracle.rope_rows(base[None], [pos], f, style)[0]
+        for i, val in ((2, np.nan), (5, np.inf), (6, -np.inf)):
+            a, b = pair(i)
+            x = base.copy()
+            x[a] = val
+            y = oracle.rope_rows(x[None], [pos], f, style)[0]
+            others = np.ones(D, bool)
+            others[[a, b]] = False
+            assert np.array_equal(y[others], clean[others])
+            ang = pos * f[i]
+            c, s_ = math.cos(ang), math.sin(ang)
+            if np.isnan(val):
+                assert np.isnan(y[a]) and np.isnan(y[b])
+            else:
+                assert y[a] == val * np.sign(c)
+                if pos == 0:
+                    assert np.isnan(y[b])
+                else:
+                    assert y[b] == val * np.sign(s_)
 
 
 def test_rope_group_laws_and_norm():

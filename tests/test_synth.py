@@ -1,5 +1,6 @@
-"""The seeded input generator: determinism, independence of streams and the
-shape of its distributions (CPU)."""
+"""The seeded input generator: determinism, independence of streams, the
+normal distribution of its bulk values and the shapes of the workloads
+(CPU)."""
 import numpy as np
 
 import synth
@@ -16,12 +17,48 @@ def test_counter_based_and_deterministic():
     assert not np.array_equal(a, synth.bf16_bits(0, 6, np.arange(1000)))
 
 
-def test_roughly_standard_normal():
-    x = synth.bf16_to_float(synth.bf16_bits(3, 1, np.arange(200_000))).astype(np.float64)
-    assert abs(x.mean()) < 0.01 and abs(x.std() - 1.0) < 0.01
-    assert np.abs(x).max() <= 6.0
-    # tails close to the normal's: P(|x| > 2) ~ 0.0455
-    assert 0.040 < np.mean(np.abs(x) > 2) < 0.050
+def test_threshold_table_is_the_normal_distribution():
+    """Q_c / 2^64 = P(|X| < h_c) for X ~ N(0, 1), h_c the midpoint between
+    bf16 codes c and c + 1: checked against scipy's normal distribution (an
+    independent implementation) to 1e-15 absolute, and non-decreasing."""
+    from scipy.stats import norm
+    first, q = synth.normal_table()
+    assert np.all(q[1:] >= q[:-1]) and q[0] > 0
+    codes = np.arange(first, first + len(q), dtype=np.uint32)
+    lo = (codes << 16).view(np.float32).astype(np.float64)
+    hi = ((codes + 1) << 16).view(np.float32).astype(np.float64)
+    h = 0.5 * (lo + hi)
+    want = np.where(h <= 1.0, 2.0 * norm.cdf(h) - 1.0, 1.0 - 2.0 * norm.sf(h))
+    assert np.max(np.abs(q.astype(np.float64) / 2.0 ** 64 - want)) < 1e-15
+    # the support: from below 2^-64 up to about 9.1
+    assert lo[0] < 2.0 ** -64 and 9.0 < hi[-1] < 9.5
+
+
+def test_standard_normal_samples():
+    """Two million samples: symmetric, unit variance, and the counts of |x|
+    in bins agree with N(0, 1) rounded to bf16 (chi-square, 11 bins; the
+    expected counts from scipy at the bf16 rounding midpoints of the bin
+    edges)."""
+    from scipy.stats import chi2, norm
+    bits = synth.bf16_bits(3, 1, np.arange(2_000_000))
+    x = synth.bf16_to_float(bits).astype(np.float64)
+    assert abs(x.mean()) < 0.003 and abs(x.std() - 1.0) < 0.003
+    assert abs(np.mean(bits >> 15) - 0.5) < 0.002
+    assert np.abs(x).max() > 4.5
+    edges = np.array([0.0, 0.125, 0.25, 0.5, 0.75, 1.0, 1.5, 2.0, 2.5, 3.0, 4.0, np.inf])
+    # a rounded value lands in [e_i, e_(i+1)) exactly when |X| lies in
+    # [m(e_i), m(e_(i+1))), m(e) the midpoint between the bf16 value e and
+    # the next one below: e - 2^(k-8) for e in (2^k, 2^(k+1)), e - 2^(k-9)
+    # for e = 2^k (the spacing halves below a power of two)
+    def mid_below(e):
+        k = np.floor(np.log2(e))
+        return e - 2.0 ** (k - 9 if e == 2.0 ** k else k - 8)
+
+    below = np.array([0.0] + [mid_below(e) for e in edges[1:-1]] + [np.inf])
+    p = 2.0 * (norm.cdf(below[1:]) - norm.cdf(below[:-1]))
+    n = np.histogram(np.abs(x), bins=edges)[0]
+    stat = float(((n - p * len(x)) ** 2 / (p * len(x))).sum())
+    assert stat < chi2.ppf(0.9995, len(p) - 1), stat
 
 
 def test_fact_rows_match_fact_tensor():
