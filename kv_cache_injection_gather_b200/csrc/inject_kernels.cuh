@@ -724,18 +724,45 @@ __device__ __forceinline__ uint4 rotate_vec(const uint4 own, int c, const float4
   return rotate_regs<D, STYLE>(own, c, t);
 }
 
-// cos and sin of an fp64 RoPE angle: reduced to [-pi, pi] by the nearest
-// multiple of 2*pi (one fused multiply-add in fp64; for positions below 2^31
-// the reduction is off by < 1e-7 rad, the fp64 angle itself by < 3e-7 rad),
-// then the hardware single-precision sin/cos of the reduced angle (absolute
-// error below 2^-21.4 on [-pi, pi]; the values are kept in fp32 anyway).  The
-// hardware form is used only on the reduced angle: on the raw angle (up to
-// ~2e9 rad) it would be far off.
+// cos and sin of an fp64 RoPE angle, each the fp32 rounding of the fp64
+// value (to within ~1e-15), so small ones are as accurate relatively as large
+// ones: a key element near 0 rotates to its partner times the sine exactly as
+// the oracle rounds it.  The angle is reduced to r in [-pi/4, pi/4] and a
+// quadrant q, ang = q * pi/2 + r, by Cody and Waite's additive reduction in
+// fp64 (pi/2 split into the nearest double and its remainder; each product is
+// exact inside its fused multiply-add; exact to < 1e-15 rad for positions
+// below 2^31).  sin r and cos r are their Taylor series through r^13 and r^14
+// (the first neglected terms are below 3e-14 on [-pi/4, pi/4]) by Horner's
+// rule in fp64, then the quadrant swaps and negates: sin(q pi/2 + r) = sin r,
+// cos r, -sin r, -cos r for q = 0..3, cos alike shifted by one.
 __device__ __forceinline__ void rope_cos_sin(double ang, float& c, float& s) {
-  constexpr double kTwoPi = 6.283185307179586476925286766559;
-  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-  const double k = rint(ang * kInvTwoPi);
-  __sincosf(float(fma(-k, kTwoPi, ang)), &s, &c);
+  constexpr double kTwoOverPi = 0.63661977236758134307553505349005745;
+  constexpr double kPiOver2Hi = 1.5707963267948965579989817342720925;   // nearest double to pi/2
+  constexpr double kPiOver2Lo = 6.1232339957367660359e-17;               // pi/2 - kPiOver2Hi
+  const double k = rint(ang * kTwoOverPi);
+  const double r = fma(-k, kPiOver2Lo, fma(-k, kPiOver2Hi, ang));
+  const double z = r * r;
+  // sin r = r (1 - z/3! + z^2/5! - ... + z^6/13!)
+  double ps = 1.0 / 6227020800.0;
+  ps = fma(ps, z, -1.0 / 39916800.0);
+  ps = fma(ps, z, 1.0 / 362880.0);
+  ps = fma(ps, z, -1.0 / 5040.0);
+  ps = fma(ps, z, 1.0 / 120.0);
+  ps = fma(ps, z, -1.0 / 6.0);
+  ps = fma(ps, z, 1.0);
+  // cos r = 1 - z/2! + z^2/4! - ... - z^7/14!
+  double pc = -1.0 / 87178291200.0;
+  pc = fma(pc, z, 1.0 / 479001600.0);
+  pc = fma(pc, z, -1.0 / 3628800.0);
+  pc = fma(pc, z, 1.0 / 40320.0);
+  pc = fma(pc, z, -1.0 / 720.0);
+  pc = fma(pc, z, 1.0 / 24.0);
+  pc = fma(pc, z, -0.5);
+  pc = fma(pc, z, 1.0);
+  const float sr = float(r * ps), cr = float(pc);
+  const int q = int((long long)k & 3);
+  s = (q == 0) ? sr : (q == 1) ? cr : (q == 2) ? -sr : -cr;
+  c = (q == 0) ? cr : (q == 1) ? -sr : (q == 2) ? -cr : sr;
 }
 
 constexpr int kMaxBlockSize = 128;

@@ -3,9 +3,10 @@ configuration: Llama-3.1-8B shapes (32 layers, 8 KV heads, D=128, llama3
 RoPE scaling), 10k facts of 16-64 tokens (about 52 GB of store), 100
 requests x k=50 distinct facts after a 64-token prefix, 25 600-block cache
 (53.7 GB of K and V), token-major and head-major.  The oracle cannot hold
-the cache, so the checks are those of fullsize_check: every slot, every V
-row, K of one whole request plus 20 000 random rows, every untouched
-element.
+the whole cache, so fullsize_check streams the batch request by request:
+every slot, every row -- each (token, layer, head) row of K and V against
+the oracle's injection of that request from regenerated inputs -- and every
+untouched element.
 """
 from __future__ import annotations
 
@@ -14,7 +15,7 @@ import torch
 
 import synth
 from fullsize_check import check_full_size
-from gpu_common import make_store
+from synth.device import make_store
 
 pytestmark = pytest.mark.gpu
 

@@ -1,5 +1,7 @@
 """Full-size parity at the other large configurations, in the launch
-configuration the benchmark times (the checks of fullsize_check):
+configuration the benchmark times (the checks of fullsize_check: every slot,
+every row of K and V against the oracle request by request, every untouched
+element):
 
   * Qwen2.5-7B shapes, 50k-fact store (~103 GB), 256 requests x k=50;
   * Mistral-7B shapes, 20k-fact store (~95 GB: 50k would not fit in HBM),
@@ -17,7 +19,7 @@ import torch
 
 import synth
 from fullsize_check import check_full_size
-from gpu_common import make_store
+from synth.device import make_store
 
 pytestmark = pytest.mark.gpu
 
