@@ -317,6 +317,27 @@ int is_inject_batch_host(is_store_t* store, int32_t num_requests,
                          const is_cache_t* cache, int64_t* slot_mapping_out,
                          int64_t slot_mapping_capacity, void* stream);
 
+/* is_inject_batch_host for a stream of batches on a host-tier store with the
+ * LRU hot set (IS_HOT_LRU): the same batch, and, while it runs, the cold
+ * facts of the NEXT batch (next_fact_ids, host array, num_next_ids entries;
+ * the caller's retrieval knows them before their injection) start moving
+ * into HBM slots by copy-engine transfers on a stream of the store -- slots
+ * not used by this batch, in least-recently-used order -- so that batch
+ * reads them from HBM (technical summary, Results, "Scalability": the KV
+ * store may live in host DRAM; this is its prefetch path).  Every later
+ * batch on the store waits for those transfers.  Ids that do not come or
+ * are outside the store only cost their transfer; results never depend on
+ * the prefetch.  On a store without the LRU policy the next ids are
+ * ignored.  Errors as for is_inject_batch_host, and INVALID_ARG for
+ * num_next_ids < 0 or a NULL list. */
+int is_inject_batch_host_next(is_store_t* store, int32_t num_requests,
+                              const int32_t* req_fact_offsets, const int32_t* fact_ids,
+                              int32_t num_fact_ids, const int32_t* start_pos,
+                              const int32_t* block_tables, int32_t max_blocks_per_req,
+                              const is_cache_t* cache, int64_t* slot_mapping_out,
+                              int64_t slot_mapping_capacity, const int32_t* next_fact_ids,
+                              int32_t num_next_ids, void* stream);
+
 /* Wait for `stream`, then return and clear the first device-side error
  * recorded since the previous call (IS_OK if none).  *detail_out, if not
  * NULL, receives the offending index (request, CSR entry or block). */

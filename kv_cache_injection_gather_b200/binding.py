@@ -92,6 +92,9 @@ _SIGNATURES = {
                                        ctypes.POINTER(is_cache_t), _P, _I64, _P]),
     "is_inject_batch_host": (ctypes.c_int, [_P, _I32, _P, _P, _I32, _P, _P, _I32,
                                             ctypes.POINTER(is_cache_t), _P, _I64, _P]),
+    "is_inject_batch_host_next": (ctypes.c_int, [_P, _I32, _P, _P, _I32, _P, _P, _I32,
+                                                 ctypes.POINTER(is_cache_t), _P, _I64, _P, _I32,
+                                                 _P]),
     "is_last_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(_I64)]),
     "is_last_error_timeout": (ctypes.c_int, [_P, _P, _I32, ctypes.POINTER(_I64)]),
     "is_store_set_timing": (ctypes.c_int, [_P, ctypes.c_int]),
@@ -258,6 +261,22 @@ def is_inject_batch_host(store: int, num_requests: int, req_fact_offsets: int, f
                                      num_fact_ids, start_pos, block_tables, max_blocks_per_req,
                                      ctypes.byref(cache), slot_mapping_out,
                                      slot_mapping_capacity, stream)
+
+
+def is_inject_batch_host_next(store: int, num_requests: int, req_fact_offsets: int,
+                              fact_ids: int, num_fact_ids: int, start_pos: int,
+                              block_tables: int, max_blocks_per_req: int, cache: is_cache_t,
+                              slot_mapping_out: int | None, slot_mapping_capacity: int,
+                              next_fact_ids: int | None, num_next_ids: int,
+                              stream: int = 0) -> int:
+    """is_inject_batch_host, and on an LRU host-tier store the next batch's
+    cold facts (host array) start moving into HBM while this batch runs.
+    Returns the batch status without raising."""
+    return _lib.is_inject_batch_host_next(store, num_requests, req_fact_offsets, fact_ids,
+                                          num_fact_ids, start_pos, block_tables,
+                                          max_blocks_per_req, ctypes.byref(cache),
+                                          slot_mapping_out, slot_mapping_capacity,
+                                          next_fact_ids, num_next_ids, stream)
 
 
 def is_last_error(store: int, stream: int = 0) -> tuple[int, int]:

@@ -83,6 +83,15 @@ struct is_store {
   int64_t* d_pend = nullptr;
   size_t pend_ne = 0, pend_np = 0;
   bool batch_pend = false;   // the batch being launched reads d_pend
+  // prefetch of the next batch's cold facts (is_inject_batch_host_next):
+  // copy-engine transfers on copy_stream; the next batch waits for pf_done
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t pf_done = nullptr;
+  bool pf_pending = false;
+  uint64_t batch_tick = 0;   // LRU tick of the last host-entry batch
+  int64_t* h_pf_pairs = nullptr;
+  int64_t* d_pf_pairs = nullptr;
+  size_t pf_cap = 0;         // pairs
   // fact table
   int64_t* d_off = nullptr;
   int32_t* d_len = nullptr;
@@ -204,6 +213,10 @@ void free_store(is_store* s) {
   cudaFree(s->d_pairs);
   cudaFree(s->d_pend);
   if (s->touch_done) cudaEventDestroy(s->touch_done);
+  if (s->pf_done) cudaEventDestroy(s->pf_done);
+  if (s->copy_stream) cudaStreamDestroy(s->copy_stream);
+  cudaFreeHost(s->h_pf_pairs);
+  cudaFree(s->d_pf_pairs);
   if (s->host_arena) {
     cudaFreeHost(s->k);
     cudaFreeHost(s->v);
@@ -788,6 +801,8 @@ int is_store_set_hot_policy(is_store_t* s, int policy, int32_t slot_tokens) {
   for (size_t i = 0; i < nslots; ++i) s->lru_at[i] = s->lru.insert(s->lru.end(), int32_t(i));
   s->fact_tick.assign(size_t(s->cfg.max_facts), 0);
   s->tick = 0;
+  s->batch_tick = 0;
+  s->pf_pending = false;  // the device is idle: any prefetch has landed
   s->lru_hits = s->lru_misses = s->lru_promoted = s->lru_promoted_tokens = 0;
   if (!s->touch_done && cudaEventCreateWithFlags(&s->touch_done, cudaEventDisableTiming) != cudaSuccess)
     return IS_ERR_CUDA;
@@ -805,13 +820,14 @@ int is_store_set_hot_policy(is_store_t* s, int policy, int32_t slot_tokens) {
 //     their rows into their HBM slots -- each row crosses the host link once
 //     and no copy runs ahead of the batch; lru_finish then enters them in
 //     the hot table.
-static int lru_touch(is_store* s, const int32_t* fact_ids, int32_t n, cudaStream_t st, bool fused,
-                     int32_t* promoted_out) {
-  // The staging of the previous touch must have been consumed.
-  if (cudaEventSynchronize(s->touch_done) != cudaSuccess) return IS_ERR_CUDA;
-  const uint64_t tick = ++s->tick;
-  std::vector<isk::Promotion> promo;
-  std::vector<int64_t> evict, prom;  // evicted facts; (fact, hot token) promoted
+// The LRU decisions for one list of ids (host only): hits move to the front
+// of the list; misses that fit a slot take the least recently used slot,
+// unless that slot was used at or after tick `protect` (this call, and a
+// batch that may still be running).  Fills the evicted facts, the
+// (fact, hot token) promotions and their copy descriptors.
+static void lru_plan(is_store* s, const int32_t* fact_ids, int32_t n, uint64_t tick, uint64_t protect,
+                     bool count_use, std::vector<int64_t>& evict, std::vector<int64_t>& prom,
+                     std::vector<isk::Promotion>& promo) {
   for (int32_t i = 0; i < n; ++i) {
     const int32_t f = fact_ids[i];
     if (f < 0 || f >= s->num_facts) continue;  // the batch itself reports it
@@ -822,13 +838,13 @@ static int lru_touch(is_store* s, const int32_t* fact_ids, int32_t n, cudaStream
       const int32_t slot = int32_t(ho / s->slot_tokens);
       s->lru.splice(s->lru.begin(), s->lru, s->lru_at[size_t(slot)]);
       s->slot_tick[size_t(slot)] = tick;
-      ++s->lru_hits;
+      if (count_use) ++s->lru_hits;
       continue;
     }
-    ++s->lru_misses;
+    if (count_use) ++s->lru_misses;
     if (s->lru.empty() || s->h_len[size_t(f)] > s->slot_tokens) continue;  // served from host
     const int32_t slot = s->lru.back();
-    if (s->slot_tick[size_t(slot)] == tick) continue;  // every slot serves this call
+    if (s->slot_tick[size_t(slot)] >= protect) continue;  // every slot is in use
     const int32_t old = s->slot_owner[size_t(slot)];
     if (old >= 0) {
       s->h_hot[size_t(old)] = -1;
@@ -848,6 +864,18 @@ static int lru_touch(is_store* s, const int32_t* fact_ids, int32_t n, cudaStream
   }
   s->lru_promoted += int64_t(promo.size());
   s->hot_used = int64_t(s->hot_facts) * s->slot_tokens;
+}
+
+static int lru_touch(is_store* s, const int32_t* fact_ids, int32_t n, cudaStream_t st, bool fused,
+                     int32_t* promoted_out) {
+  // The staging of the previous touch must have been consumed, and a
+  // prefetch's transfers must have landed before its slots are reconsidered.
+  if (cudaEventSynchronize(s->touch_done) != cudaSuccess) return IS_ERR_CUDA;
+  if (s->pf_pending && cudaEventSynchronize(s->pf_done) != cudaSuccess) return IS_ERR_CUDA;
+  const uint64_t tick = ++s->tick;
+  std::vector<isk::Promotion> promo;
+  std::vector<int64_t> evict, prom;  // evicted facts; (fact, hot token) promoted
+  lru_plan(s, fact_ids, n, tick, tick, true, evict, prom, promo);
   if (promoted_out) *promoted_out = int32_t(promo.size());
   s->pend_ne = s->pend_np = 0;
   if (promo.empty()) return IS_OK;
@@ -929,6 +957,64 @@ static int lru_finish(is_store* s, cudaStream_t st, bool batch_ok) {
   return IS_OK;
 }
 
+// Prefetch for the next batch (LRU): its cold facts take slots not used by
+// the batch just launched (tick s->batch_tick or later) and move into HBM by
+// copy-engine transfers on the store's copy stream, one 2-D copy per fact
+// and tensor (its L x H plane rows), while that batch runs; then the hot
+// table learns them.  The next batch on the store waits for pf_done.
+static int lru_prefetch(is_store* s, const int32_t* fact_ids, int32_t n) {
+  if (!s->copy_stream &&
+      cudaStreamCreateWithFlags(&s->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return IS_ERR_CUDA;
+  if (!s->pf_done && cudaEventCreateWithFlags(&s->pf_done, cudaEventDisableTiming) != cudaSuccess)
+    return IS_ERR_CUDA;
+  // the previous prefetch's pair list must have been consumed
+  if (s->pf_pending && cudaEventSynchronize(s->pf_done) != cudaSuccess) return IS_ERR_CUDA;
+  const uint64_t tick = ++s->tick;
+  std::vector<isk::Promotion> promo;
+  std::vector<int64_t> evict, prom;
+  lru_plan(s, fact_ids, n, tick, s->batch_tick, false, evict, prom, promo);
+  if (promo.empty()) return IS_OK;
+  std::vector<int64_t> pairs;
+  for (int64_t f : evict) { pairs.push_back(f); pairs.push_back(-1); }
+  pairs.insert(pairs.end(), prom.begin(), prom.end());
+  const size_t nq = pairs.size() / 2;
+  if (nq > s->pf_cap) {
+    cudaFreeHost(s->h_pf_pairs);
+    cudaFree(s->d_pf_pairs);
+    s->h_pf_pairs = nullptr;
+    s->d_pf_pairs = nullptr;
+    s->pf_cap = 0;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&s->h_pf_pairs), nq * 2 * 2 * sizeof(int64_t), 0) != cudaSuccess ||
+        dalloc(&s->d_pf_pairs, nq * 2 * 2) != cudaSuccess)
+      return IS_ERR_OOM;
+    s->pf_cap = nq * 2;
+  }
+  std::memcpy(s->h_pf_pairs, pairs.data(), pairs.size() * sizeof(int64_t));
+  const is_store_config_t& c = s->cfg;
+  const size_t row = size_t(c.head_dim) * sizeof(uint16_t);
+  const size_t height = size_t(c.num_layers) * size_t(c.num_kv_heads);
+  const size_t spitch = size_t(c.capacity_tokens) * row, dpitch = size_t(s->hot_cap) * row;
+  cudaStream_t cs = s->copy_stream;
+  for (const isk::Promotion& p : promo) {
+    const size_t width = size_t(p.len) * row;
+    const size_t so = size_t(p.src_tok) * row, dof = size_t(p.dst_tok) * row;
+    if (cudaMemcpy2DAsync(reinterpret_cast<char*>(s->k_hot) + dof, dpitch, reinterpret_cast<const char*>(s->k) + so,
+                          spitch, width, height, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpy2DAsync(reinterpret_cast<char*>(s->v_hot) + dof, dpitch, reinterpret_cast<const char*>(s->v) + so,
+                          spitch, width, height, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+      return IS_ERR_CUDA;
+  }
+  if (cudaMemcpyAsync(s->d_pf_pairs, s->h_pf_pairs, pairs.size() * sizeof(int64_t), cudaMemcpyHostToDevice, cs) !=
+      cudaSuccess)
+    return IS_ERR_CUDA;
+  isk::hot_table_kernel<<<unsigned((nq + 255) / 256), 256, 0, cs>>>(s->d_hot, s->d_hot, s->d_pf_pairs,
+                                                                   int32_t(nq), 0);
+  if (cudaEventRecord(s->pf_done, cs) != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
+  s->pf_pending = true;
+  return IS_OK;
+}
+
 int is_store_touch(is_store_t* s, const int32_t* fact_ids, int32_t n, void* stream, int32_t* promoted_out) {
   if (!s || n < 0 || (n > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
   if (!s->host_arena || s->hot_policy != IS_HOT_LRU) return IS_ERR_NOT_SUPPORTED;
@@ -978,6 +1064,8 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   DeviceGuard guard(s->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const is_store_config_t& cf = s->cfg;
+  // a prefetch's transfers and hot-table changes land before this batch reads
+  if (s->pf_pending && cudaStreamWaitEvent(st, s->pf_done, 0) != cudaSuccess) return IS_ERR_CUDA;
 
   isk::PlanArgs pa;
   pa.R = R;
@@ -1114,12 +1202,13 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   return IS_OK;
 }
 
-int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const int32_t* fact_ids,
-                         int32_t num_ids, const int32_t* start_pos, const int32_t* block_tables,
-                         int32_t max_blocks_per_req, const is_cache_t* cache, int64_t* slot_out,
-                         int64_t slot_cap, void* stream) {
+static int host_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int32_t* fact_ids,
+                      int32_t num_ids, const int32_t* start_pos, const int32_t* block_tables,
+                      int32_t max_blocks_per_req, const is_cache_t* cache, int64_t* slot_out,
+                      int64_t slot_cap, const int32_t* next_ids, int32_t num_next, void* stream) {
   if (!s || !cache || R < 0 || num_ids < 0 || max_blocks_per_req < 1 || !req_off) return IS_ERR_INVALID_ARG;
   if ((R > 0 && (!start_pos || !block_tables)) || (num_ids > 0 && !fact_ids)) return IS_ERR_INVALID_ARG;
+  if (num_next < 0 || (num_next > 0 && !next_ids)) return IS_ERR_INVALID_ARG;
   if (R > s->max_req || num_ids > s->max_ids) return IS_ERR_CAPACITY;
   if (slot_out && slot_cap < 0) return IS_ERR_INVALID_ARG;
   DeviceGuard guard(s->device);
@@ -1133,6 +1222,7 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
   if (lru) {  // this batch's cold facts: promotions fused into the batch
     rc = lru_touch(s, fact_ids, num_ids, st, true, nullptr);
     if (rc != IS_OK) return rc;
+    s->batch_tick = s->tick;
   }
   // Pack the four index arrays into one pinned buffer: one host-to-device copy.
   int32_t* h = s->host_stage;
@@ -1156,6 +1246,8 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
     lru_finish(s, st, false);  // nothing ran: copy the promoted facts instead
     return rc;
   }
+  // The next batch's cold facts move over the host link while this one runs.
+  if (lru && num_next > 0 && (rc = lru_prefetch(s, next_ids, num_next)) != IS_OK) return rc;
   if (slot_out && slot_cap > 0 &&
       cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost, st) !=
           cudaSuccess)
@@ -1170,6 +1262,23 @@ int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const
     return IS_ERR_CUDA;
   if (code != 0 && cudaMemset(s->d_status, 0, sizeof(isk::DevStatus)) != cudaSuccess) return IS_ERR_CUDA;
   return code;
+}
+
+int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const int32_t* fact_ids,
+                         int32_t num_ids, const int32_t* start_pos, const int32_t* block_tables,
+                         int32_t max_blocks_per_req, const is_cache_t* cache, int64_t* slot_out,
+                         int64_t slot_cap, void* stream) {
+  return host_batch(s, R, req_off, fact_ids, num_ids, start_pos, block_tables, max_blocks_per_req, cache,
+                    slot_out, slot_cap, nullptr, 0, stream);
+}
+
+int is_inject_batch_host_next(is_store_t* s, int32_t R, const int32_t* req_off, const int32_t* fact_ids,
+                              int32_t num_ids, const int32_t* start_pos, const int32_t* block_tables,
+                              int32_t max_blocks_per_req, const is_cache_t* cache, int64_t* slot_out,
+                              int64_t slot_cap, const int32_t* next_fact_ids, int32_t num_next_ids,
+                              void* stream) {
+  return host_batch(s, R, req_off, fact_ids, num_ids, start_pos, block_tables, max_blocks_per_req, cache,
+                    slot_out, slot_cap, next_fact_ids, num_next_ids, stream);
 }
 
 int is_last_error(is_store_t* s, void* stream, int64_t* detail) {

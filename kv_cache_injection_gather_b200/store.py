@@ -217,20 +217,28 @@ class FactStore:
 
     def inject_host(self, req_offsets: torch.Tensor, fact_ids: torch.Tensor,
                     start_pos: torch.Tensor, block_tables: torch.Tensor, cache: B.is_cache_t,
-                    slot_mapping: torch.Tensor | None = None, stream: int | None = None) -> int:
+                    slot_mapping: torch.Tensor | None = None, stream: int | None = None,
+                    next_fact_ids: torch.Tensor | None = None) -> int:
         """Index tensors in host memory (pinned for asynchronous copies);
-        waits and returns the batch status."""
+        waits and returns the batch status.  next_fact_ids (host int32): the
+        next batch's ids, whose cold facts an LRU host-tier store prefetches
+        into HBM while this batch runs."""
         for t in (req_offsets, fact_ids, start_pos, block_tables):
             if t.is_cuda:
                 raise ValueError("inject_host takes host tensors")
         if stream is None:
             stream = torch.cuda.current_stream(self.device).cuda_stream
-        return B.is_inject_batch_host(
-            self.handle, start_pos.numel(), req_offsets.data_ptr(), fact_ids.data_ptr(),
-            fact_ids.numel(), start_pos.data_ptr(), block_tables.data_ptr(),
-            block_tables.shape[1], cache,
-            None if slot_mapping is None else slot_mapping.data_ptr(),
-            0 if slot_mapping is None else slot_mapping.numel(), stream)
+        args = (self.handle, start_pos.numel(), req_offsets.data_ptr(), fact_ids.data_ptr(),
+                fact_ids.numel(), start_pos.data_ptr(), block_tables.data_ptr(),
+                block_tables.shape[1], cache,
+                None if slot_mapping is None else slot_mapping.data_ptr(),
+                0 if slot_mapping is None else slot_mapping.numel())
+        if next_fact_ids is None:
+            return B.is_inject_batch_host(*args, stream)
+        nxt = _i32(next_fact_ids, "next_fact_ids")
+        if nxt.is_cuda:
+            raise ValueError("next_fact_ids is a host tensor")
+        return B.is_inject_batch_host_next(*args, nxt.data_ptr(), nxt.numel(), stream)
 
     def last_error(self, stream: int | None = None) -> tuple[int, int]:
         if stream is None:

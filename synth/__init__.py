@@ -272,12 +272,17 @@ def llama_single(seed: int = 0, num_facts: int = 10_000, k: int = 5,
 
 
 def llama_batch(seed: int = 0, num_facts: int = 10_000, R: int = 100, k: int = 50,
-                slots_per_request: int = 4096) -> Workload:
+                slots_per_request: int = 4096, distinct_batch: bool = False) -> Workload:
     """Llama-3.1-8B shapes; 100 requests x k=50 distinct facts after a 64-token
-    prefix, each request owning 4096 slots (256 blocks) of a shuffled cache."""
+    prefix, each request owning 4096 slots (256 blocks) of a shuffled cache.
+    distinct_batch: no fact repeats anywhere in the batch (R * k ids drawn
+    without replacement)."""
     rng = np.random.default_rng(seed)
     lens = uniform_lengths(rng, num_facts, 16, 64)
-    ids = [distinct_ids(rng, num_facts, k) for _ in range(R)]
+    if distinct_batch:
+        ids = list(distinct_ids(rng, num_facts, R * k).reshape(R, k))
+    else:
+        ids = [distinct_ids(rng, num_facts, k) for _ in range(R)]
     mb = slots_per_request // 16
     batch = make_batch(rng, ids, 64, 16, R * mb, mb)
     return Workload(f"llama3.1-8b R={R} k={k}", LLAMA31_8B, lens, batch, seed)

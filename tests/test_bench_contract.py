@@ -77,3 +77,13 @@ def test_gpu_arm_fails_loudly_without_a_gpu():
     assert r.returncode != 0
     assert "CUDA device" in (r.stderr + r.stdout)
     assert not _json_lines(r.stdout)
+
+
+def test_l2_flush_runs_on_any_device():
+    """The flush between singly timed steps (a write of twice L2, then a read
+    of twice L2) is plain torch work; on the CPU it must run as written."""
+    sys.path.insert(0, ROOT)
+    import bench
+    f = bench.L2Flush("cpu")
+    f()
+    assert f.buf.numel() == 2 * bench.L2_BYTES and int(f.acc) == 0

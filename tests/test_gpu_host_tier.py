@@ -177,3 +177,46 @@ def test_lru_promotion_survives_a_batch_with_errors():
     assert store.lru_stats()["promoted"] == promoted       # nothing left to promote
     assert_parity(want, gpu_run(wl, store=store))          # device entry point, same hot set
     store.close()
+
+
+def test_lru_prefetch_of_the_next_batch():
+    """A stream of batches through is_inject_batch_host_next: each call
+    injects its batch and starts moving the next batch's cold facts into HBM
+    slots (copy-engine transfers, slots not used by the running batch) while
+    it runs.  With 30 slots and 20 facts per batch, part of each next batch
+    fits beside the running one and the rest is promoted by its own batch.
+    Every batch equals the oracle -- also when the announced next ids are not
+    the ones that come, and through the device entry point after a
+    prefetch."""
+    _need_gpu()
+    from synth.device import make_cache
+    from test_gpu_parity import to_bits
+    model = synth.Model("qwen-like", 2, 4, 128, 1e6)
+    rng = np.random.default_rng(71)
+    lens = rng.integers(4, 33, 80).astype(np.int32)
+    slot = 32
+    store = None
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
+    batches = []
+    for _ in range(6):
+        ids = [rng.choice(80, 5, replace=False) for _ in range(4)]
+        batches.append(synth.make_batch(rng, ids, [0, 17, 40, 64], 16, 4 * 10, 10))
+    wls = [synth.Workload("pf", model, lens, bb, seed=9) for bb in batches]
+    store = make_store(wls[0], host_tier=True, hot_capacity_tokens=slot * 30)
+    store.set_hot_policy(True, slot)
+    promoted = []
+    for i, wl in enumerate(wls):
+        b = wl.batch
+        nxt = batches[(i + 1) % len(batches)].fact_ids if i != 3 else rng.choice(80, 12)
+        k, v, desc = make_cache(wl)
+        n_tok = wl.tokens()
+        slots = torch.empty(max(n_tok, 1), dtype=torch.int64).pin_memory()
+        before = store.lru_stats()["promoted"]
+        rc = store.inject_host(pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos),
+                               pin(b.block_tables), desc, slots[:n_tok],
+                               next_fact_ids=pin(nxt))
+        assert_parity(oracle_run(wl), (rc, slots[:n_tok].numpy().copy(), to_bits(k), to_bits(v)))
+        promoted.append(store.lru_stats()["promoted"] - before)
+    assert promoted[0] > 0
+    assert_parity(oracle_run(wls[0]), gpu_run(wls[0], store=store))
+    store.close()
