@@ -240,11 +240,12 @@ WORKLOADS = {
                           "cache 640 blocks (profiling case, ~4 GB on the device)",
                           lambda seed: _synth().llama_batch(seed, num_facts=500, R=10, k=20,
                                                             slots_per_request=1024)),
-    "llama-batch-distinct-small": ("llama3.1-8b-shapes 600-fact store, 8 requests x k=25, no fact "
-                                   "repeated in the batch, block 16, cache 832 blocks (profiling "
-                                   "case for DRAM traffic, ~5 GB on the device)",
-                                   lambda seed: _synth().llama_batch(seed, num_facts=600, R=8, k=25,
-                                                                     slots_per_request=1664,
+    "llama-batch-distinct-small": ("llama3.1-8b-shapes 600-fact store, 9 requests x k=22, no fact "
+                                   "repeated in the batch, block 16, cache 864 blocks (profiling "
+                                   "case for DRAM traffic of the plan + inject path, ~5 GB on the "
+                                   "device)",
+                                   lambda seed: _synth().llama_batch(seed, num_facts=600, R=9, k=22,
+                                                                     slots_per_request=1536,
                                                                      distinct_batch=True)),
     "llama-single": ("llama3.1-8b-shapes 10k-fact store, 1 request x k=5, block 16, 64 blocks",
                      lambda seed: _synth().llama_single(seed)),
@@ -483,9 +484,9 @@ def max_over_ranks(values, world):
 def run_offload(args, rank, world, local_rank):
     """Host-tier store: a stream of 8 different Zipf batches, cycled.  Static
     hot set (top 20% by rank, device-index entry point) or LRU hot set (same
-    HBM capacity in 48-token slots, host-index entry point: each call injects
-    its batch and prefetches the next batch's cold facts while it runs; what
-    the prefetch could not place is promoted by the batch itself)."""
+    HBM capacity in 48-token slots, host-index entry point: each batch promotes
+    its cold facts as it reads them; with --lru-prefetch each call also starts
+    the next batch's cold facts while it runs)."""
     import psutil
     import torch
 
@@ -527,9 +528,10 @@ def run_offload(args, rank, world, local_rank):
     def step(i):
         j = i % len(batches)
         if lru:
-            # the next batch's cold facts move into HBM (copy engine) while this one runs
+            # with --lru-prefetch, the next batch's cold facts move into HBM while this one runs
             rc = store.inject_host(*host_b[j], desc, h_slots[:ntoks[j]], stream.cuda_stream,
-                                   next_fact_ids=host_b[(i + 1) % len(batches)][1])
+                                   next_fact_ids=(host_b[(i + 1) % len(batches)][1]
+                                                  if args.lru_prefetch else None))
             if rc != 0:
                 raise RuntimeError(f"inject_host failed: {B.status_string(rc)}")
         else:
@@ -602,7 +604,7 @@ def run_offload(args, rank, world, local_rank):
             "facts_note": f"{n_facts} facts (host memory available {avail / 1e9:.0f} GB)",
             "hot_policy": args.hot_policy, "hot_tokens_per_plane": hot_tokens,
             "prefetch": ("each batch's call starts the next batch's cold facts over the host link "
-                         "(copy engine) while the batch runs" if lru else None),
+                         "while the batch runs" if lru and args.lru_prefetch else None),
             "batches": f"{len(batches)} Zipf batches cycled", "parallelism": f"replicas x{world}"}),
         "us_per_batch": ms / args.steps * 1e3, "kernel_us": kern_avg_ms * 1e3, "clocks": clk,
         "gpu_launches": (4 if lru else 2) * args.steps,
@@ -882,8 +884,10 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
         # the library's kernels per step: one fused kernel for batches of at
-        # most 8 requests and 256 ids, else the plan and the inject kernel
-        "gpu_launches": (1 if b.num_requests <= 8 and len(b.fact_ids) <= 256 else 2) * args.steps,
+        # most 8 requests, 256 ids and 6 144 tokens by the bound (ids x the
+        # longest fact), else the plan and the inject kernel
+        "gpu_launches": (1 if (b.num_requests <= 8 and len(b.fact_ids) <= 256 and
+                               len(b.fact_ids) * int(wl.fact_lens.max()) <= 6144) else 2) * args.steps,
         "roofline": roofline,
         "cpu_baseline": baseline,
     }
@@ -901,6 +905,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--hot-policy", choices=["static", "lru"], default="static",
                     help="offload workload: static top-20%% hot set or LRU promotion")
+    ap.add_argument("--lru-prefetch", action="store_true",
+                    help="offload workload, LRU: each call also prefetches the next batch's cold facts")
     ap.add_argument("--shard", choices=["replicas", "heads", "facts"], default="replicas",
                     help="multi-GPU: independent replicas (default), KV-head shards of one "
                          "batch of 100 x N requests (both weak scaling, no collective), or fact "

@@ -321,8 +321,8 @@ int is_inject_batch_host(is_store_t* store, int32_t num_requests,
  * LRU hot set (IS_HOT_LRU): the same batch, and, while it runs, the cold
  * facts of the NEXT batch (next_fact_ids, host array, num_next_ids entries;
  * the caller's retrieval knows them before their injection) start moving
- * into HBM slots by copy-engine transfers on a stream of the store -- slots
- * not used by this batch, in least-recently-used order -- so that batch
+ * into HBM slots on a stream of the store -- slots not used by this batch,
+ * in least-recently-used order -- so that batch
  * reads them from HBM (technical summary, Results, "Scalability": the KV
  * store may live in host DRAM; this is its prefetch path).  Every later
  * batch on the store waits for those transfers.  Ids that do not come or
@@ -350,10 +350,11 @@ int is_last_error(is_store_t* store, void* stream, int64_t* detail_out);
 int is_last_error_timeout(is_store_t* store, void* stream, int32_t timeout_ms,
                           int64_t* detail_out);
 
-/* Batches with at most max_requests requests (0..8; default 8) and at most
- * 256 fact ids run as one kernel that composes the batch in every CTA
+/* Batches with at most max_requests requests (0..8; default 8), at most
+ * 256 fact ids and at most 6 144 tokens by the bound (ids x the store's
+ * longest fact) run as one kernel that composes the batch in every CTA
  * instead of a plan kernel followed by the inject kernel (lower latency for
- * small batches; same results).  0 always uses the two-kernel path. */
+ * short batches; same results).  0 always uses the two-kernel path. */
 int is_store_set_small_batch_limit(is_store_t* store, int32_t max_requests);
 
 /* ---- measurement -------------------------------------------------------- */

@@ -408,8 +408,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   // Phase 3, one warp per request: block descriptors (lanes over blocks, so
   // a warp writes consecutive descriptors), the check of every touched
   // block-table entry, and -1 slots for the tokens of invalid requests.
-  auto check_entry = [&](int r, int32_t b) {
-    const int32_t phys = a.block_tables[(long long)r * a.max_blocks + b];
+  auto check_entry = [&](int r, int32_t b, int32_t phys) {
     if (phys < 0 || phys >= a.num_blocks) atomicMin(&s_err_key, ((unsigned long long)r << 32) | unsigned(b));
   };
   for (int r = warp; r < a.R; r += NW) {
@@ -433,6 +432,8 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
       // <= its first index (binary search in shared memory); a warp writes
       // consecutive descriptors.
       for (int32_t bi = lane; bi < nblk; bi += 32) {
+        // the table entry's load is issued first: it overlaps the search
+        const int32_t phys = a.block_tables[(long long)r * a.max_blocks + fb + bi];
         const int32_t i0 = bi == 0 ? 0 : (fb + bi) * a.B - start;
         int32_t lo = j0, hi = j1 - 1;  // seg[j0] = 0 <= i0
         while (lo < hi) {
@@ -445,7 +446,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
         d.j = lo;
         d.pad = 0;
         a.desc[g0 + bi] = d;
-        check_entry(r, fb + bi);
+        check_entry(r, fb + bi, phys);
       }
     } else {
       // Lanes over facts (no dependent L2 reads): fact j [s, e) owns the
@@ -467,7 +468,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
           d.j = j;
           d.pad = 0;
           a.desc[g0 + bi] = d;
-          check_entry(r, fb + bi);
+          check_entry(r, fb + bi, a.block_tables[(long long)r * a.max_blocks + fb + bi]);
         }
       }
     }

@@ -36,6 +36,7 @@ constexpr int kInjectMinBlocks = IS_INJECT_MIN_BLOCKS;
 constexpr int kDefaultMaxRequests = 4096;
 constexpr int kDefaultMaxFactIds = 1 << 20;
 constexpr int kMaxTimedLaunches = 4096;
+constexpr int64_t kSmallTokens = 6144;  // single-kernel path: ids x longest fact at most
 
 struct TimedLaunch {
   cudaEvent_t start, stop;
@@ -91,7 +92,9 @@ struct is_store {
   uint64_t batch_tick = 0;   // LRU tick of the last host-entry batch
   int64_t* h_pf_pairs = nullptr;
   int64_t* d_pf_pairs = nullptr;
-  size_t pf_cap = 0;         // pairs
+  isk::Promotion* h_pf_promo = nullptr;
+  isk::Promotion* d_pf_promo = nullptr;
+  size_t pf_cap = 0;         // pairs (and promotions)
   // fact table
   int64_t* d_off = nullptr;
   int32_t* d_len = nullptr;
@@ -217,6 +220,8 @@ void free_store(is_store* s) {
   if (s->copy_stream) cudaStreamDestroy(s->copy_stream);
   cudaFreeHost(s->h_pf_pairs);
   cudaFree(s->d_pf_pairs);
+  cudaFreeHost(s->h_pf_promo);
+  cudaFree(s->d_pf_promo);
   if (s->host_arena) {
     cudaFreeHost(s->k);
     cudaFreeHost(s->v);
@@ -958,17 +963,19 @@ static int lru_finish(is_store* s, cudaStream_t st, bool batch_ok) {
 }
 
 // Prefetch for the next batch (LRU): its cold facts take slots not used by
-// the batch just launched (tick s->batch_tick or later) and move into HBM by
-// copy-engine transfers on the store's copy stream, one 2-D copy per fact
-// and tensor (its L x H plane rows), while that batch runs; then the hot
-// table learns them.  The next batch on the store waits for pf_done.
+// the batch just launched (tick s->batch_tick or later) and are copied into
+// HBM on the store's copy stream while that batch runs, by promote_kernel
+// (the SMs' reads of the mapped host arenas: on B200 they keep ~0.91 of a
+// large copy-engine transfer's host-link rate, where one copy-engine transfer
+// per fact, ~1 MB each, keeps ~0.78); then the hot table learns them.  The
+// next batch on the store waits for pf_done.
 static int lru_prefetch(is_store* s, const int32_t* fact_ids, int32_t n) {
   if (!s->copy_stream &&
       cudaStreamCreateWithFlags(&s->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
     return IS_ERR_CUDA;
   if (!s->pf_done && cudaEventCreateWithFlags(&s->pf_done, cudaEventDisableTiming) != cudaSuccess)
     return IS_ERR_CUDA;
-  // the previous prefetch's pair list must have been consumed
+  // the previous prefetch's lists must have been consumed
   if (s->pf_pending && cudaEventSynchronize(s->pf_done) != cudaSuccess) return IS_ERR_CUDA;
   const uint64_t tick = ++s->tick;
   std::vector<isk::Promotion> promo;
@@ -978,36 +985,39 @@ static int lru_prefetch(is_store* s, const int32_t* fact_ids, int32_t n) {
   std::vector<int64_t> pairs;
   for (int64_t f : evict) { pairs.push_back(f); pairs.push_back(-1); }
   pairs.insert(pairs.end(), prom.begin(), prom.end());
-  const size_t nq = pairs.size() / 2;
+  const size_t nq = pairs.size() / 2, np = promo.size();
   if (nq > s->pf_cap) {
     cudaFreeHost(s->h_pf_pairs);
     cudaFree(s->d_pf_pairs);
+    cudaFreeHost(s->h_pf_promo);
+    cudaFree(s->d_pf_promo);
     s->h_pf_pairs = nullptr;
     s->d_pf_pairs = nullptr;
+    s->h_pf_promo = nullptr;
+    s->d_pf_promo = nullptr;
     s->pf_cap = 0;
-    if (cudaHostAlloc(reinterpret_cast<void**>(&s->h_pf_pairs), nq * 2 * 2 * sizeof(int64_t), 0) != cudaSuccess ||
-        dalloc(&s->d_pf_pairs, nq * 2 * 2) != cudaSuccess)
+    const size_t cap = nq * 2;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&s->h_pf_pairs), cap * 2 * sizeof(int64_t), 0) != cudaSuccess ||
+        dalloc(&s->d_pf_pairs, cap * 2) != cudaSuccess ||
+        cudaHostAlloc(reinterpret_cast<void**>(&s->h_pf_promo), cap * sizeof(isk::Promotion), 0) != cudaSuccess ||
+        dalloc(&s->d_pf_promo, cap) != cudaSuccess)
       return IS_ERR_OOM;
-    s->pf_cap = nq * 2;
+    s->pf_cap = cap;
   }
   std::memcpy(s->h_pf_pairs, pairs.data(), pairs.size() * sizeof(int64_t));
+  std::memcpy(s->h_pf_promo, promo.data(), np * sizeof(isk::Promotion));
   const is_store_config_t& c = s->cfg;
-  const size_t row = size_t(c.head_dim) * sizeof(uint16_t);
-  const size_t height = size_t(c.num_layers) * size_t(c.num_kv_heads);
-  const size_t spitch = size_t(c.capacity_tokens) * row, dpitch = size_t(s->hot_cap) * row;
   cudaStream_t cs = s->copy_stream;
-  for (const isk::Promotion& p : promo) {
-    const size_t width = size_t(p.len) * row;
-    const size_t so = size_t(p.src_tok) * row, dof = size_t(p.dst_tok) * row;
-    if (cudaMemcpy2DAsync(reinterpret_cast<char*>(s->k_hot) + dof, dpitch, reinterpret_cast<const char*>(s->k) + so,
-                          spitch, width, height, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-        cudaMemcpy2DAsync(reinterpret_cast<char*>(s->v_hot) + dof, dpitch, reinterpret_cast<const char*>(s->v) + so,
-                          spitch, width, height, cudaMemcpyHostToDevice, cs) != cudaSuccess)
-      return IS_ERR_CUDA;
-  }
-  if (cudaMemcpyAsync(s->d_pf_pairs, s->h_pf_pairs, pairs.size() * sizeof(int64_t), cudaMemcpyHostToDevice, cs) !=
-      cudaSuccess)
+  if (cudaMemcpyAsync(s->d_pf_promo, s->h_pf_promo, np * sizeof(isk::Promotion), cudaMemcpyHostToDevice, cs) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(s->d_pf_pairs, s->h_pf_pairs, pairs.size() * sizeof(int64_t), cudaMemcpyHostToDevice, cs) !=
+          cudaSuccess)
     return IS_ERR_CUDA;
+  dim3 grid(unsigned(std::max(1, s->sm_count / 2)), unsigned(std::min<size_t>(np, 65535)));
+  isk::promote_kernel<<<grid, 256, 0, cs>>>(s->d_pf_promo, int32_t(np), c.num_layers * c.num_kv_heads,
+                                             c.head_dim / 8, s->k_view, s->v_view,
+                                             int64_t(c.capacity_tokens) * c.head_dim, s->k_hot, s->v_hot,
+                                             s->hot_cap * c.head_dim);
   isk::hot_table_kernel<<<unsigned((nq + 255) / 256), 256, 0, cs>>>(s->d_hot, s->d_hot, s->d_pf_pairs,
                                                                    int32_t(nq), 0);
   if (cudaEventRecord(s->pf_done, cs) != cudaSuccess || cudaGetLastError() != cudaSuccess) return IS_ERR_CUDA;
@@ -1103,11 +1113,15 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.desc = s->ws_desc;
   pa.hdr = s->ws_hdr;
   pa.st = s->d_status;
-  // The single-kernel path sums a batch's lengths in 32 bits: only batches
-  // whose ids cannot total more than 2^31 - 1 tokens take it.
+  // The single kernel saves the plan launch but schedules its units
+  // statically: it wins while a batch is short (measured on B200, Llama-3.1
+  // shapes: 16.3 vs 21.6 us for 152 tokens, level at ~4 000 tokens, 2% slower
+  // at 8 000), so it takes batches whose ids cannot total more than
+  // kSmallTokens tokens (ids x the longest fact; this also keeps its 32-bit
+  // sums from wrapping).
   const int64_t longest = view ? s->shard_max_len : s->max_len;
   const bool small = R <= s->small_limit && num_ids <= isk::kSmallIds &&
-                     int64_t(num_ids) * longest <= int64_t(0x7fffffff);
+                     int64_t(num_ids) * longest <= kSmallTokens;
   if (!small) {
     if (R <= isk::kPlanSmemRequests && num_ids <= isk::kPlanSmemIds)
       isk::plan_kernel<kPlanThreads, true><<<1, kPlanThreads, isk::plan_smem_bytes(R, num_ids), st>>>(pa);
