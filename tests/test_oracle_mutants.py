@@ -50,6 +50,11 @@ MUTANTS = {
     # linear in orig / wavelength
     "llama3_blend_squared": ("double smooth = (orig / lam - low) / (high - low);",
                              "double smooth = (orig / lam - low) / (high - low);\n  smooth = smooth * smooth;"),
+    # a NaN rounded to an infinity
+    "nan_to_inf": ("if (isnan(x)) return 0x7FC0;", "if (isnan(x)) return 0x7F80;"),
+    # the rotation pair taken from the interleaved layout under rotate-half
+    "pair_style_swapped": ("if (style == 0) { *a = i; *b = i + D / 2; }",
+                           "if (style != 0) { *a = i; *b = i + D / 2; }"),
     # K left unrotated
     "k_not_rotated": ("c->k[dst + d] = orc_f64_to_bf16(y[d]);", "c->k[dst + d] = orc_f64_to_bf16(x[d]);"),
 }
