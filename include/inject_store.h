@@ -329,7 +329,9 @@ int is_inject_batch_host(is_store_t* store, int32_t num_requests,
  * are outside the store only cost their transfer; results never depend on
  * the prefetch.  On a store without the LRU policy the next ids are
  * ignored.  Errors as for is_inject_batch_host, and INVALID_ARG for
- * num_next_ids < 0 or a NULL list. */
+ * num_next_ids < 0 or a NULL list; when this batch ran clean but the
+ * prefetch could not be started (OOM, CUDA), that error is returned after
+ * the batch has completed. */
 int is_inject_batch_host_next(is_store_t* store, int32_t num_requests,
                               const int32_t* req_fact_offsets, const int32_t* fact_ids,
                               int32_t num_fact_ids, const int32_t* start_pos,

@@ -33,6 +33,16 @@ constexpr int kPlanThreads = 1024;
 constexpr int kInjectThreads = IS_INJECT_THREADS;
 constexpr int kVecsPerThread = IS_INJECT_VECS;
 constexpr int kInjectMinBlocks = IS_INJECT_MIN_BLOCKS;
+// The single-kernel path for short batches has its own launch shape: its
+// batches fit about one wave, so more, lighter CTAs per SM can help there.
+#ifndef IS_SMALL_VECS
+#define IS_SMALL_VECS IS_INJECT_VECS
+#endif
+#ifndef IS_SMALL_MIN_BLOCKS
+#define IS_SMALL_MIN_BLOCKS IS_INJECT_MIN_BLOCKS
+#endif
+constexpr int kSmallVecsPerThread = IS_SMALL_VECS;
+constexpr int kSmallMinBlocks = IS_SMALL_MIN_BLOCKS;
 constexpr int kDefaultMaxRequests = 4096;
 constexpr int kDefaultMaxFactIds = 1 << 20;
 constexpr int kMaxTimedLaunches = 4096;
@@ -139,6 +149,7 @@ struct is_store {
   int32_t shard_max_len = 0;
   // kernel configuration
   int inject_grid = 0;
+  int small_grid = 0;        // resident CTAs of the single-kernel path
   int32_t small_limit = isk::kSmallRequests;  // batches up to this many requests: one kernel
 };
 
@@ -248,8 +259,8 @@ void* inject_fn() {
 
 template <int D, int STYLE, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0, int FAST = 0>
 void* small_fn() {
-  return reinterpret_cast<void*>(&isk::small_inject_kernel<D, STYLE, kInjectThreads, kVecsPerThread,
-                                                           kInjectMinBlocks, POW2, HOST_TIER, HC, BC, FAST>);
+  return reinterpret_cast<void*>(&isk::small_inject_kernel<D, STYLE, kInjectThreads, kSmallVecsPerThread,
+                                                           kSmallMinBlocks, POW2, HOST_TIER, HC, BC, FAST>);
 }
 
 template <bool POW2, bool HOST_TIER = false>
@@ -527,6 +538,10 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
   int per_sm = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kInjectThreads, cs_smem_bytes(c.head_dim, 16));
   s->inject_grid = std::max(1, per_sm) * s->sm_count;
+  int per_sm_small = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_small, pick_small_t<true>(c.head_dim, c.rope_style),
+                                                kInjectThreads, cs_smem_bytes(c.head_dim, 16));
+  s->small_grid = std::max(1, per_sm_small) * s->sm_count;
   if (cudaDeviceSynchronize() != cudaSuccess || cudaGetLastError() != cudaSuccess) {
     free_store(s);
     return IS_ERR_CUDA;
@@ -1174,7 +1189,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   const bool per_slot = s->host_arena || view;
   void* fn = small ? pick_small(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop)
                    : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop);
-  int32_t small_R = R, small_ids = num_ids, small_grid = s->inject_grid, small_blocks = s->max_blocks;
+  int32_t small_R = R, small_ids = num_ids, small_grid = s->small_grid, small_blocks = s->max_blocks;
   int64_t small_cap = slot_cap;
   void* small_args[] = {&ia, &small_R, &small_ids, &small_cap, &small_grid, &small_blocks};
   void* args[] = {&ia};
@@ -1192,7 +1207,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   if (ev) cudaEventRecord(ev->start, st);
   if (small) {
     // One kernel composes and injects the whole small batch.
-    e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), small_args, smem, st);
+    e = cudaLaunchKernel(fn, dim3(unsigned(s->small_grid)), dim3(kInjectThreads), small_args, smem, st);
   } else if (ev) {
     // Timed: events bracket the inject kernel alone (no early launch).
     e = cudaLaunchKernel(fn, dim3(unsigned(s->inject_grid)), dim3(kInjectThreads), args, smem, st);
@@ -1261,21 +1276,22 @@ static int host_batch(is_store_t* s, int32_t R, const int32_t* req_off, const in
     return rc;
   }
   // The next batch's cold facts move over the host link while this one runs.
-  if (lru && num_next > 0 && (rc = lru_prefetch(s, next_ids, num_next)) != IS_OK) return rc;
-  if (slot_out && slot_cap > 0 &&
-      cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost, st) !=
-          cudaSuccess)
-    return IS_ERR_CUDA;
+  // (A failure here is reported after this batch has been completed: its
+  // pending promotions must still enter the hot table.)
+  const int rc_pf = (lru && num_next > 0) ? lru_prefetch(s, next_ids, num_next) : IS_OK;
+  bool copied = !(slot_out && slot_cap > 0) ||
+                cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost,
+                                st) == cudaSuccess;
   // Status back in the same stream, then one wait.
-  if (cudaMemcpyAsync(s->host_status, s->d_status, sizeof(isk::DevStatus), cudaMemcpyDeviceToHost, st) !=
-          cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return IS_ERR_CUDA;
-  const int code = s->host_status->code;
+  copied = copied && cudaMemcpyAsync(s->host_status, s->d_status, sizeof(isk::DevStatus),
+                                     cudaMemcpyDeviceToHost, st) == cudaSuccess;
+  const bool waited = cudaStreamSynchronize(st) == cudaSuccess;
+  const int code = (copied && waited) ? s->host_status->code : IS_ERR_CUDA;
   if (s->pend_np > 0 && (lru_finish(s, st, code == 0) != IS_OK || cudaStreamSynchronize(st) != cudaSuccess))
     return IS_ERR_CUDA;
+  if (!copied || !waited) return IS_ERR_CUDA;
   if (code != 0 && cudaMemset(s->d_status, 0, sizeof(isk::DevStatus)) != cudaSuccess) return IS_ERR_CUDA;
-  return code;
+  return code != IS_OK ? code : rc_pf;
 }
 
 int is_inject_batch_host(is_store_t* s, int32_t R, const int32_t* req_off, const int32_t* fact_ids,
