@@ -223,8 +223,8 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     int32_t* s_start = s_blk0 + (a.R + 1);   // [R]
     int32_t* s_nblk = s_start + a.R;         // [R]
     int32_t* s_len = s_nblk + a.R;           // [R]
-    int32_t* s_valid = s_len + a.R;          // [R]
-    int32_t* s_seg = s_valid + a.R;          // [num_ids]
+    int32_t* s_err = s_len + a.R;            // [R]
+    int32_t* s_seg = s_err + a.R;            // [num_ids]
     for (int i = tid; i <= a.R; i += NT) s_off[i] = a.req_off[i];
     for (int i = tid; i < a.R; i += NT) s_start[i] = a.start_pos[i];
     __syncthreads();
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     req_blk0 = s_blk0;
     req_tok0 = s_tok0;
     req_len = s_len;
-    req_err = s_valid;
+    req_err = s_err;
   }
 
   // The CSR must start at 0, end at num_ids and never decrease; otherwise
@@ -391,19 +391,24 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   const bool over_slots = (a.slot_out != nullptr && total_tokens > a.slot_cap) || s_len_over;
   const bool over_blocks = s_total_blk > a.max_batch_blocks;
 
+  // Work units are counted in 32 bits: a batch needing more is over capacity.
+  __shared__ int s_over_units;
   if (tid == 0) {
     int32_t rpu, upb;
     unit_size(total_blocks, a.L, a.H, a.grid_ctas, a.row_units != 0, rpu, upb);
+    s_over_units = (long long)total_blocks * upb > 0x7fffffffLL;
+    const bool over = over_slots || over_blocks || s_over_units;
     a.hdr->rows_per_unit = rpu;
     a.hdr->units_per_block = upb;
     a.hdr->total_blocks = total_blocks;
     a.hdr->total_tokens = total_tokens;
     a.hdr->next_unit = 0;
-    a.hdr->total_units = (over_slots || over_blocks) ? 0 : total_blocks * upb;
+    a.hdr->total_units = over ? 0 : total_blocks * upb;
     // A batch over capacity writes nothing and reports only that.
-    if (over_slots || over_blocks) record_error(a.st, kErrCapacity, total_tokens);
+    if (over) record_error(a.st, kErrCapacity, total_tokens);
   }
-  if (over_slots || over_blocks) return;
+  __syncthreads();
+  if (over_slots || over_blocks || s_over_units) return;
 
   // Phase 3, one warp per request: block descriptors (lanes over blocks, so
   // a warp writes consecutive descriptors), the check of every touched
@@ -431,22 +436,34 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
       // Lanes over blocks: the block's first fact is the last j with seg[j]
       // <= its first index (binary search in shared memory); a warp writes
       // consecutive descriptors.
-      for (int32_t bi = lane; bi < nblk; bi += 32) {
-        // the table entry's load is issued first: it overlaps the search
-        const int32_t phys = a.block_tables[(long long)r * a.max_blocks + fb + bi];
-        const int32_t i0 = bi == 0 ? 0 : (fb + bi) * a.B - start;
-        int32_t lo = j0, hi = j1 - 1;  // seg[j0] = 0 <= i0
-        while (lo < hi) {
-          const int32_t mid = (lo + hi + 1) >> 1;
-          if (seg[mid] <= i0) lo = mid; else hi = mid - 1;
+      // Four blocks per lane per round; their table entries are loaded first,
+      // so the loads are in flight together and overlap the searches.
+      constexpr int PB = 4;
+      for (int32_t base = lane; base < nblk; base += 32 * PB) {
+        int32_t phys[PB];
+#pragma unroll
+        for (int q = 0; q < PB; ++q) {
+          const int32_t bi = base + 32 * q;
+          phys[q] = bi < nblk ? a.block_tables[(long long)r * a.max_blocks + fb + bi] : 0;
         }
-        BlockDesc d;
-        d.r = r;
-        d.b = fb + bi;
-        d.j = lo;
-        d.pad = 0;
-        a.desc[g0 + bi] = d;
-        check_entry(r, fb + bi, phys);
+#pragma unroll
+        for (int q = 0; q < PB; ++q) {
+          const int32_t bi = base + 32 * q;
+          if (bi >= nblk) break;
+          const int32_t i0 = bi == 0 ? 0 : (fb + bi) * a.B - start;
+          int32_t lo = j0, hi = j1 - 1;  // seg[j0] = 0 <= i0
+          while (lo < hi) {
+            const int32_t mid = (lo + hi + 1) >> 1;
+            if (seg[mid] <= i0) lo = mid; else hi = mid - 1;
+          }
+          BlockDesc d;
+          d.r = r;
+          d.b = fb + bi;
+          d.j = lo;
+          d.pad = 0;
+          a.desc[g0 + bi] = d;
+          check_entry(r, fb + bi, phys[q]);
+        }
       }
     } else {
       // Lanes over facts (no dependent L2 reads): fact j [s, e) owns the
