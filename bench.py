@@ -272,7 +272,7 @@ def _synth():
 def workload_config(wl, name="llama-batch", extra=None):
     m, b = wl.model, wl.batch
     cfg = {"workload": WORKLOADS[name][0],
-           "model_shapes": m.name, "layers": m.num_layers, "kv_heads": m.num_kv_heads,
+           "shapes": m.name, "layers": m.num_layers, "kv_heads": m.num_kv_heads,
            "head_dim": m.head_dim,
            "rope": f"theta {m.rope_theta:g}" + (", llama3 scaling (8, 1, 4, 8192)" if m.llama3 else ""),
            "requests": b.num_requests, "k": int(b.req_offsets[1] - b.req_offsets[0]),
@@ -683,7 +683,7 @@ def run_sweep(args, rank, world, local_rank):
             if rank == 0:
                 print(json.dumps({
                     "metric": METRIC, "workload": WORKLOADS[args.workload][0].split(",")[0],
-                    "model_shapes": model.name, "requests": R, "k": k, "tokens_per_batch": n_tok,
+                    "shapes": model.name, "requests": R, "k": k, "tokens_per_batch": n_tok,
                     "steps": steps, "l2": "flushed before every step" if flush else "reads > 4x L2",
                     "us_per_batch": ms / steps * 1e3, "tokens_per_s": n_tok / (ms / steps / 1e3),
                     "kernel_us": kern * 1e3,
