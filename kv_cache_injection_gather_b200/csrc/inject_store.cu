@@ -370,6 +370,24 @@ int grow_stage(is_store* s, size_t elems, int64_t slot_elems) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Device address of host range [p, p + bytes) when the whole range is
+// page-locked host memory mapped for the current device (cudaHostAlloc,
+// cudaMallocHost or a mapped registration), else nullptr.  Both ends are
+// looked up and must lie in one contiguous mapping.
+void* mapped_host_range(void* p, size_t bytes) {
+  if (!p || bytes == 0) return nullptr;
+  cudaPointerAttributes a{}, b{};
+  void* last = static_cast<char*>(p) + (bytes - 1);
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess || cudaPointerGetAttributes(&b, last) != cudaSuccess) {
+    cudaGetLastError();  // a failed lookup is not a CUDA error of the call
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || b.type != cudaMemoryTypeHost || !a.devicePointer || !b.devicePointer)
+    return nullptr;
+  if (static_cast<char*>(b.devicePointer) != static_cast<char*>(a.devicePointer) + (bytes - 1)) return nullptr;
+  return a.devicePointer;
+}
+
 // Vector order of the inject kernel for a cache layout: the row index with
 // the larger cache stride runs fastest (token-major: slots; head-major:
 // heads).
@@ -1244,7 +1262,12 @@ static int host_batch(is_store_t* s, int32_t R, const int32_t* req_off, const in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t n_off = size_t(R) + 1, n_ids = size_t(num_ids), n_sp = size_t(R);
   const size_t n_bt = size_t(R) * size_t(max_blocks_per_req);
-  const int64_t n_slots = slot_out ? slot_cap : 0;
+  // A slot mapping in page-locked host memory is written in place by the
+  // kernels (its bytes cross the host link while the batch runs, no copy
+  // follows); any other host buffer gets a device buffer and a copy back.
+  int64_t* direct_slots = (slot_out && slot_cap > 0)
+      ? static_cast<int64_t*>(mapped_host_range(slot_out, size_t(slot_cap) * 8)) : nullptr;
+  const int64_t n_slots = (slot_out && !direct_slots) ? slot_cap : 0;
   int rc = grow_stage(s, n_off + n_ids + n_sp + n_bt + 4, n_slots);
   if (rc != IS_OK) return rc;
   const bool lru = s->hot_policy == IS_HOT_LRU;
@@ -1269,7 +1292,7 @@ static int host_batch(is_store_t* s, int32_t R, const int32_t* req_off, const in
   }
   s->batch_pend = s->pend_np > 0;
   rc = is_inject_batch(s, R, d_off, d_ids, num_ids, d_sp, d_bt, max_blocks_per_req, cache,
-                       slot_out ? s->stage_slots : nullptr, slot_cap, stream);
+                       direct_slots ? direct_slots : slot_out ? s->stage_slots : nullptr, slot_cap, stream);
   s->batch_pend = false;
   if (rc != IS_OK) {
     lru_finish(s, st, false);  // nothing ran: copy the promoted facts instead
@@ -1279,7 +1302,7 @@ static int host_batch(is_store_t* s, int32_t R, const int32_t* req_off, const in
   // (A failure here is reported after this batch has been completed: its
   // pending promotions must still enter the hot table.)
   const int rc_pf = (lru && num_next > 0) ? lru_prefetch(s, next_ids, num_next) : IS_OK;
-  bool copied = !(slot_out && slot_cap > 0) ||
+  bool copied = !(slot_out && slot_cap > 0) || direct_slots ||
                 cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost,
                                 st) == cudaSuccess;
   // Status back in the same stream, then one wait.

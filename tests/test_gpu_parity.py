@@ -346,6 +346,48 @@ def test_host_entry_point_matches_device_entry_point():
     store.close()
 
 
+def test_host_entry_point_slot_buffers():
+    """The slot mapping of the host entry point: a pinned buffer is written in
+    place (entries past the batch's tokens untouched, nothing at all on
+    CAPACITY); a pageable buffer gets the same slots through a copy."""
+    _need_gpu()
+    wl = _ragged(synth.Model("h", 2, 4, 128, 1e6), seed=12)
+    store = make_store(wl)
+    b = wl.batch
+    n_tok = wl.tokens()
+    o = oracle_run(wl)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
+    args = (pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos), pin(b.block_tables))
+    sentinel = 0x5A5A5A5A5A5A5A5A
+    # pinned, with room to spare
+    k, v, d = make_cache(wl)
+    buf = torch.full((n_tok + 37,), sentinel, dtype=torch.int64).pin_memory()
+    rc = store.inject_host(*args, d, buf)
+    assert_parity(o, (rc, buf[:n_tok].numpy().copy(), to_bits(k), to_bits(v)))
+    assert (buf[n_tok:] == sentinel).all()
+    # a pinned slice that starts inside the allocation
+    k, v, d = make_cache(wl)
+    buf = torch.full((n_tok + 64,), sentinel, dtype=torch.int64).pin_memory()
+    rc = store.inject_host(*args, d, buf[13:13 + n_tok])
+    assert_parity(o, (rc, buf[13:13 + n_tok].numpy().copy(), to_bits(k), to_bits(v)))
+    assert (buf[:13] == sentinel).all() and (buf[13 + n_tok:] == sentinel).all()
+    # pageable
+    k, v, d = make_cache(wl)
+    page = torch.full((n_tok,), sentinel, dtype=torch.int64)
+    assert not page.is_pinned()
+    rc = store.inject_host(*args, d, page)
+    assert_parity(o, (rc, page.numpy().copy(), to_bits(k), to_bits(v)))
+    # pinned, one entry short: CAPACITY, buffer and cache untouched
+    k, v, d = make_cache(wl)
+    k0, v0 = k.clone(), v.clone()
+    buf = torch.full((n_tok,), sentinel, dtype=torch.int64).pin_memory()
+    rc = store.inject_host(*args, d, buf[:n_tok - 1])
+    assert rc == oracle.ERR_CAPACITY
+    assert (buf == sentinel).all()
+    assert torch.equal(k, k0) and torch.equal(v, v0)
+    store.close()
+
+
 def test_store_put_read_and_arena():
     _need_gpu()
     wl = synth.tiny(0)
