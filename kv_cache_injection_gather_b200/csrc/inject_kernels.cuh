@@ -97,11 +97,12 @@ __device__ __forceinline__ void record_error(DevStatus* st, int32_t code, long l
 // Work-unit size: rows per unit rpu and units per block upb, where a row is
 // one (layer, head) pair of a cache block, numbered w = layer * H + head, and
 // unit g of a block covers rows [g * rpu, min(L * H, (g + 1) * rpu)).  A batch
-// whose one-layer units fit in about two waves of the grid is split into
-// about one wave of units (latency: everything is in flight at once and no
-// CTA runs a second unit after the first): with row_units (the per-thread
-// copy loops, which take any row range) into equal row ranges, otherwise
-// into equal layer ranges.  Larger batches aim at ~IS_UNITS_PER_CTA units
+// whose one-layer units fit in about two waves of the grid is split into at
+// most one wave of units (latency: everything is in flight at once and no
+// CTA runs a second unit after the first -- one more unit than the grid
+// holds doubles the time of a single request), as many as fit: with
+// row_units (the per-thread copy loops, which take any row range) into
+// equal row ranges, otherwise into equal layer ranges.  Larger batches aim at ~IS_UNITS_PER_CTA units
 // per CTA, so the dynamic schedule's tail (at most one unit) stays short,
 // in whole layers with at least IS_UNIT_MIN_ROWS rows (and at least two
 // layers) per unit so a unit's set-up (slot walk, cos/sin table, barriers)
@@ -114,17 +115,18 @@ __device__ __forceinline__ void unit_size(int32_t total_blocks, int32_t L, int32
                                           bool row_units, int32_t& rpu, int32_t& upb) {
   const long long grid = grid_ctas;
   const int32_t LH = L * H;
-  if (total_blocks > 0 && row_units && (long long)total_blocks * L <= 2 * grid) {
-    const long long per = ((long long)total_blocks * LH + grid - 1) / grid;  // rows per unit
-    upb = int32_t((LH + per - 1) / per);
-    rpu = (LH + upb - 1) / upb;
-    upb = (LH + rpu - 1) / rpu;
-    return;
-  }
   upb = 1;
   if (total_blocks > 0 && (long long)total_blocks * L <= 2 * grid) {
-    const long long per = ((long long)total_blocks * L + grid - 1) / grid;  // 1 or 2 layers per unit
-    upb = int32_t((L + per - 1) / per);
+    // units per block such that every unit has a CTA of its own (ceil-ing
+    // the range lengths below only lowers the count)
+    const int32_t fit = max(1, grid_ctas / total_blocks);
+    if (row_units) {
+      upb = min(LH, fit);
+      rpu = (LH + upb - 1) / upb;
+      upb = (LH + rpu - 1) / rpu;
+      return;
+    }
+    upb = min(L, fit);
   } else if (total_blocks > 0) {
     const int32_t h = max(H, 1);
     const int32_t lmin = min(L, max(2, (IS_UNIT_MIN_ROWS + h - 1) / h));
@@ -1270,7 +1272,7 @@ struct SmallPlan {
   int32_t err[kSmallRequests];
   int32_t nblk[kSmallRequests];
   int32_t blk0[kSmallRequests + 1];
-  int32_t bad, total_units, total_blocks, rpu;
+  int32_t total_units, total_blocks, rpu;
 };
 
 template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0,
@@ -1304,24 +1306,23 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     p.len[tid] = lf;
     len = id_ok ? lf : 0;
   }
-  if (tid == 0) {
-    p.bad = 0;
-    s_bad_ids = 0u;
-  }
-  // CSR: starts at 0, ends at num_ids, never decreases.
+  if (tid == 0) s_bad_ids = 0u;
+  // Block size: a shift when it is a power of two.  The plan's sums fit 32
+  // bits: the batch's ids total at most kSmallTokens tokens (the host's
+  // bound), and start + segment <= max_blocks * B < 2^31 once checked.
+  const int lb = POW2 ? ilog2(a.B) : 0;
+  auto div_b = [&](int32_t x) { return POW2 ? (x >> lb) : x / a.B; };
   __syncthreads();
-  if ((tid < R && p.roff[tid + 1] < p.roff[tid]) || (tid == 0 && (p.roff[0] != 0 || p.roff[R] != num_ids)))
-    p.bad = 1;
-  __syncthreads();
-  if (p.bad) {
-    if (reporter && tid == 0) record_error(a.st, kErrInvalidArg, -1);
-    return;
-  }
+  // The CSR must start at 0, end at num_ids and never decrease (checked
+  // with the scan's barrier below; until then nothing leaves shared memory
+  // but L2 prefetches of table rows inside the table).
+  const bool csr_bad = (tid < R && p.roff[tid + 1] < p.roff[tid]) ||
+                       (tid == 0 && (p.roff[0] != 0 || p.roff[R] != num_ids));
   // Warm L2 with the block-table lines of each request's first blocks (up to
   // 128 entries), read later by every unit's slot set-up.
   if (tid < R * 4) {
     const int r = tid >> 2, st0 = p.start[r];
-    const int b = (st0 >= 0 ? st0 / a.B : a.max_blocks) + 32 * (tid & 3);
+    const int b = (st0 >= 0 ? div_b(st0) : a.max_blocks) + 32 * (tid & 3);
     if (b < a.max_blocks)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(a.block_tables + (long long)r * a.max_blocks + b));
   }
@@ -1329,7 +1330,8 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   int myr = 0;
   while (myr + 1 < R && p.roff[myr + 1] <= tid) ++myr;
   if (tid < num_ids && !id_ok) atomicOr(&s_bad_ids, 1u << myr);
-  // Exclusive prefix of the lengths over the batch.
+  // Exclusive prefix of the lengths over the batch: warp scans, then the
+  // warps' totals.
   int32_t x = len;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -1337,39 +1339,58 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     if (lane >= d) x += y;
   }
   if (lane == 31) s_wsum[warp] = x;
-  __syncthreads();
-  int32_t wbase = 0;
-  for (int w = 0; w < warp; ++w) wbase += s_wsum[w];
+  if (__syncthreads_or(csr_bad)) {
+    if (reporter && tid == 0) record_error(a.st, kErrInvalidArg, -1);
+    return;
+  }
+  int32_t ws = lane < NT / 32 ? s_wsum[lane] : 0;
+#pragma unroll
+  for (int d = 1; d < NT / 32; d <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, ws, d);
+    if (lane >= d) ws += y;
+  }
+  const int32_t wbase = warp > 0 ? __shfl_sync(0xffffffffu, ws, warp - 1) : 0;
   p.pref[tid] = wbase + x - len;
   if (tid == NT - 1) p.pref[NT] = wbase + x;  // so p.pref[num_ids] is the batch total
   __syncthreads();
-  // Per request: validity and touched blocks.
-  if (tid < R) {
-    const int r = tid, j0 = p.roff[r], j1 = p.roff[r + 1];
-    const long long S = p.pref[j1] - p.pref[j0];
-    int32_t err = (s_bad_ids >> r) & 1u ? kErrBadFactId : kOk;
-    if (err == kOk && p.start[r] < 0) err = kErrInvalidArg;
-    if (err == kOk && (long long)p.start[r] + S > (long long)a.max_blocks * a.B) err = kErrPosition;
-    p.err[r] = err;
-    p.nblk[r] = (err == kOk && S > 0) ? int32_t((p.start[r] + S - 1) / a.B - p.start[r] / a.B + 1) : 0;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int32_t acc = 0;
-    for (int r = 0; r < R; ++r) { p.blk0[r] = acc; acc += p.nblk[r]; }
-    p.blk0[R] = acc;
-    const long long total_tokens = p.pref[num_ids];
-    // the same limits as the two-kernel path, so results never depend on
-    // which path a batch takes
-    const bool over = (a.slot_out != nullptr && total_tokens > slot_cap) || acc > max_batch_blocks;
-    int32_t rpu, upb;
-    unit_size(acc, a.L, a.H, grid_ctas, FAST != 0, rpu, upb);
-    p.rpu = rpu;
-    p.total_blocks = acc;
-    p.total_units = over ? 0 : acc * upb;
-    // A batch over capacity writes nothing and reports only that.
-    if (reporter && over) record_error(a.st, kErrCapacity, total_tokens);
-    s_err_key = ~0ull;
+  // Warp 0, lane r per request: validity, touched blocks and their prefix;
+  // lane 0 then sizes the work units.
+  if (warp == 0) {
+    const int r = lane;
+    int32_t err = kOk, nblk = 0;
+    if (r < R) {
+      const int32_t st0 = p.start[r];
+      const int32_t S = p.pref[p.roff[r + 1]] - p.pref[p.roff[r]];
+      err = (s_bad_ids >> r) & 1u ? kErrBadFactId : kOk;
+      if (err == kOk && st0 < 0) err = kErrInvalidArg;
+      if (err == kOk && (long long)st0 + S > (long long)a.max_blocks * a.B) err = kErrPosition;
+      if (err == kOk && S > 0) nblk = div_b(st0 + S - 1) - div_b(st0) + 1;
+      p.err[r] = err;
+      p.nblk[r] = nblk;
+    }
+    int32_t acc = nblk;  // inclusive prefix over requests
+#pragma unroll
+    for (int d = 1; d < kSmallRequests; d <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, acc, d);
+      if (lane >= d) acc += y;
+    }
+    if (r < R) p.blk0[r] = acc - nblk;
+    const int32_t total = __shfl_sync(0xffffffffu, acc, kSmallRequests - 1);
+    if (lane == 0) {
+      p.blk0[R] = total;
+      const int32_t total_tokens = p.pref[num_ids];
+      // the same limits as the two-kernel path, so results never depend on
+      // which path a batch takes
+      const bool over = (a.slot_out != nullptr && total_tokens > slot_cap) || total > max_batch_blocks;
+      int32_t rpu, upb;
+      unit_size(total, a.L, a.H, grid_ctas, FAST != 0, rpu, upb);
+      p.rpu = rpu;
+      p.total_blocks = total;
+      p.total_units = over ? 0 : total * upb;
+      // A batch over capacity writes nothing and reports only that.
+      if (reporter && over) record_error(a.st, kErrCapacity, total_tokens);
+      s_err_key = ~0ull;
+    }
   }
   // Segment offsets inside each request.
   if (tid < num_ids) p.seg[tid] = p.pref[tid] - p.pref[p.roff[myr]];
@@ -1392,7 +1413,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     for (int gb = tid; gb < p.total_blocks; gb += NT) {
       int r = 0;
       while (r + 1 < R && p.blk0[r + 1] <= gb) ++r;
-      const int b = p.start[r] / a.B + (gb - p.blk0[r]);
+      const int b = div_b(p.start[r]) + (gb - p.blk0[r]);
       const int32_t phys = a.block_tables[(long long)r * a.max_blocks + b];
       if (phys < 0 || phys >= a.num_blocks) atomicMin(&s_err_key, ((unsigned long long)r << 32) | unsigned(b));
     }
@@ -1412,7 +1433,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     int r = 0;
     while (r + 1 < R && p.blk0[r + 1] <= gb) ++r;
     const int start = p.start[r];
-    const int b = start / a.B + (gb - p.blk0[r]);
+    const int b = div_b(start) + (gb - p.blk0[r]);
     const int j0 = p.roff[r], j1 = p.roff[r + 1];
     const int i_first = max(0, b * a.B - start);
     int lo = j0, hi = j1 - 1;  // last fact with seg <= i_first

@@ -7,9 +7,9 @@ block, row = layer * H + head:
 
   * the row ranges of a block's units partition [0, L * H), none empty;
   * without row units (the generic copy loop) every range is whole layers;
-  * a batch whose one-layer units fit in two waves gets about one wave of
-    units (latency): at most the grid plus one unit per block, since rows
-    (or layers) are grouped in equal ranges;
+  * a batch whose one-layer units fit in two waves gets at most one wave of
+    units (latency: no CTA runs a second unit), one unit per block when the
+    blocks alone outnumber the grid;
   * a large batch gets units of whole layers, at least 16 rows and two
     layers whenever the model has them, with or without row units;
   * the unit count fits the kernels' 32-bit counters.
@@ -23,15 +23,14 @@ UNITS_PER_CTA, MIN_ROWS, ROWS_LARGE, UNITS_PER_CTA_MIN = 256, 16, 32, 32
 
 def unit_size(total_blocks: int, L: int, H: int, grid: int, row_units: bool = False):
     LH = L * H
-    if total_blocks > 0 and row_units and total_blocks * L <= 2 * grid:
-        per = (total_blocks * LH + grid - 1) // grid
-        upb = (LH + per - 1) // per
-        rpu = (LH + upb - 1) // upb
-        return rpu, (LH + rpu - 1) // rpu
     upb = 1
     if total_blocks > 0 and total_blocks * L <= 2 * grid:
-        per = (total_blocks * L + grid - 1) // grid
-        upb = (L + per - 1) // per
+        fit = max(1, grid // total_blocks)
+        if row_units:
+            upb = min(LH, fit)
+            rpu = (LH + upb - 1) // upb
+            return rpu, (LH + rpu - 1) // rpu
+        upb = min(L, fit)
     elif total_blocks > 0:
         h = max(H, 1)
         lmin = min(L, max(2, (MIN_ROWS + h - 1) // h))
@@ -62,7 +61,11 @@ def test_unit_sizing_invariants():
         if not rows:
             assert all(a % H == 0 and (b % H == 0) for a, b in ranges), "whole layers"
         if tb * L <= 2 * grid:
-            assert tb * upb <= grid + tb, "one-wave batch: about one wave of units"
+            assert tb * upb <= max(grid, tb), "one-wave batch: at most one unit per CTA"
+            # and not needlessly large: ranges one row (layer) shorter would
+            # overflow the grid, or the units are single rows (layers)
+            n, q = (LH, rpu) if rows else (L, rpu // H)
+            assert q == 1 or tb * -(-n // (q - 1)) > grid
         else:
             assert rpu % H == 0, "large batches: whole layers"
             assert rpu // H >= min(L, 2)
@@ -80,3 +83,7 @@ def test_unit_sizing_at_the_benchmark_shapes():
     # two layers, row units 290 units of 9 rows
     assert unit_size(10, 32, 8, 296) == (16, 16)
     assert unit_size(10, 32, 8, 296, True) == (9, 29)
+    # 15 blocks (a request of ~240 tokens): 285 units of 14 rows, not 300 of
+    # 13 (four CTAs would run a second unit)
+    assert unit_size(15, 32, 8, 296, True) == (14, 19)
+    assert unit_size(13, 28, 4, 296, True) == (6, 19)
