@@ -460,6 +460,23 @@ def test_llama_single_request_full_store():
     assert_parity((rc, slots, kc, vc, kref), g)
 
 
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("nblk", [13, 15, 16, 17, 18])
+def test_llama_single_request_block_counts(nblk, path):
+    """One Llama-3.1-8B request of k=5 after a 64-token prefix touching nblk
+    cache blocks (the last one half full).  With one wave of work units per
+    batch this size, 15 to 17 blocks are where rounding the units' row ranges
+    once gave more units than the 296-CTA grid; every count, on both paths,
+    gives the oracle's cache."""
+    k = 5
+    T = 16 * nblk - 8
+    lens = np.array([T // k + (i < T % k) for i in range(k)], np.int32)
+    batch = synth.make_batch(np.random.default_rng(nblk), [np.arange(k)], 64, 16, 24, 24)
+    wl = synth.Workload("llama-blocks", synth.LLAMA31_8B, lens, batch, seed=nblk)
+    assert wl.tokens() == T
+    assert_parity(oracle_run(wl), gpu_run(wl, path=path))
+
+
 def test_head_sharded_stores_reproduce_the_full_cache():
     """KV-head shards (the multi-GPU tensor-parallel partition): a store and
     cache holding heads [h0, h1) only, fed the whole batch, produce exactly
