@@ -242,8 +242,8 @@ WORKLOADS = {
                                                             slots_per_request=1024)),
     "llama-batch-distinct-small": ("llama3.1-8b-shapes 600-fact store, 9 requests x k=22, no fact "
                                    "repeated in the batch, block 16, cache 864 blocks (profiling "
-                                   "case for DRAM traffic of the plan + inject path, ~5 GB on the "
-                                   "device)",
+                                   "case for DRAM traffic of the plan + inject path with "
+                                   "--small-limit 0, ~5 GB on the device)",
                                    lambda seed: _synth().llama_batch(seed, num_facts=600, R=9, k=22,
                                                                      slots_per_request=1536,
                                                                      distinct_batch=True)),
@@ -627,6 +627,16 @@ SWEEP_R = (1, 16, 100, 256)
 SWEEP_K = (5, 10, 20, 50)
 
 
+SMALL_REQUESTS, SMALL_IDS = 32, 256  # the library's single-kernel limits (default)
+
+
+def single_kernel(R, num_ids, longest, limit=None):
+    """Whether the library runs a batch as its one fused kernel: at most
+    `limit` (default 32) requests and 256 ids, 32-bit token sums."""
+    lim = SMALL_REQUESTS if limit is None else limit
+    return R <= lim and num_ids <= SMALL_IDS and num_ids * longest < 2 ** 31
+
+
 def run_sweep(args, rank, world, local_rank):
     """Every (R, k) point of the Mistral / Qwen sweep with one store: the
     sweep's fact lengths come first from its seed, so every point draws from
@@ -680,6 +690,16 @@ def run_sweep(args, rank, world, local_rank):
             kern_ms, kern_n = store.kernel_time()
             store.set_timing(False)
             kern = kern_ms / max(kern_n, 1)
+            extra = {}
+            if single_kernel(R, len(wl.batch.fact_ids), int(wl.fact_lens.max())):
+                # the same batch through the plan + inject kernels, for the path choice
+                store.set_small_batch_limit(0)
+                for _ in range(args.warmup):
+                    step()
+                torch.cuda.synchronize(dev)
+                ms2 = timed_steps(step, steps, stream, flush)
+                store.set_small_batch_limit(SMALL_REQUESTS)
+                extra = {"path": "single kernel", "two_kernel_us_per_batch": ms2 / steps * 1e3}
             if rank == 0:
                 print(json.dumps({
                     "metric": METRIC, "workload": WORKLOADS[args.workload][0].split(",")[0],
@@ -688,7 +708,7 @@ def run_sweep(args, rank, world, local_rank):
                     "us_per_batch": ms / steps * 1e3, "tokens_per_s": n_tok / (ms / steps / 1e3),
                     "kernel_us": kern * 1e3,
                     "kernel_frac_of_peak": 2 * read_bytes / (kern / 1e3) / 1e9 / peak,
-                    "peak_gbs": peak, "peak_source": f"{peak_kind} hbm_gbs"}), flush=True)
+                    "peak_gbs": peak, "peak_source": f"{peak_kind} hbm_gbs", **extra}), flush=True)
             del kc, vc, desc, slots
             torch.cuda.empty_cache()
     store.close()
@@ -738,7 +758,8 @@ def run_ours(args, rank, world, local_rank):
     else:
         wl = WORKLOADS[args.workload][1](rank)
     store = make_store(wl, on_device_gen=True, device=local_rank, heads=heads,
-                       facts=None if owner is None else shard.owned_facts(owner, rank))
+                       facts=None if owner is None else shard.owned_facts(owner, rank),
+                       small_limit=args.small_limit)
     group = None
     if owner is not None:
         if world > 1:
@@ -753,6 +774,9 @@ def run_ours(args, rank, world, local_rank):
     kcache, vcache, desc = make_cache(wl, device=local_rank, fill=False, head_major=args.head_major,
                                       num_kv_heads=None if heads is None else heads[1] - heads[0])
     extra_cfg["cache_layout"] = "[L][num_blocks][H][B][D]" if args.head_major else "[L][num_blocks][B][H][D]"
+    extra_cfg["path"] = ("single fused kernel" if single_kernel(
+        b.num_requests, len(b.fact_ids), int(wl.fact_lens.max()), args.small_limit)
+        else "plan + inject kernels")
     copy_ref, copy_sus = copy_probe(dev)
     # every rank takes part in the same collectives, in the same order
     peer_gbs = peer_probe(dev, world) if (owner is not None and world > 1) else None
@@ -883,11 +907,10 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": tokens_all / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
-        # the library's kernels per step: one fused kernel for batches of at
-        # most 8 requests, 256 ids and 6 144 tokens by the bound (ids x the
-        # longest fact), else the plan and the inject kernel
-        "gpu_launches": (1 if (b.num_requests <= 8 and len(b.fact_ids) <= 256 and
-                               len(b.fact_ids) * int(wl.fact_lens.max()) <= 6144) else 2) * args.steps,
+        # the library's kernels per step: one fused kernel for a batch the
+        # single-kernel path takes, else the plan and the inject kernel
+        "gpu_launches": (1 if single_kernel(b.num_requests, len(b.fact_ids), int(wl.fact_lens.max()),
+                                            args.small_limit) else 2) * args.steps,
         "roofline": roofline,
         "cpu_baseline": baseline,
     }
@@ -912,6 +935,9 @@ def main():
                          "batch of 100 x N requests (both weak scaling, no collective), or fact "
                          "shards (each rank holds 1/N of the facts and injects 100 requests, "
                          "reading the rest from peers over NVLink)")
+    ap.add_argument("--small-limit", type=int, default=None,
+                    help="batches of up to this many requests (0..32, default 32) run as the "
+                         "single fused kernel; 0: always the plan + inject kernels")
     ap.add_argument("--sweep", action="store_true",
                     help="qwen-sweep / mistral-sweep: every point of R in {1, 16, 100, 256} x k in "
                          "{5, 10, 20, 50} with one store, one JSON line per point")

@@ -357,11 +357,11 @@ int is_last_error(is_store_t* store, void* stream, int64_t* detail_out);
 int is_last_error_timeout(is_store_t* store, void* stream, int32_t timeout_ms,
                           int64_t* detail_out);
 
-/* Batches with at most max_requests requests (0..8; default 8), at most
- * 256 fact ids and at most 6 144 tokens by the bound (ids x the store's
- * longest fact) run as one kernel that composes the batch in every CTA
- * instead of a plan kernel followed by the inject kernel (lower latency for
- * short batches; same results).  0 always uses the two-kernel path. */
+/* Batches with at most max_requests requests (0..32; default 32) and at
+ * most 256 fact ids (whose count times the store's longest fact stays below
+ * 2^31 tokens) run as one kernel that composes the batch in every CTA
+ * instead of a plan kernel followed by the inject kernel (lower latency;
+ * same results).  0 always uses the two-kernel path. */
 int is_store_set_small_batch_limit(is_store_t* store, int32_t max_requests);
 
 /* ---- measurement -------------------------------------------------------- */

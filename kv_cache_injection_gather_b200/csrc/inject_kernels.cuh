@@ -1254,12 +1254,15 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
 // one kernel.  Every CTA of the persistent grid composes the batch itself in
 // shared memory -- the same definitions as plan_kernel (CSR check, lengths,
 // segment offsets, validity, token and block prefixes, work-unit size) --
-// and takes units u = blockIdx.x, blockIdx.x + gridDim.x, ...  The last CTA
-// (the one a small batch leaves without units) alone records the batch's
-// errors and writes the -1 slots of invalid requests.  No work space, no
-// second launch.
-constexpr int kSmallRequests = 8;
-constexpr int kSmallIds = 256;
+// and takes unit blockIdx.x, then units gridDim.x, gridDim.x + 1, ... from
+// a counter (dynamic, as the inject kernel).  The counter pair (next unit,
+// CTAs done) is the store's and starts at zero: the last CTA to leave, when
+// no CTA takes units any more, sets both back to zero for the next batch
+// (batches on one store run one at a time).  The last CTA (the one a small
+// batch leaves without units) alone records the batch's errors and writes
+// the -1 slots of invalid requests.  No work space, no second launch.
+constexpr int kSmallRequests = 32;  // one lane of a warp per request
+constexpr int kSmallIds = 256;      // one thread per fact id
 
 struct SmallPlan {
   long long off[kSmallIds];    // store token offset per CSR entry (valid ids)
@@ -1279,7 +1282,8 @@ template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER
           int FAST = 0>
 __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, int32_t R, int32_t num_ids,
                                                                 int64_t slot_cap, int32_t grid_ctas,
-                                                                int32_t max_batch_blocks) {
+                                                                int32_t max_batch_blocks,
+                                                                unsigned int* ctr) {
   static_assert(NT == kSmallIds, "one thread per fact id");
   extern __shared__ float4 s_cs4[];
   __shared__ UnitShared<HOST_TIER> sm;
@@ -1287,8 +1291,21 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   __shared__ int32_t s_wsum[NT / 32];
   __shared__ unsigned long long s_err_key;
   __shared__ unsigned int s_bad_ids;  // bit r: request r lists an id outside the store
+  __shared__ int s_unit;
+  static_assert(kSmallRequests <= 32, "request bit mask and warp-0 lanes");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool reporter = blockIdx.x == gridDim.x - 1;
+  // Leaving: count this CTA out; the last one resets the unit counter (no
+  // CTA takes a unit after it has counted itself out).
+  auto leave = [&]() {
+    if (tid == 0) {
+      __threadfence();
+      if (atomicAdd(&ctr[1], 1u) == gridDim.x - 1) {
+        atomicExch(&ctr[0], 0u);
+        atomicExch(&ctr[1], 0u);
+      }
+    }
+  };
 
   // Everything the plan reads from the caller is loaded at once: the CSR,
   // the starts, the ids and right behind them their lengths and store
@@ -1326,9 +1343,18 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
     if (b < a.max_blocks)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(a.block_tables + (long long)r * a.max_blocks + b));
   }
+  // Request of the entry at CSR index x (of the block at batch index x):
+  // the last request whose first entry (block) is at or before x.
+  auto request_of = [&](const int32_t* first, int x) {
+    int lo = 0, hi = max(R - 1, 0);
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (first[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
   // This id's request; requests holding an id outside the store.
-  int myr = 0;
-  while (myr + 1 < R && p.roff[myr + 1] <= tid) ++myr;
+  const int myr = request_of(p.roff, tid);
   if (tid < num_ids && !id_ok) atomicOr(&s_bad_ids, 1u << myr);
   // Exclusive prefix of the lengths over the batch: warp scans, then the
   // warps' totals.
@@ -1341,6 +1367,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   if (lane == 31) s_wsum[warp] = x;
   if (__syncthreads_or(csr_bad)) {
     if (reporter && tid == 0) record_error(a.st, kErrInvalidArg, -1);
+    leave();
     return;
   }
   int32_t ws = lane < NT / 32 ? s_wsum[lane] : 0;
@@ -1411,8 +1438,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   if (reporter && !over_cap) {
     if (tid < R && p.err[tid] != kOk) atomicMin(&s_err_key, (unsigned long long)tid << 32);
     for (int gb = tid; gb < p.total_blocks; gb += NT) {
-      int r = 0;
-      while (r + 1 < R && p.blk0[r + 1] <= gb) ++r;
+      const int r = request_of(p.blk0, gb);
       const int b = div_b(p.start[r]) + (gb - p.blk0[r]);
       const int32_t phys = a.block_tables[(long long)r * a.max_blocks + b];
       if (phys < 0 || phys >= a.num_blocks) atomicMin(&s_err_key, ((unsigned long long)r << 32) | unsigned(b));
@@ -1427,11 +1453,18 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   }
 
   const int total_units = p.total_units, total_blocks = p.total_blocks, rpu = p.rpu;
-  for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-    __syncthreads();  // the previous unit's tables are no longer read
+  int next = blockIdx.x;  // the first wave is static
+  for (;;) {
+    __syncthreads();  // the previous unit's tables (and s_unit) are no longer read
+    if (tid == 0) {
+      s_unit = next;
+      if (next < total_units) next = int(gridDim.x + atomicAdd(&ctr[0], 1u));
+    }
+    __syncthreads();
+    const int u = s_unit;
+    if (u >= total_units) break;
     const int gb = u % total_blocks, lg = u / total_blocks;
-    int r = 0;
-    while (r + 1 < R && p.blk0[r + 1] <= gb) ++r;
+    const int r = request_of(p.blk0, gb);
     const int start = p.start[r];
     const int b = div_b(start) + (gb - p.blk0[r]);
     const int j0 = p.roff[r], j1 = p.roff[r + 1];
@@ -1446,6 +1479,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
                                                  p.pref[j1] - p.pref[j0], p.pref[j0], w0,
                                                  min(a.L * a.H, w0 + rpu), lg == 0, p.fid, p.off);
   }
+  leave();
 }
 
 // Host tier, least-recently-used hot set: copy newly promoted facts from the

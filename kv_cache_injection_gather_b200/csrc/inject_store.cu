@@ -46,7 +46,8 @@ constexpr int kSmallMinBlocks = IS_SMALL_MIN_BLOCKS;
 constexpr int kDefaultMaxRequests = 4096;
 constexpr int kDefaultMaxFactIds = 1 << 20;
 constexpr int kMaxTimedLaunches = 4096;
-constexpr int64_t kSmallTokens = 6144;  // single-kernel path: ids x longest fact at most
+// single-kernel path: ids x longest fact below 2^31 (its sums are 32-bit)
+constexpr int64_t kSmallTokens = (int64_t(1) << 31) - 1;
 
 struct TimedLaunch {
   cudaEvent_t start, stop;
@@ -150,6 +151,7 @@ struct is_store {
   // kernel configuration
   int inject_grid = 0;
   int small_grid = 0;        // resident CTAs of the single-kernel path
+  unsigned int* d_small_ctr = nullptr;  // its unit counter pair (zero between batches)
   int32_t small_limit = isk::kSmallRequests;  // batches up to this many requests: one kernel
 };
 
@@ -214,6 +216,7 @@ void free_store(is_store* s) {
   cudaFree(s->ws_desc);
   cudaFree(s->ws_hdr);
   cudaFree(s->d_status);
+  cudaFree(s->d_small_ctr);
   cudaFree(s->stage);
   cudaFree(s->stage_slots);
   cudaFreeHost(s->host_stage);
@@ -515,7 +518,8 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
             dalloc(&s->ws_len, size_t(s->max_req)) == cudaSuccess &&
             dalloc(&s->ws_err, size_t(s->max_req)) == cudaSuccess &&
             dalloc(&s->ws_desc, size_t(s->max_blocks)) == cudaSuccess &&
-            dalloc(&s->ws_hdr, 1) == cudaSuccess && dalloc(&s->d_status, 1) == cudaSuccess;
+            dalloc(&s->ws_hdr, 1) == cudaSuccess && dalloc(&s->d_status, 1) == cudaSuccess &&
+            dalloc(&s->d_small_ctr, 2) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     free_store(s);
@@ -527,6 +531,7 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
   cudaMemset(s->d_off, 0, sizeof(int64_t) * size_t(c.max_facts));
   cudaMemset(s->d_status, 0, sizeof(isk::DevStatus));
   cudaMemset(s->ws_hdr, 0, sizeof(isk::PlanHeader));
+  cudaMemset(s->d_small_ctr, 0, 2 * sizeof(unsigned int));
   const int nf = c.head_dim / 2;
   isk::inv_freq_kernel<<<(nf + 127) / 128, 128>>>(
       s->d_inv_freq, c.head_dim, c.rope_theta, c.rope_scaling, c.scale_factor, c.low_freq_factor,
@@ -1146,12 +1151,10 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.desc = s->ws_desc;
   pa.hdr = s->ws_hdr;
   pa.st = s->d_status;
-  // The single kernel saves the plan launch but schedules its units
-  // statically: it wins while a batch is short (measured on B200, Llama-3.1
-  // shapes: 16.3 vs 21.6 us for 152 tokens, level at ~4 000 tokens, 2% slower
-  // at 8 000), so it takes batches whose ids cannot total more than
-  // kSmallTokens tokens (ids x the longest fact; this also keeps its 32-bit
-  // sums from wrapping).
+  // The single kernel saves the plan launch (and the inject kernel's reads
+  // of the plan); its units come from a counter like the inject kernel's.
+  // It takes batches of up to small_limit requests and kSmallIds ids whose
+  // 32-bit sums cannot wrap (ids x the longest fact below 2^31).
   const int64_t longest = view ? s->shard_max_len : s->max_len;
   const bool small = R <= s->small_limit && num_ids <= isk::kSmallIds &&
                      int64_t(num_ids) * longest <= kSmallTokens;
@@ -1209,7 +1212,8 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
                    : pick_inject(cf.head_dim, cf.rope_style, cf.num_kv_heads, c.block_size, per_slot, loop);
   int32_t small_R = R, small_ids = num_ids, small_grid = s->small_grid, small_blocks = s->max_blocks;
   int64_t small_cap = slot_cap;
-  void* small_args[] = {&ia, &small_R, &small_ids, &small_cap, &small_grid, &small_blocks};
+  unsigned int* small_ctr = s->d_small_ctr;
+  void* small_args[] = {&ia, &small_R, &small_ids, &small_cap, &small_grid, &small_blocks, &small_ctr};
   void* args[] = {&ia};
   TimedLaunch* ev = nullptr;
   if (s->timing && s->events_used < size_t(kMaxTimedLaunches)) {

@@ -252,7 +252,8 @@ class FactStore:
         return B.is_last_error_timeout(self.handle, stream, timeout_ms)
 
     def set_small_batch_limit(self, max_requests: int) -> None:
-        """Batches up to max_requests (<= 8) requests run as one kernel; 0: never."""
+        """Batches up to max_requests (<= 32) requests and 256 ids run as one
+        kernel; 0: never."""
         B.is_store_set_small_batch_limit(self.handle, max_requests)
 
     def set_timing(self, enable: bool) -> None:

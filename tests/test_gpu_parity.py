@@ -477,6 +477,41 @@ def test_llama_single_request_block_counts(nblk, path):
     assert_parity(oracle_run(wl), gpu_run(wl, path=path))
 
 
+def test_single_kernel_takes_units_from_its_counter_back_to_back():
+    """The single kernel past one wave: 32 requests and up to 256 ids with
+    more work units than a 296-CTA grid holds, so CTAs take units from the
+    store's counter, which the last CTA out sets back to zero.  Three such
+    batches queued back to back on one stream (each needs the counter at
+    zero) all give the oracle's cache."""
+    _need_gpu()
+    model = synth.Model("l4h8", 4, 8, 128, 5e5, llama3=True)
+    base = _ragged(model, seed=41, R=32, max_k=8, lens=(8, 40), num_facts=64)
+    wls = []
+    for i in range(3):
+        rng = np.random.default_rng(100 + i)
+        ids = [rng.choice(64, int(rng.integers(4, 9)), replace=False) for _ in range(32)]
+        sp = rng.integers(0, 70, 32).astype(np.int32)
+        need = max(-(-(int(sp[r]) + int(base.fact_lens[ids[r]].sum())) // 16) for r in range(32)) + 2
+        b = synth.make_batch(rng, ids, sp, 16, 32 * need, need)
+        wl = synth.Workload("dyn", model, base.fact_lens, b, base.seed)
+        blocks = sum(-(-(int(sp[r]) + int(base.fact_lens[ids[r]].sum())) // 16) - int(sp[r]) // 16
+                     for r in range(32))
+        assert len(b.fact_ids) <= 256 and blocks * model.num_layers > 2 * 296
+        wls.append(wl)
+    store = make_store(base)
+    runs = []
+    for wl in wls:
+        k, v, desc = make_cache(wl)
+        ro, ids, sp, bt = batch_tensors(wl.batch)
+        slots = torch.full((wl.tokens(),), -7, dtype=torch.int64, device="cuda")
+        store.inject(ro, ids, sp, bt, desc, slots)
+        runs.append((k, v, slots, (ro, ids, sp, bt)))
+    rc, _ = store.last_error()
+    for wl, (k, v, slots, _) in zip(wls, runs):
+        assert_parity(oracle_run(wl), (rc, slots.cpu().numpy(), to_bits(k), to_bits(v)))
+    store.close()
+
+
 def test_head_sharded_stores_reproduce_the_full_cache():
     """KV-head shards (the multi-GPU tensor-parallel partition): a store and
     cache holding heads [h0, h1) only, fed the whole batch, produce exactly
