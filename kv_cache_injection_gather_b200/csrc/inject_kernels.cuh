@@ -1227,13 +1227,19 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
   const int total_blocks = a.hdr->total_blocks;
   const int rpu = a.hdr->rows_per_unit;
 
-  int next = 0;
-  if (tid == 0) next = int(atomicAdd(&a.hdr->next_unit, 1u));
+  // Unit blockIdx.x first (no CTA waits on the counter to start), then
+  // gridDim.x + the counter's answer, fetched one unit ahead.
+  int next = blockIdx.x;
+  unsigned int fetched = ~0u;
   for (;;) {
     __syncthreads();  // the previous unit's tables are no longer read
     if (tid == 0) {
+      if (fetched != ~0u) {
+        next = fetched < unsigned(total_units) - gridDim.x ? int(gridDim.x + fetched) : total_units;
+        fetched = ~0u;
+      }
       s_unit = next;
-      if (next < total_units) next = int(atomicAdd(&a.hdr->next_unit, 1u));
+      if (next < total_units) fetched = atomicAdd(&a.hdr->next_unit, 1u);
     }
     __syncthreads();
     const int u = s_unit;
@@ -1254,13 +1260,16 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
 // one kernel.  Every CTA of the persistent grid composes the batch itself in
 // shared memory -- the same definitions as plan_kernel (CSR check, lengths,
 // segment offsets, validity, token and block prefixes, work-unit size) --
-// and takes unit blockIdx.x, then units gridDim.x, gridDim.x + 1, ... from
-// a counter (dynamic, as the inject kernel).  The counter pair (next unit,
-// CTAs done) is the store's and starts at zero: the last CTA to leave, when
-// no CTA takes units any more, sets both back to zero for the next batch
-// (batches on one store run one at a time).  The last CTA (the one a small
-// batch leaves without units) alone records the batch's errors and writes
-// the -1 slots of invalid requests.  No work space, no second launch.
+// and takes unit blockIdx.x, then, when the batch has more than two waves
+// of units, units gridDim.x, gridDim.x + 1, ... from the store's counter
+// (dynamic, as the inject kernel; up to two waves, blockIdx.x + gridDim.x).  The counter is zero when a launch
+// starts and is fetched exactly once per unit (each unit a CTA takes makes
+// it fetch the next; the fetch after a CTA's last unit returns one past the
+// end), so the fetch that returns total_units - 1 is the launch's last and
+// its CTA sets the counter back to zero (batches on one store run one at a
+// time).  The last CTA (the one a small batch leaves without units) alone
+// records the batch's errors and writes the -1 slots of invalid requests.
+// No work space, no second launch.
 constexpr int kSmallRequests = 32;  // one lane of a warp per request
 constexpr int kSmallIds = 256;      // one thread per fact id
 
@@ -1276,6 +1285,7 @@ struct SmallPlan {
   int32_t nblk[kSmallRequests];
   int32_t blk0[kSmallRequests + 1];
   int32_t total_units, total_blocks, rpu;
+  int32_t over;  // over a capacity: the batch writes nothing
 };
 
 template <int D, int STYLE, int NT, int VPT, int MINB, bool POW2, bool HOST_TIER, int HC = 0, int BC = 0,
@@ -1295,17 +1305,6 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   static_assert(kSmallRequests <= 32, "request bit mask and warp-0 lanes");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool reporter = blockIdx.x == gridDim.x - 1;
-  // Leaving: count this CTA out; the last one resets the unit counter (no
-  // CTA takes a unit after it has counted itself out).
-  auto leave = [&]() {
-    if (tid == 0) {
-      __threadfence();
-      if (atomicAdd(&ctr[1], 1u) == gridDim.x - 1) {
-        atomicExch(&ctr[0], 0u);
-        atomicExch(&ctr[1], 0u);
-      }
-    }
-  };
 
   // Everything the plan reads from the caller is loaded at once: the CSR,
   // the starts, the ids and right behind them their lengths and store
@@ -1367,7 +1366,6 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   if (lane == 31) s_wsum[warp] = x;
   if (__syncthreads_or(csr_bad)) {
     if (reporter && tid == 0) record_error(a.st, kErrInvalidArg, -1);
-    leave();
     return;
   }
   int32_t ws = lane < NT / 32 ? s_wsum[lane] : 0;
@@ -1408,12 +1406,16 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
       const int32_t total_tokens = p.pref[num_ids];
       // the same limits as the two-kernel path, so results never depend on
       // which path a batch takes
-      const bool over = (a.slot_out != nullptr && total_tokens > slot_cap) || total > max_batch_blocks;
       int32_t rpu, upb;
       unit_size(total, a.L, a.H, grid_ctas, FAST != 0, rpu, upb);
+      // (work units are counted in 32 bits: a batch needing more is over
+      // capacity, as in the two-kernel path)
+      const bool over = (a.slot_out != nullptr && total_tokens > slot_cap) || total > max_batch_blocks ||
+                        (long long)total * upb > 0x7fffffffLL;
       p.rpu = rpu;
       p.total_blocks = total;
       p.total_units = over ? 0 : total * upb;
+      p.over = over;
       // A batch over capacity writes nothing and reports only that.
       if (reporter && over) record_error(a.st, kErrCapacity, total_tokens);
       s_err_key = ~0ull;
@@ -1423,8 +1425,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   if (tid < num_ids) p.seg[tid] = p.pref[tid] - p.pref[p.roff[myr]];
   __syncthreads();
   // -1 slots for the tokens of invalid requests (nothing at all on capacity).
-  const bool over_cap =
-      (a.slot_out != nullptr && p.pref[num_ids] > slot_cap) || p.blk0[R] > max_batch_blocks;
+  const bool over_cap = p.over != 0;
   if (reporter && a.slot_out && !over_cap) {
     for (int r = 0; r < R; ++r) {
       if (p.err[r] == kOk) continue;
@@ -1453,12 +1454,24 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   }
 
   const int total_units = p.total_units, total_blocks = p.total_blocks, rpu = p.rpu;
+  // Up to two waves the units are strided (u, u + gridDim.x: as balanced as
+  // the counter, without 296 CTAs' atomics on one word); beyond, counted.
+  const bool counted = total_units > 2 * int(gridDim.x);
   int next = blockIdx.x;  // the first wave is static
+  unsigned int fetched = ~0u;  // the counter's answer for the next unit, read one unit later
   for (;;) {
     __syncthreads();  // the previous unit's tables (and s_unit) are no longer read
     if (tid == 0) {
+      if (fetched != ~0u) {
+        if (fetched == unsigned(total_units) - 1u) atomicExch(ctr, 0u);  // the launch's last fetch
+        next = fetched < unsigned(total_units) - gridDim.x ? int(gridDim.x + fetched) : total_units;
+        fetched = ~0u;
+      }
       s_unit = next;
-      if (next < total_units) next = int(gridDim.x + atomicAdd(&ctr[0], 1u));
+      if (next < total_units) {
+        if (counted) fetched = atomicAdd(ctr, 1u);
+        else next += gridDim.x;
+      }
     }
     __syncthreads();
     const int u = s_unit;
@@ -1479,7 +1492,6 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
                                                  p.pref[j1] - p.pref[j0], p.pref[j0], w0,
                                                  min(a.L * a.H, w0 + rpu), lg == 0, p.fid, p.off);
   }
-  leave();
 }
 
 // Host tier, least-recently-used hot set: copy newly promoted facts from the

@@ -478,25 +478,27 @@ def test_llama_single_request_block_counts(nblk, path):
 
 
 def test_single_kernel_takes_units_from_its_counter_back_to_back():
-    """The single kernel past one wave: 32 requests and up to 256 ids with
-    more work units than a 296-CTA grid holds, so CTAs take units from the
-    store's counter, which the last CTA out sets back to zero.  Three such
-    batches queued back to back on one stream (each needs the counter at
-    zero) all give the oracle's cache."""
+    """The single kernel past two waves: 32 requests and up to 256 ids with
+    more than twice the work units a 296-CTA grid holds, so CTAs take units
+    from the store's counter, which the launch's last fetch sets back to
+    zero.  Three such batches queued back to back on one stream (each needs
+    the counter at zero) all give the oracle's cache."""
+    from test_unit_sizing_model import unit_size
     _need_gpu()
     model = synth.Model("l4h8", 4, 8, 128, 5e5, llama3=True)
     base = _ragged(model, seed=41, R=32, max_k=8, lens=(8, 40), num_facts=64)
     wls = []
     for i in range(3):
         rng = np.random.default_rng(100 + i)
-        ids = [rng.choice(64, int(rng.integers(4, 9)), replace=False) for _ in range(32)]
+        ids = [rng.choice(64, int(rng.integers(6, 9)), replace=False) for _ in range(32)]
         sp = rng.integers(0, 70, 32).astype(np.int32)
         need = max(-(-(int(sp[r]) + int(base.fact_lens[ids[r]].sum())) // 16) for r in range(32)) + 2
         b = synth.make_batch(rng, ids, sp, 16, 32 * need, need)
         wl = synth.Workload("dyn", model, base.fact_lens, b, base.seed)
         blocks = sum(-(-(int(sp[r]) + int(base.fact_lens[ids[r]].sum())) // 16) - int(sp[r]) // 16
                      for r in range(32))
-        assert len(b.fact_ids) <= 256 and blocks * model.num_layers > 2 * 296
+        upb = unit_size(blocks, model.num_layers, model.num_kv_heads, 296, True)[1]
+        assert len(b.fact_ids) <= 256 and blocks * upb > 2 * 296
         wls.append(wl)
     store = make_store(base)
     runs = []
