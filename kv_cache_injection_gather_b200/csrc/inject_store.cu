@@ -151,7 +151,7 @@ struct is_store {
   // kernel configuration
   int inject_grid = 0;
   int small_grid = 0;        // resident CTAs of the single-kernel path
-  unsigned int* d_small_ctr = nullptr;  // its unit counter pair (zero between batches)
+  unsigned int* d_small_ctr = nullptr;  // its unit counter (zero between batches)
   int32_t small_limit = isk::kSmallRequests;  // batches up to this many requests: one kernel
 };
 
@@ -519,7 +519,7 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
             dalloc(&s->ws_err, size_t(s->max_req)) == cudaSuccess &&
             dalloc(&s->ws_desc, size_t(s->max_blocks)) == cudaSuccess &&
             dalloc(&s->ws_hdr, 1) == cudaSuccess && dalloc(&s->d_status, 1) == cudaSuccess &&
-            dalloc(&s->d_small_ctr, 2) == cudaSuccess;
+            dalloc(&s->d_small_ctr, 1) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     free_store(s);
@@ -531,7 +531,7 @@ int is_store_create(const is_store_config_t* cfg, int device, is_store_t** out) 
   cudaMemset(s->d_off, 0, sizeof(int64_t) * size_t(c.max_facts));
   cudaMemset(s->d_status, 0, sizeof(isk::DevStatus));
   cudaMemset(s->ws_hdr, 0, sizeof(isk::PlanHeader));
-  cudaMemset(s->d_small_ctr, 0, 2 * sizeof(unsigned int));
+  cudaMemset(s->d_small_ctr, 0, sizeof(unsigned int));
   const int nf = c.head_dim / 2;
   isk::inv_freq_kernel<<<(nf + 127) / 128, 128>>>(
       s->d_inv_freq, c.head_dim, c.rope_theta, c.rope_scaling, c.scale_factor, c.low_freq_factor,
