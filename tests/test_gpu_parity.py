@@ -514,6 +514,49 @@ def test_single_kernel_takes_units_from_its_counter_back_to_back():
     store.close()
 
 
+def test_single_kernel_counter_across_batches_with_errors():
+    """The single kernel's counter through batches with errors: past two
+    waves, a batch with a block-table entry outside the cache in request 5
+    (those units are taken and skip their stores) and an id outside the
+    store in request 9 (its blocks make no units); then a batch whose CSR
+    does not end at the id count (rejected before any unit); then a clean
+    batch past two waves.  Each gives the oracle's status and cache."""
+    from test_unit_sizing_model import unit_size
+    _need_gpu()
+    model = synth.Model("l4h8", 4, 8, 128, 5e5, llama3=True)
+    base = _ragged(model, seed=41, R=32, max_k=8, lens=(8, 40), num_facts=64)
+
+    def batch(seed, skip=()):
+        rng = np.random.default_rng(seed)
+        ids = [rng.choice(64, int(rng.integers(6, 9)), replace=False) for _ in range(32)]
+        sp = rng.integers(0, 70, 32).astype(np.int32)
+        span = [-(-(int(sp[r]) + int(base.fact_lens[ids[r]].sum())) // 16) for r in range(32)]
+        b = synth.make_batch(rng, ids, sp, 16, 32 * (max(span) + 2), max(span) + 2)
+        blocks = sum(span[r] - int(sp[r]) // 16 for r in range(32) if r not in skip)
+        upb = unit_size(blocks, model.num_layers, model.num_kv_heads, 296, True)[1]
+        assert len(b.fact_ids) <= 256 and blocks * upb > 2 * 296
+        return b
+
+    b = batch(200, skip=(9,))
+    bt = b.block_tables.copy()
+    bt[5, int(b.start_pos[5]) // 16 + 1] = b.num_blocks + 3
+    fids = b.fact_ids.copy()
+    fids[b.req_offsets[9]] = 9999
+    b1 = synth.Batch(b.req_offsets, fids, b.start_pos, bt, 16, b.num_blocks)
+    b = batch(201)
+    ro = b.req_offsets.copy()
+    ro[-1] -= 1
+    b2 = synth.Batch(ro, b.fact_ids, b.start_pos, b.block_tables, 16, b.num_blocks)
+    b3 = batch(202)
+    store = make_store(base)
+    for bb, code in ((b1, oracle.ERR_BAD_BLOCK), (b2, oracle.ERR_INVALID_ARG), (b3, oracle.OK)):
+        wl = synth.Workload("dyn-err", model, base.fact_lens, bb, base.seed)
+        o = oracle_run(wl)
+        assert o[0] == code
+        assert_parity(o, gpu_run(wl, store=store))
+    store.close()
+
+
 def test_head_sharded_stores_reproduce_the_full_cache():
     """KV-head shards (the multi-GPU tensor-parallel partition): a store and
     cache holding heads [h0, h1) only, fed the whole batch, produce exactly
