@@ -1324,8 +1324,9 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   }
   if (tid == 0) s_bad_ids = 0u;
   // Block size: a shift when it is a power of two.  The plan's sums fit 32
-  // bits: the batch's ids total at most kSmallTokens tokens (the host's
-  // bound), and start + segment <= max_blocks * B < 2^31 once checked.
+  // bits: the host launches this kernel only when ids x the store's longest
+  // fact is below 2^31, and start + segment <= max_blocks * B < 2^31 once
+  // checked.
   const int lb = POW2 ? ilog2(a.B) : 0;
   auto div_b = [&](int32_t x) { return POW2 ? (x >> lb) : x / a.B; };
   __syncthreads();

@@ -46,8 +46,8 @@ constexpr int kSmallMinBlocks = IS_SMALL_MIN_BLOCKS;
 constexpr int kDefaultMaxRequests = 4096;
 constexpr int kDefaultMaxFactIds = 1 << 20;
 constexpr int kMaxTimedLaunches = 4096;
-// single-kernel path: ids x longest fact below 2^31 (its sums are 32-bit)
-constexpr int64_t kSmallTokens = (int64_t(1) << 31) - 1;
+// single-kernel path: ids x the longest fact at most this (its sums are 32-bit)
+constexpr int64_t kSmallSumLimit = (int64_t(1) << 31) - 1;
 
 struct TimedLaunch {
   cudaEvent_t start, stop;
@@ -1157,7 +1157,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   // 32-bit sums cannot wrap (ids x the longest fact below 2^31).
   const int64_t longest = view ? s->shard_max_len : s->max_len;
   const bool small = R <= s->small_limit && num_ids <= isk::kSmallIds &&
-                     int64_t(num_ids) * longest <= kSmallTokens;
+                     int64_t(num_ids) * longest <= kSmallSumLimit;
   if (!small) {
     if (R <= isk::kPlanSmemRequests && num_ids <= isk::kPlanSmemIds)
       isk::plan_kernel<kPlanThreads, true><<<1, kPlanThreads, isk::plan_smem_bytes(R, num_ids), st>>>(pa);
