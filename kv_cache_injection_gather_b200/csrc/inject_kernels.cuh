@@ -92,6 +92,16 @@ __device__ __forceinline__ void record_error(DevStatus* st, int32_t code, long l
   if (atomicCAS(&st->code, 0, code) == 0) st->detail = detail;
 }
 
+// The status once the batch's errors are recorded (by the thread that
+// records them), copied to m when set: pinned host memory mapped for the
+// device, which the host entry point reads after its wait instead of
+// copying the status back.
+__device__ __forceinline__ void mirror_status(const DevStatus* st, DevStatus* m) {
+  if (m == nullptr) return;
+  m->detail = __ldcg(&st->detail);
+  m->code = __ldcg(&st->code);
+}
+
 // ---------------------------------------------------------------- plan kernel
 
 // Work-unit size: rows per unit rpu and units per block upb, where a row is
@@ -177,6 +187,7 @@ struct PlanArgs {
   BlockDesc* desc;           // [max_batch_blocks]
   PlanHeader* hdr;
   DevStatus* st;
+  DevStatus* st_mirror;      // optional: see mirror_status
 };
 
 // Shared-memory plan: batches of at most kPlanSmemRequests requests and
@@ -253,6 +264,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
   __syncthreads();
   if (tid == 0 && s_bad) {
     record_error(a.st, kErrInvalidArg, -1);
+    mirror_status(a.st, a.st_mirror);
     a.hdr->total_blocks = 0;
     a.hdr->total_units = 0;
     a.hdr->units_per_block = 1;
@@ -407,7 +419,10 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     a.hdr->next_unit = 0;
     a.hdr->total_units = over ? 0 : total_blocks * upb;
     // A batch over capacity writes nothing and reports only that.
-    if (over) record_error(a.st, kErrCapacity, total_tokens);
+    if (over) {
+      record_error(a.st, kErrCapacity, total_tokens);
+      mirror_status(a.st, a.st_mirror);
+    }
   }
   __syncthreads();
   if (over_slots || over_blocks || s_over_units) return;
@@ -502,6 +517,7 @@ __global__ void __launch_bounds__(NT) plan_kernel(PlanArgs a) {
     if (req_err[r] != kOk) record_error(a.st, req_err[r], r);
     else record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
   }
+  if (tid == 0) mirror_status(a.st, a.st_mirror);
 }
 
 // -------------------------------------------------------------- inject kernel
@@ -531,6 +547,7 @@ struct InjectArgs {
   const BlockDesc* desc;
   PlanHeader* hdr;
   DevStatus* st;
+  DevStatus* st_mirror;      // optional: see mirror_status
   // host tier only: the arenas above are device-mapped pinned host memory,
   // and facts with hot_off[f] >= 0 are also held in these HBM arenas
   const uint16_t* k_hot;     // [L][H][hot_cap][D]
@@ -1366,7 +1383,10 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
   }
   if (lane == 31) s_wsum[warp] = x;
   if (__syncthreads_or(csr_bad)) {
-    if (reporter && tid == 0) record_error(a.st, kErrInvalidArg, -1);
+    if (reporter && tid == 0) {
+      record_error(a.st, kErrInvalidArg, -1);
+      mirror_status(a.st, a.st_mirror);
+    }
     return;
   }
   int32_t ws = lane < NT / 32 ? s_wsum[lane] : 0;
@@ -1453,6 +1473,7 @@ __global__ void __launch_bounds__(NT, MINB) small_inject_kernel(InjectArgs a, in
       else record_error(a.st, kErrBadBlock, (long long)r * a.max_blocks + b);
     }
   }
+  if (reporter && tid == 0) mirror_status(a.st, a.st_mirror);  // the batch's errors are in
 
   const int total_units = p.total_units, total_blocks = p.total_blocks, rpu = p.rpu;
   // Up to two waves the units are strided (u, u + gridDim.x: as balanced as

@@ -130,7 +130,9 @@ struct is_store {
   int32_t* stage = nullptr;
   size_t stage_elems = 0;
   int32_t* host_stage = nullptr;   // pinned mirror of `stage`
-  isk::DevStatus* host_status = nullptr;  // pinned
+  isk::DevStatus* host_status = nullptr;  // pinned, mapped
+  isk::DevStatus* host_status_dev = nullptr;  // its device address
+  isk::DevStatus* batch_mirror = nullptr;     // set while the host entry point runs a batch
   int64_t* stage_slots = nullptr;
   int64_t stage_slot_elems = 0;
   // timing
@@ -358,9 +360,16 @@ int grow_stage(is_store* s, size_t elems, int64_t slot_elems) {
       return IS_ERR_OOM;
     s->stage_elems = elems;
   }
-  if (!s->host_status && cudaHostAlloc(reinterpret_cast<void**>(&s->host_status), sizeof(isk::DevStatus),
-                                       cudaHostAllocDefault) != cudaSuccess)
-    return IS_ERR_OOM;
+  if (!s->host_status) {
+    if (cudaHostAlloc(reinterpret_cast<void**>(&s->host_status), sizeof(isk::DevStatus),
+                      cudaHostAllocMapped) != cudaSuccess)
+      return IS_ERR_OOM;
+    if (cudaHostGetDevicePointer(reinterpret_cast<void**>(&s->host_status_dev), s->host_status, 0) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      s->host_status_dev = nullptr;  // not mapped: the status is copied back instead
+    }
+  }
   if (slot_elems > s->stage_slot_elems) {
     cudaFree(s->stage_slots);
     s->stage_slots = nullptr;
@@ -1151,6 +1160,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   pa.desc = s->ws_desc;
   pa.hdr = s->ws_hdr;
   pa.st = s->d_status;
+  pa.st_mirror = s->batch_mirror;
   // The single kernel saves the plan launch (and the inject kernel's reads
   // of the plan); its units come from a counter like the inject kernel's.
   // It takes batches of up to small_limit requests and kSmallIds ids whose
@@ -1205,6 +1215,7 @@ int is_inject_batch(is_store_t* s, int32_t R, const int32_t* req_off, const int3
   ia.desc = s->ws_desc;
   ia.hdr = s->ws_hdr;
   ia.st = s->d_status;
+  ia.st_mirror = s->batch_mirror;
   ia.fact_len_count = nfacts;
   // Per-slot sources: the host tier, or the arenas of a sharded view.
   const bool per_slot = s->host_arena || view;
@@ -1295,8 +1306,15 @@ static int host_batch(is_store_t* s, int32_t R, const int32_t* req_off, const in
     return IS_ERR_CUDA;
   }
   s->batch_pend = s->pend_np > 0;
+  // The kernel that records the batch's errors also writes the status into
+  // the mapped pinned copy: no copy back after the batch.  (A value it did
+  // not write is seen as the marker, and the status is then copied.)
+  constexpr int32_t kUnwritten = INT32_MIN;
+  s->host_status->code = kUnwritten;
+  s->batch_mirror = s->host_status_dev;
   rc = is_inject_batch(s, R, d_off, d_ids, num_ids, d_sp, d_bt, max_blocks_per_req, cache,
                        direct_slots ? direct_slots : slot_out ? s->stage_slots : nullptr, slot_cap, stream);
+  s->batch_mirror = nullptr;
   s->batch_pend = false;
   if (rc != IS_OK) {
     lru_finish(s, st, false);  // nothing ran: copy the promoted facts instead
@@ -1309,10 +1327,15 @@ static int host_batch(is_store_t* s, int32_t R, const int32_t* req_off, const in
   bool copied = !(slot_out && slot_cap > 0) || direct_slots ||
                 cudaMemcpyAsync(slot_out, s->stage_slots, size_t(slot_cap) * 8, cudaMemcpyDeviceToHost,
                                 st) == cudaSuccess;
-  // Status back in the same stream, then one wait.
-  copied = copied && cudaMemcpyAsync(s->host_status, s->d_status, sizeof(isk::DevStatus),
-                                     cudaMemcpyDeviceToHost, st) == cudaSuccess;
-  const bool waited = cudaStreamSynchronize(st) == cudaSuccess;
+  // One wait; the status is already on its way to the pinned copy.
+  const bool mirrored = s->host_status_dev != nullptr;
+  if (!mirrored)
+    copied = copied && cudaMemcpyAsync(s->host_status, s->d_status, sizeof(isk::DevStatus),
+                                       cudaMemcpyDeviceToHost, st) == cudaSuccess;
+  bool waited = cudaStreamSynchronize(st) == cudaSuccess;
+  if (copied && waited && s->host_status->code == kUnwritten)
+    waited = cudaMemcpy(s->host_status, s->d_status, sizeof(isk::DevStatus), cudaMemcpyDeviceToHost) ==
+             cudaSuccess;
   const int code = (copied && waited) ? s->host_status->code : IS_ERR_CUDA;
   if (s->pend_np > 0 && (lru_finish(s, st, code == 0) != IS_OK || cudaStreamSynchronize(st) != cudaSuccess))
     return IS_ERR_CUDA;
@@ -1572,6 +1595,7 @@ extern "C" int is_inject_batch_noalloc(const is_store_config_t* cfg, const void*
   pa.desc = reinterpret_cast<isk::BlockDesc*>(ws + kNaDesc);
   pa.hdr = hdr;
   pa.st = status;
+  pa.st_mirror = nullptr;
   isk::plan_kernel<kPlanThreads, false><<<1, kPlanThreads, 0, st>>>(pa);
 
   isk::InjectArgs ia{};

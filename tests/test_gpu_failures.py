@@ -66,20 +66,38 @@ def test_device_status_is_cleared_after_reading():
     store.close()
 
 
-def test_host_entry_point_reports_device_errors():
+@pytest.mark.parametrize("small_limit", [None, 0], ids=["single-kernel", "two-kernel"])
+def test_host_entry_point_reports_device_errors(small_limit):
+    """The host entry point returns the status the batch's kernels recorded
+    (they also write it into the store's mapped pinned copy): a bad block,
+    a malformed CSR, slot capacity, an error left by an earlier asynchronous
+    batch on the store (then cleared), and OK."""
     _need_gpu()
     wl = synth.tiny(0)
-    store = make_store(wl)
+    store = make_store(wl, small_limit=small_limit)
     k, v, desc = make_cache(wl)
     b = wl.batch
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).pin_memory()  # noqa: E731
-    bt = b.block_tables.copy()
-    bt[0, 2] = 9999  # the first fact's tokens start at position 32: block 2
-    rc = store.inject_host(pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos), pin(bt), desc)
-    assert rc == B.IS_ERR_BAD_BLOCK
-    rc = store.inject_host(pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos),
-                           pin(b.block_tables), desc)
-    assert rc == B.IS_OK
+    ro, ids, sp, bt = pin(b.req_offsets), pin(b.fact_ids), pin(b.start_pos), pin(b.block_tables)
+    bad_bt = b.block_tables.copy()
+    bad_bt[0, 2] = 9999  # the first fact's tokens start at position 32: block 2
+    assert store.inject_host(ro, ids, sp, pin(bad_bt), desc) == B.IS_ERR_BAD_BLOCK
+    assert store.inject_host(ro, ids, sp, bt, desc) == B.IS_OK
+    bad_ro = b.req_offsets.copy()
+    bad_ro[-1] -= 1
+    assert store.inject_host(pin(bad_ro), ids, sp, bt, desc) == B.IS_ERR_INVALID_ARG
+    n_tok = wl.tokens()
+    short = torch.empty(n_tok - 1, dtype=torch.int64).pin_memory()
+    assert store.inject_host(ro, ids, sp, bt, desc, short) == B.IS_ERR_CAPACITY
+    # an asynchronous batch's error, not yet read, comes back with the next
+    # host-entry batch, which clears it
+    d_ro, d_ids, d_sp, d_bt = batch_tensors(b)
+    bad_ids = d_ids.clone()
+    bad_ids[0] = 9999
+    store.inject(d_ro, bad_ids, d_sp, d_bt, desc)
+    assert store.inject_host(ro, ids, sp, bt, desc) == B.IS_ERR_BAD_FACT_ID
+    assert store.inject_host(ro, ids, sp, bt, desc) == B.IS_OK
+    assert store.last_error()[0] == B.IS_OK
     store.close()
 
 
