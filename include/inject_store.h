@@ -309,12 +309,14 @@ int is_inject_batch(is_store_t* store, int32_t num_requests, const int32_t* req_
  * memory.  Copies the arrays into store-owned device buffers, runs the
  * batch, waits for `stream` and returns the batch's status (host-side or
  * device-side, as for is_inject_batch + is_last_error).  The caches stay on
- * the device.  slot_mapping_out in page-locked memory mapped for the store's
- * device (cudaHostAlloc, cudaMallocHost, a mapped registration; the whole
- * slot_mapping_capacity entries) is written in place by the kernels, with
- * exactly the entries is_inject_batch writes; any other host buffer receives
- * all slot_mapping_capacity entries of a store-owned device buffer, whose
- * entries past the batch's tokens (all of them on CAPACITY) are stale. */
+ * the device.  On a device-tier store, slot_mapping_out in page-locked
+ * memory mapped for the store's device (cudaHostAlloc, cudaMallocHost, a
+ * mapped registration; the whole slot_mapping_capacity entries) is written
+ * in place by the kernels, with exactly the entries is_inject_batch writes;
+ * any other host buffer, and every buffer of a host-tier store (whose batch
+ * keeps the host link busy), receives all slot_mapping_capacity entries of a
+ * store-owned device buffer, whose entries past the batch's tokens (all of
+ * them on CAPACITY) are stale. */
 int is_inject_batch_host(is_store_t* store, int32_t num_requests,
                          const int32_t* req_fact_offsets, const int32_t* fact_ids,
                          int32_t num_fact_ids, const int32_t* start_pos,
