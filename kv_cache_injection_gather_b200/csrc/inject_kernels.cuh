@@ -1279,12 +1279,12 @@ __global__ void __launch_bounds__(NT, MINB) inject_kernel(InjectArgs a) {
 // segment offsets, validity, token and block prefixes, work-unit size) --
 // and takes unit blockIdx.x, then, when the batch has more than two waves
 // of units, units gridDim.x, gridDim.x + 1, ... from the store's counter
-// (dynamic, as the inject kernel; up to two waves, blockIdx.x + gridDim.x).  The counter is zero when a launch
-// starts and is fetched exactly once per unit (each unit a CTA takes makes
-// it fetch the next; the fetch after a CTA's last unit returns one past the
-// end), so the fetch that returns total_units - 1 is the launch's last and
-// its CTA sets the counter back to zero (batches on one store run one at a
-// time).  The last CTA (the one a small batch leaves without units) alone
+// (dynamic, as the inject kernel; up to two waves, blockIdx.x + gridDim.x).
+// The counter is zero when a launch starts and is fetched exactly once per
+// unit (each unit a CTA takes makes it fetch the next; the fetch after a
+// CTA's last unit returns one past the end), so the fetch that returns
+// total_units - 1 is the launch's last and its CTA sets the counter back to
+// zero (batches on one store run one at a time).  The last CTA (the one a small batch leaves without units) alone
 // records the batch's errors and writes the -1 slots of invalid requests.
 // No work space, no second launch.
 constexpr int kSmallRequests = 32;  // one lane of a warp per request
