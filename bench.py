@@ -336,6 +336,28 @@ def gpu_id(dev, local_rank: int) -> str:
         return str(local_rank)
 
 
+def launch_probe(dev, flush, reps: int = 200) -> float:
+    """Microseconds between two CUDA events around the smallest kernel (a
+    one-element fill), median of reps timed as the small batches are (each
+    after an L2 flush, which the GPU is still running when the events and
+    the kernel are queued, so no host time falls between them): the fixed
+    cost any single launch timed this way carries on this machine.  Context for
+    batches bound by latency, not their denominator."""
+    import torch
+    t = torch.zeros(1, device=dev)
+    pairs = []
+    for _ in range(reps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        t.fill_(1.0)
+        e1.record()
+        pairs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    return float(np.median([a.elapsed_time(b) * 1e3 for a, b in pairs]))
+
+
 def copy_probe(dev, elems: int = 1 << 30, reps: int = 10):
     """Device copy bandwidth on this machine now (read + write bytes / time): the
     best of reps single copies (the kind of figure the measured peak is) and
@@ -776,7 +798,7 @@ def run_ours(args, rank, world, local_rank):
     extra_cfg["cache_layout"] = "[L][num_blocks][H][B][D]" if args.head_major else "[L][num_blocks][B][H][D]"
     extra_cfg["path"] = ("single fused kernel" if single_kernel(
         b.num_requests, len(b.fact_ids), int(wl.fact_lens.max()), args.small_limit)
-        else "plan + inject kernels")
+        else "plan + inject kernels")  # the kernel the roofline times
     copy_ref, copy_sus = copy_probe(dev)
     # every rank takes part in the same collectives, in the same order
     peer_gbs = peer_probe(dev, world) if (owner is not None and world > 1) else None
@@ -859,6 +881,7 @@ def run_ours(args, rank, world, local_rank):
     algo_bytes = n_tok * 2 * m.bytes_per_token   # read K+V + write K+V
     peak, peak_kind = hbm_peak()
     achieved = algo_bytes / (kern_avg_ms / 1e3) / 1e9
+    single = single_kernel(b.num_requests, len(b.fact_ids), int(wl.fact_lens.max()), args.small_limit)
     traffic_pt, rec = recorded_traffic()
     if args.workload != "llama-batch" or args.head_major or owner is not None:
         traffic_pt = None  # the committed counters are for the benchmark workload
@@ -869,7 +892,11 @@ def run_ours(args, rank, world, local_rank):
                 "frac_of_same_box_sustained_copy": achieved / copy_sus,
                 "traffic": None if traffic_pt is None else traffic_pt * n_tok,
                 "algorithmic_bytes": algo_bytes,
-                "kernel": "inject_kernel (plan_kernel excluded)"}
+                "kernel": ("small_inject_kernel (its in-kernel plan included)" if single else
+                           "inject_kernel (plan_kernel excluded)")}
+    if flush is not None:
+        # a batch this small is timed alone: what an empty kernel costs so
+        roofline["empty_kernel_us"] = launch_probe(dev, flush)
     if owner is not None and world > 1:
         # Peer reads: rows of facts other ranks own cross NVLink once; the
         # bound is those bytes at the peer bandwidth measured in this run.
