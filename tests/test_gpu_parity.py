@@ -17,6 +17,8 @@ the N(0, 1) inputs.
 """
 from __future__ import annotations
 
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -84,12 +86,21 @@ def _need_gpu():
 
 # ------------------------------------------------------------------ oracle side
 
-def oracle_run(wl: synth.Workload, style=0, head_major=False, slot_capacity=None):
-    m, b = wl.model, wl.batch
+def oracle_store(wl: synth.Workload):
+    """The oracle's store of every fact of wl (read-only for inject_batch,
+    so batches over the same facts may share it)."""
+    m = wl.model
     st = oracle.Store(m.num_layers, m.num_kv_heads, m.head_dim, max(int(wl.fact_lens.sum()), 1),
                       len(wl.fact_lens))
     for f, n in enumerate(wl.fact_lens):
         st.put(*synth.fact_kv(wl.seed, f, m.num_layers, m.num_kv_heads, int(n), m.head_dim))
+    return st
+
+
+def oracle_run(wl: synth.Workload, style=0, head_major=False, slot_capacity=None, st=None):
+    m, b = wl.model, wl.batch
+    if st is None:
+        st = oracle_store(wl)
     shape = ((m.num_layers, b.num_blocks, m.num_kv_heads, b.block_size, m.head_dim) if head_major
              else (m.num_layers, b.num_blocks, b.block_size, m.num_kv_heads, m.head_dim))
     kc = synth.bf16_block(CACHE_FILL_SEED, synth.TAG_CACHE | 0, shape)
@@ -460,6 +471,17 @@ def test_llama_single_request_full_store():
     assert_parity((rc, slots, kc, vc, kref), g)
 
 
+@functools.lru_cache(maxsize=None)
+def _block_count_case(nblk):
+    k = 5
+    T = 16 * nblk - 8
+    lens = np.array([T // k + (i < T % k) for i in range(k)], np.int32)
+    batch = synth.make_batch(np.random.default_rng(nblk), [np.arange(k)], 64, 16, 24, 24)
+    wl = synth.Workload("llama-blocks", synth.LLAMA31_8B, lens, batch, seed=nblk)
+    assert wl.tokens() == T
+    return wl, oracle_run(wl)
+
+
 @pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("nblk", [13, 15, 16, 17, 18])
 def test_llama_single_request_block_counts(nblk, path):
@@ -468,13 +490,9 @@ def test_llama_single_request_block_counts(nblk, path):
     batch this size, 15 to 17 blocks are where rounding the units' row ranges
     once gave more units than the 296-CTA grid; every count, on both paths,
     gives the oracle's cache."""
-    k = 5
-    T = 16 * nblk - 8
-    lens = np.array([T // k + (i < T % k) for i in range(k)], np.int32)
-    batch = synth.make_batch(np.random.default_rng(nblk), [np.arange(k)], 64, 16, 24, 24)
-    wl = synth.Workload("llama-blocks", synth.LLAMA31_8B, lens, batch, seed=nblk)
-    assert wl.tokens() == T
-    assert_parity(oracle_run(wl), gpu_run(wl, path=path))
+    _need_gpu()
+    wl, o = _block_count_case(nblk)  # the oracle's cache, shared by both paths
+    assert_parity(o, gpu_run(wl, path=path))
 
 
 def test_single_kernel_takes_units_from_its_counter_back_to_back():
@@ -554,6 +572,59 @@ def test_single_kernel_counter_across_batches_with_errors():
         o = oracle_run(wl)
         assert o[0] == code
         assert_parity(o, gpu_run(wl, store=store))
+    store.close()
+
+
+def test_single_kernel_random_stream_of_batches():
+    """Twelve seeded batches of 1..32 requests queued back to back on one
+    stream through the single kernel -- one wave or several, some with an id
+    outside the store, a block-table entry outside the cache or a CSR that
+    does not end at the id count -- each into its own cache: every cache is
+    the oracle's, and the status read once at the end is the first error in
+    stream order (each batch's own first error in request order)."""
+    _need_gpu()
+    model = synth.Model("l4h8", 4, 8, 128, 5e5, llama3=True)
+    base = _ragged(model, seed=43, R=32, max_k=8, lens=(4, 48), num_facts=64)
+    rng = np.random.default_rng(2024)
+    wls = []
+    for i in range(12):
+        R = int(rng.integers(1, 33))
+        kmax = int(rng.choice([2, 8]))
+        ids = [rng.choice(64, int(rng.integers(0, kmax + 1)), replace=False) for _ in range(R)]
+        sp = rng.integers(0, 100, R).astype(np.int32)
+        need = max(-(-(int(sp[r]) + int(base.fact_lens[ids[r]].sum())) // 16) for r in range(R)) + 1
+        b = synth.make_batch(rng, ids, sp, 16, R * need, need)
+        fids, bt, ro = b.fact_ids.copy(), b.block_tables.copy(), b.req_offsets.copy()
+        kind = rng.choice(["clean"] * 5 + ["bad_id", "bad_block", "csr"])
+        if kind == "bad_id" and len(fids):
+            fids[int(rng.integers(0, len(fids)))] = 64 + int(rng.integers(0, 5))
+        elif kind == "bad_block":
+            r = int(rng.integers(0, R))
+            bt[r, int(sp[r]) // 16] = -2
+        elif kind == "csr" and R > 1:
+            ro[-1] += 1
+        wls.append(synth.Workload("stream", model, base.fact_lens,
+                                  synth.Batch(ro, fids, sp, bt, 16, b.num_blocks), base.seed))
+    store = make_store(base)
+    runs = []
+    for wl in wls:
+        k, v, desc = make_cache(wl)
+        ro_t, ids_t, sp_t, bt_t = batch_tensors(wl.batch)
+        fids = wl.batch.fact_ids
+        n_tok = int(wl.fact_lens[fids[(fids >= 0) & (fids < 64)]].sum())
+        slots = torch.full((max(n_tok, 1),), -7, dtype=torch.int64, device="cuda")
+        store.inject(ro_t, ids_t, sp_t, bt_t, desc, slots[:n_tok])
+        runs.append((k, v, slots, n_tok, (ro_t, ids_t, sp_t, bt_t)))
+    rc, _ = store.last_error()
+    first = oracle.OK
+    ost = oracle_store(base)
+    for wl, (k, v, slots, n_tok, _) in zip(wls, runs):
+        o = oracle_run(wl, st=ost)
+        if first == oracle.OK:
+            first = o[0]
+        assert_parity((oracle.OK,) + tuple(o[1:]), (oracle.OK, slots[:n_tok].cpu().numpy(), to_bits(k),
+                                                    to_bits(v)))
+    assert rc == first
     store.close()
 
 
