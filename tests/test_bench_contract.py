@@ -87,3 +87,28 @@ def test_l2_flush_runs_on_any_device():
     f = bench.L2Flush("cpu")
     f()
     assert f.buf.numel() == 2 * bench.L2_BYTES and int(f.acc) == 0
+
+
+def test_launch_count_follows_the_library_path_choice():
+    """bench.py counts one kernel per step for a batch the library runs as its
+    single kernel and two (plan + inject) otherwise; its limits must be the
+    library's (the constants of the kernel header and the host's 32-bit sum
+    bound), and its rule the host's: requests <= limit, ids <= 256,
+    ids x the longest fact <= 2^31 - 1."""
+    import re
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = os.path.join(ROOT, "kv_cache_injection_gather_b200", "csrc")
+    hdr = open(os.path.join(csrc, "inject_kernels.cuh")).read()
+    host = open(os.path.join(csrc, "inject_store.cu")).read()
+    assert int(re.search(r"constexpr int kSmallRequests = (\d+);", hdr).group(1)) == bench.SMALL_REQUESTS
+    assert int(re.search(r"constexpr int kSmallIds = (\d+);", hdr).group(1)) == bench.SMALL_IDS
+    assert "kSmallSumLimit = (int64_t(1) << 31) - 1" in host
+    assert bench.single_kernel(1, 5, 64)
+    assert bench.single_kernel(32, 256, 96)
+    assert not bench.single_kernel(33, 5, 64)
+    assert not bench.single_kernel(1, 257, 64)
+    assert not bench.single_kernel(1, 256, 1 << 23)       # 2^31 tokens by the bound
+    assert bench.single_kernel(1, 255, 1 << 23)
+    assert not bench.single_kernel(4, 5, 64, limit=0)     # --small-limit 0
+    assert bench.single_kernel(8, 5, 64, limit=8) and not bench.single_kernel(9, 5, 64, limit=8)
