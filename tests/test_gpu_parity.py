@@ -527,8 +527,9 @@ def test_single_kernel_takes_units_from_its_counter_back_to_back():
         store.inject(ro, ids, sp, bt, desc, slots)
         runs.append((k, v, slots, (ro, ids, sp, bt)))
     rc, _ = store.last_error()
+    ost = oracle_store(base)
     for wl, (k, v, slots, _) in zip(wls, runs):
-        assert_parity(oracle_run(wl), (rc, slots.cpu().numpy(), to_bits(k), to_bits(v)))
+        assert_parity(oracle_run(wl, st=ost), (rc, slots.cpu().numpy(), to_bits(k), to_bits(v)))
     store.close()
 
 
@@ -567,9 +568,10 @@ def test_single_kernel_counter_across_batches_with_errors():
     b2 = synth.Batch(ro, b.fact_ids, b.start_pos, b.block_tables, 16, b.num_blocks)
     b3 = batch(202)
     store = make_store(base)
+    ost = oracle_store(base)
     for bb, code in ((b1, oracle.ERR_BAD_BLOCK), (b2, oracle.ERR_INVALID_ARG), (b3, oracle.OK)):
         wl = synth.Workload("dyn-err", model, base.fact_lens, bb, base.seed)
-        o = oracle_run(wl)
+        o = oracle_run(wl, st=ost)
         assert o[0] == code
         assert_parity(o, gpu_run(wl, store=store))
     store.close()
