@@ -394,9 +394,8 @@ const char* is_status_string(int status);
  *
  * Who needs it: code that runs where cudaMalloc is off limits -- inside a
  * serving engine whose memory pool already owns the whole GPU (a call to
- * cudaMalloc would fail or fragment the pool), in a region the engine is
- * recording into a CUDA graph, or in a plugin whose host may not create
- * allocations behind its back.  Such a caller cannot create an is_store_t
+ * cudaMalloc would fail or fragment the pool), or in a plugin whose host
+ * may not create allocations behind its back.  Such a caller cannot create an is_store_t
  * (creation allocates), so it passes the store's contents itself.
  *
  * The per-batch work space (segment offsets, per-request sums, block

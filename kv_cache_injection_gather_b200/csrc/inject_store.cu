@@ -1426,8 +1426,7 @@ int is_store_kernel_time(is_store_t* s, double* total_ms, int64_t* launches) {
 // Allocation-free entry point (is_inject_batch_noalloc).
 //
 // For callers that must not allocate device memory (an engine whose pool
-// owns the GPU, a region being captured into a CUDA graph, a plugin host
-// that forbids hidden allocations).  The per-batch work space is one fixed
+// owns the GPU, a plugin host that forbids hidden allocations).  The per-batch work space is one fixed
 // device array in this module; the same plan and inject kernels as
 // is_inject_batch run on it.
 // ===================================================================

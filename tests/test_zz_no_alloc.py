@@ -1,7 +1,6 @@
 """is_inject_batch_noalloc, the entry point for callers that cannot allocate
 device memory: an engine whose memory pool already owns the whole GPU, a
-region the engine is recording into a CUDA graph, a plugin whose host forbids
-allocations behind its back.  Such a caller hands over the store's arenas and
+plugin whose host forbids allocations behind its back.  Such a caller hands over the store's arenas and
 fact table as its own buffers; the per-batch work space is the library's
 fixed device array.
 
